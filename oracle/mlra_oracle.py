@@ -1,0 +1,152 @@
+"""CPU float64 oracle for MLRA single-token decode attention (step 2, absorbed form).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module.  It shares no code with
+the CUDA path and must never be used as a fallback for it.
+
+What it computes (sources: "Multi-Head Low-Rank Attention", yunpan.plus page):
+  * section 1.3, steps 1-3 of MLA's efficient decode: the absorbed query
+    ``q~`` is dotted with the cached latent vectors directly, as MQA-style
+    attention with the latent as the shared key/value, and the value
+    up-projection comes afterwards (step 3, not computed here);
+  * section 2: the per-head NoPE key is a sum of B block projections of the
+    latent, so splitting ``c_t`` into B column blocks ``c_{t,b}`` is exact;
+  * section 3 / 3.1 (MLRA-4): the block sum moves behind the attention; each
+    branch b runs its own attention over its block with its own softmax over
+    positions, and the RoPE key ``k^R_t`` is shared by all branches;
+  * section 3.3: the sum of the branch outputs is scaled (``gamma``).
+
+For sequence s, head h, branch b and position j < L_s (row(s, j) from the page
+table or the contiguous layout):
+
+    score[j] = sigma * ( q_lat[s,h,b-block] . c[row, b-block]  +  q_rope[s,h] . k_rope[row] )
+    p        = softmax over j of score          (independent per branch)
+    out[s,h,b-block] = gamma * sum_j p[j] * c[row, b-block]
+
+Readings where the pages are silent (each listed in the design doc): one RoPE query
+per head shared by all branches; ``sigma`` and ``gamma`` are parameters; the
+current token is already in the cache and no other mask applies; an empty
+sequence gives a zero output and ``lse = -inf``; ``lse = log sum_j exp(score_j)``
+per (s, h, b); "summed" output mode adds the B scaled branch outputs.
+
+Every function below is written in float64 with NumPy; matrix products use
+``numpy.matmul``.  Parity of the reconstructed MLRA-4 formula against the
+published paper is unpinned (the equation is missing from the pages); the
+oracle is pinned by the identities and closed forms in tests/test_oracle_pins.py.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = ["resolve_rows", "decode", "decode_heads", "branch_probabilities", "to_f64"]
+
+
+def to_f64(x) -> np.ndarray:
+    """Convert a tensor/array to a float64 NumPy array (exact for bf16 and fp32)."""
+    if hasattr(x, "detach"):
+        x = x.detach().cpu().double().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def resolve_rows(seq_len: int, s: int, page_table, page_size: int, max_seq_len: int) -> np.ndarray:
+    """Cache row of every position j < seq_len of sequence s.
+
+    Contiguous layout (no page table): row = s * max_seq_len + j.
+    Paged layout: row = page_table[s, j // P] * P + j % P.
+    """
+    j = np.arange(seq_len, dtype=np.int64)
+    if page_table is None:
+        return s * np.int64(max_seq_len) + j
+    pt = np.asarray(page_table, dtype=np.int64)
+    return pt[s, j // page_size] * page_size + j % page_size
+
+
+def _rope_scores(q_rope_s: np.ndarray, kr: np.ndarray) -> np.ndarray:
+    """Shared RoPE term q^R_h . k^R_j for all heads h and positions j: [H, L]."""
+    return q_rope_s @ kr.T
+
+
+def _branch_scores(q_blk: np.ndarray, c_blk: np.ndarray, rope: np.ndarray, sigma: float) -> np.ndarray:
+    """sigma * (q~_{h,b} . c_{j,b} + q^R_h . k^R_j): [H, L]."""
+    return sigma * (q_blk @ c_blk.T + rope)
+
+
+def _softmax_positions(scores: np.ndarray):
+    """Softmax over positions (last axis) with the row max subtracted; returns (p, lse)."""
+    m = scores.max(axis=-1, keepdims=True)
+    e = np.exp(scores - m)
+    z = e.sum(axis=-1, keepdims=True)
+    return e / z, (m + np.log(z))[..., 0]
+
+
+def _apply_probs(p: np.ndarray, c_blk: np.ndarray) -> np.ndarray:
+    """sum_j p[h, j] c_{j,b}: [H, d_blk]."""
+    return p @ c_blk
+
+
+def _gather(seq_len, s, c_kv, k_rope, page_table, page_size, max_seq_len):
+    rows = resolve_rows(seq_len, s, page_table, page_size, max_seq_len)
+    return c_kv[rows], k_rope[rows]
+
+
+def decode_heads(q_lat_s, q_rope_s, c_rows, kr_rows, num_branches, sigma, gamma,
+                 out_mode="branches", with_probs=False):
+    """Decode for one sequence whose cache rows are already gathered.
+
+    q_lat_s [H', d_c], q_rope_s [H', d_R] (any subset of heads), c_rows [L, d_c],
+    kr_rows [L, d_R].  Returns (out, lse[, probs]) with out [H', d_c] in
+    "branches" mode or [H', d_blk] in "summed" mode, lse [H', B] and, on request,
+    probs [B, H', L].
+    """
+    hq, d_c = q_lat_s.shape
+    B = num_branches
+    d = d_c // B
+    L = c_rows.shape[0]
+    if L == 0:
+        out = np.zeros((hq, d_c if out_mode == "branches" else d))
+        lse = np.full((hq, B), -np.inf)
+        return (out, lse, np.zeros((B, hq, 0))) if with_probs else (out, lse)
+    rope = _rope_scores(q_rope_s, kr_rows)
+    outs, lses, probs = [], [], []
+    for b in range(B):
+        cols = slice(b * d, (b + 1) * d)
+        scores = _branch_scores(q_lat_s[:, cols], c_rows[:, cols], rope, sigma)
+        p, lse = _softmax_positions(scores)
+        outs.append(gamma * _apply_probs(p, c_rows[:, cols]))
+        lses.append(lse)
+        probs.append(p)
+    out = np.concatenate(outs, axis=1) if out_mode == "branches" else np.sum(outs, axis=0)
+    lse = np.stack(lses, axis=1)
+    return (out, lse, np.stack(probs)) if with_probs else (out, lse)
+
+
+def decode(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table, num_branches, sigma, gamma,
+           page_size=0, max_seq_len=0, out_mode="branches", seqs=None, heads=None):
+    """Decode attention for a batch.
+
+    q_lat [N, H, d_c], q_rope [N, H, d_R], c_kv [rows, d_c], k_rope [rows, d_R],
+    seq_lens [N], page_table [N, max_pages] or None.  ``seqs`` / ``heads`` pick a
+    subset (default: all).  Returns (out [n, h, ...], lse [n, h, B]) in float64.
+    """
+    q_lat, q_rope = to_f64(q_lat), to_f64(q_rope)
+    c_kv, k_rope = to_f64(c_kv), to_f64(k_rope)
+    lens = np.asarray(seq_lens.tolist() if hasattr(seq_lens, "tolist") else seq_lens, dtype=np.int64)
+    pt = None if page_table is None else np.asarray(
+        page_table.tolist() if hasattr(page_table, "tolist") else page_table, dtype=np.int64)
+    seqs = range(q_lat.shape[0]) if seqs is None else seqs
+    heads = slice(None) if heads is None else heads
+    outs, lses = [], []
+    for s in seqs:
+        c_rows, kr_rows = _gather(int(lens[s]), s, c_kv, k_rope, pt, page_size, max_seq_len)
+        o, l = decode_heads(q_lat[s][heads], q_rope[s][heads], c_rows, kr_rows, num_branches,
+                            sigma, gamma, out_mode)
+        outs.append(o)
+        lses.append(l)
+    return np.stack(outs), np.stack(lses)
+
+
+def branch_probabilities(q_lat_s, q_rope_s, c_rows, kr_rows, num_branches, sigma):
+    """Attention weights p[b, h, j] of one sequence (for the sum-to-one checks)."""
+    _, _, probs = decode_heads(to_f64(q_lat_s), to_f64(q_rope_s), to_f64(c_rows), to_f64(kr_rows),
+                               num_branches, sigma, 1.0, with_probs=True)
+    return probs

@@ -1,0 +1,319 @@
+"""Checks that pin the CPU oracle to facts fixed outside of it.
+
+Each ``pin_*`` takes the oracle module (so that the same checks can be run
+against copies with a planted mistake, see test_oracle_mutants.py) and raises
+AssertionError when the oracle disagrees.  None of them retypes the oracle's
+formula: they compare it with an independent library routine (PyTorch's
+scaled-dot-product attention, SciPy's logsumexp), with pure-Python brute force,
+with closed forms, or with invariants.
+
+Sources ("Multi-Head Low-Rank Attention", yunpan.plus page):
+  * section 1.3: absorbed three-step decode equals attention with the
+    decompressed keys/values;
+  * section 2: the NoPE key is a sum of block projections;
+  * section 3 / 3.1: per-branch attention with its own softmax, shared RoPE key,
+    branch outputs summed;
+  * section 3.3: the branch sum is scaled.
+"""
+from __future__ import annotations
+
+import math
+import pathlib
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+from scipy.special import logsumexp
+
+GOLDEN = pathlib.Path(__file__).parent / "golden"
+
+
+def _rand(rng, *shape, scale=1.0):
+    return rng.standard_normal(shape) * scale
+
+
+def _one_seq(orc, q_lat, q_rope, c, kr, B, sigma, gamma, out_mode="branches"):
+    out, lse = orc.decode(q_lat[None], q_rope[None], c, kr, [c.shape[0]], None, B, sigma, gamma,
+                          max_seq_len=c.shape[0], out_mode=out_mode)
+    return out[0], lse[0]
+
+
+# --------------------------------------------------------------------------- explicit form
+def explicit_mlra(q_nope, q_rope, c, kr, W_uk, W_uv, sigma, gamma):
+    """Per-branch attention with decompressed keys/values (SDPA, float64).
+
+    q_nope [H, B, d_h], q_rope [H, d_R], c [L, d_c], kr [L, d_R],
+    W_uk / W_uv [H, B, d_h, d_blk].  Branch b keys: [W_uk[h,b] c_{j,b} ; k^R_j],
+    values W_uv[h,b] c_{j,b}; the branch outputs are summed and scaled.
+    """
+    H, B, d_h, d_blk = W_uk.shape
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x))
+    y = torch.zeros(H, d_h, dtype=torch.float64)
+    for b in range(B):
+        cb = t(c[:, b * d_blk:(b + 1) * d_blk])                       # [L, d_blk]
+        k_nope = torch.einsum("hkd,ld->hlk", t(W_uk[:, b]), cb)        # [H, L, d_h]
+        v = torch.einsum("hkd,ld->hlk", t(W_uv[:, b]), cb)             # [H, L, d_h]
+        k = torch.cat([k_nope, t(kr)[None].expand(H, -1, -1)], dim=-1)
+        q = torch.cat([t(q_nope[:, b]), t(q_rope)], dim=-1)[:, None]   # [H, 1, d_h+d_R]
+        o = F.scaled_dot_product_attention(q[None], k[None], v[None], scale=sigma)[0, :, 0]
+        y += o
+    return (gamma * y).numpy()
+
+
+def pin_absorbed_equals_explicit(orc, seed=0, H=6, B=4, d_blk=8, d_R=4, d_h=5, L=37):
+    """Step 1 absorption + step 2 + step 3 == explicit decompressed attention (section 1.3, 2, 3)."""
+    rng = np.random.default_rng(seed)
+    W_uk, W_uv = _rand(rng, H, B, d_h, d_blk), _rand(rng, H, B, d_h, d_blk)
+    q_nope, q_rope = _rand(rng, H, B, d_h), _rand(rng, H, d_R)
+    c, kr = _rand(rng, L, B * d_blk), _rand(rng, L, d_R)
+    sigma, gamma = 0.37, 1.0 / B
+    ref = explicit_mlra(q_nope, q_rope, c, kr, W_uk, W_uv, sigma, gamma)
+    q_lat = np.concatenate([np.einsum("hkd,hk->hd", W_uk[:, b], q_nope[:, b]) for b in range(B)], 1)
+    out, _ = _one_seq(orc, q_lat, q_rope, c, kr, B, sigma, gamma)
+    y = sum(np.einsum("hkd,hd->hk", W_uv[:, b], out[:, b * d_blk:(b + 1) * d_blk]) for b in range(B))
+    err = np.abs(y - ref).max() / np.abs(ref).max()
+    assert err <= 1e-12, f"absorbed vs explicit rel err {err:.3e}"
+
+
+def pin_summed_equals_explicit_shared_wuv(orc, seed=1, H=5, B=2, d_blk=6, d_R=4, d_h=3, L=29):
+    """Summed output mode == explicit form when every branch shares W^UV (section 3.3 sum)."""
+    rng = np.random.default_rng(seed)
+    W_uk = _rand(rng, H, B, d_h, d_blk)
+    W_uv = np.repeat(_rand(rng, H, 1, d_h, d_blk), B, axis=1)
+    q_nope, q_rope = _rand(rng, H, B, d_h), _rand(rng, H, d_R)
+    c, kr = _rand(rng, L, B * d_blk), _rand(rng, L, d_R)
+    sigma, gamma = 0.5, 1.0 / B
+    ref = explicit_mlra(q_nope, q_rope, c, kr, W_uk, W_uv, sigma, gamma)
+    q_lat = np.concatenate([np.einsum("hkd,hk->hd", W_uk[:, b], q_nope[:, b]) for b in range(B)], 1)
+    out, _ = _one_seq(orc, q_lat, q_rope, c, kr, B, sigma, gamma, out_mode="summed")
+    y = np.einsum("hkd,hd->hk", W_uv[:, 0], out)
+    err = np.abs(y - ref).max() / np.abs(ref).max()
+    assert err <= 1e-12, f"summed vs explicit rel err {err:.3e}"
+
+
+def pin_b1_equals_mqa(orc, seed=2, H=8, d_c=16, d_R=8, L=50):
+    """B=1 is MLA decode: MQA attention with key [c; k^R] and value c (section 1.3, step 2)."""
+    rng = np.random.default_rng(seed)
+    q_lat, q_rope = _rand(rng, H, d_c), _rand(rng, H, d_R)
+    c, kr = _rand(rng, L, d_c), _rand(rng, L, d_R)
+    sigma = 1 / math.sqrt(d_c + d_R)
+    q = torch.from_numpy(np.concatenate([q_lat, q_rope], 1))[None, :, None]      # [1,H,1,D]
+    k = torch.from_numpy(np.concatenate([c, kr], 1))[None, None].expand(1, H, L, -1)
+    v = torch.from_numpy(c)[None, None].expand(1, H, L, -1)
+    ref = F.scaled_dot_product_attention(q, k, v, scale=sigma)[0, :, 0].numpy()
+    out, lse = _one_seq(orc, q_lat, q_rope, c, kr, 1, sigma, 1.0)
+    assert np.abs(out - ref).max() <= 1e-12 * np.abs(ref).max(), "B=1 differs from MQA attention"
+    scores = sigma * (np.concatenate([q_lat, q_rope], 1) @ np.concatenate([c, kr], 1).T)
+    assert np.allclose(lse[:, 0], logsumexp(scores, axis=1), rtol=0, atol=1e-12), "lse"
+
+
+def brute_force(q_lat, q_rope, c, kr, B, sigma, gamma):
+    """Pure-Python loops, unshifted exp: for tiny inputs only."""
+    H, d_c = len(q_lat), len(q_lat[0])
+    d = d_c // B
+    L = len(c)
+    out = [[0.0] * d_c for _ in range(H)]
+    lse = [[0.0] * B for _ in range(H)]
+    for h in range(H):
+        for b in range(B):
+            w = []
+            for j in range(L):
+                s = 0.0
+                for k in range(d):
+                    s += q_lat[h][b * d + k] * c[j][b * d + k]
+                for k in range(len(kr[j])):
+                    s += q_rope[h][k] * kr[j][k]
+                w.append(math.exp(sigma * s))
+            z = sum(w)
+            lse[h][b] = math.log(z)
+            for i in range(d):
+                out[h][b * d + i] = gamma * sum(w[j] * c[j][b * d + i] for j in range(L)) / z
+    return np.array(out), np.array(lse)
+
+
+def pin_brute_force(orc, seed=3):
+    """Two-pass shifted softmax == unshifted brute force on tiny inputs, B in {1, 2, 4}."""
+    rng = np.random.default_rng(seed)
+    for B, H, d_c, d_R, L in [(1, 2, 4, 2, 5), (2, 3, 6, 2, 9), (4, 2, 8, 3, 13)]:
+        q_lat, q_rope = _rand(rng, H, d_c), _rand(rng, H, d_R)
+        c, kr = _rand(rng, L, d_c), _rand(rng, L, d_R)
+        ref, ref_lse = brute_force(q_lat.tolist(), q_rope.tolist(), c.tolist(), kr.tolist(), B, 0.7, 0.3)
+        out, lse = _one_seq(orc, q_lat, q_rope, c, kr, B, 0.7, 0.3)
+        assert np.allclose(out, ref, rtol=1e-12, atol=1e-13), f"brute force out B={B}"
+        assert np.allclose(lse, ref_lse, rtol=1e-12, atol=1e-13), f"brute force lse B={B}"
+
+
+def pin_probabilities(orc, seed=4, H=7, B=4, d_c=32, d_R=8, L=40):
+    """Each branch's weights are >= 0 and sum to 1 over positions (independent softmax, 3.1)."""
+    rng = np.random.default_rng(seed)
+    q_lat, q_rope = _rand(rng, H, d_c, scale=3), _rand(rng, H, d_R, scale=3)
+    c, kr = _rand(rng, L, d_c), _rand(rng, L, d_R)
+    p = orc.branch_probabilities(q_lat, q_rope, c, kr, B, 0.9)
+    assert p.shape == (B, H, L)
+    assert (p >= 0).all()
+    assert np.abs(p.sum(-1) - 1).max() <= 1e-13, "weights do not sum to one"
+    # different branches see different blocks -> different weights
+    assert np.abs(p[0] - p[1]).max() > 1e-3
+
+
+def pin_closed_forms(orc, seed=5):
+    """Special cases with closed-form results."""
+    rng = np.random.default_rng(seed)
+    H, B, d_c, d_R, gamma = 4, 4, 16, 4, 0.25
+    d = d_c // B
+    # one position: the output is gamma * c_0
+    q_lat, q_rope = _rand(rng, H, d_c), _rand(rng, H, d_R)
+    c, kr = _rand(rng, 1, d_c), _rand(rng, 1, d_R)
+    out, lse = _one_seq(orc, q_lat, q_rope, c, kr, B, 0.8, gamma)
+    assert np.allclose(out, gamma * np.broadcast_to(c[0], (H, d_c)), rtol=0, atol=1e-15), "L=1"
+    scores0 = [[0.8 * (q_lat[h, b * d:(b + 1) * d] @ c[0, b * d:(b + 1) * d] + q_rope[h] @ kr[0])
+                for b in range(B)] for h in range(H)]
+    assert np.allclose(lse, scores0, rtol=0, atol=1e-13), "L=1 lse equals the single score"
+    # zero queries: uniform weights, the output is gamma * mean_j c_j
+    L = 23
+    c, kr = _rand(rng, L, d_c), _rand(rng, L, d_R)
+    out, lse = _one_seq(orc, np.zeros((H, d_c)), np.zeros((H, d_R)), c, kr, B, 0.8, gamma)
+    assert np.allclose(out, gamma * c.mean(0)[None], rtol=0, atol=1e-14), "q=0 mean"
+    assert np.allclose(lse, math.log(L), rtol=0, atol=1e-13), "q=0 lse = log L"
+    # constant latent block: weights sum to one, so the output is gamma * const
+    c = np.full((L, d_c), 1.5)
+    out, _ = _one_seq(orc, _rand(rng, H, d_c), _rand(rng, H, d_R), c, kr, B, 0.8, gamma)
+    assert np.allclose(out, gamma * 1.5, rtol=0, atol=1e-14), "constant c"
+    # one dominant score (the RoPE term, shared by every branch): output ~ gamma * c_j*
+    c = _rand(rng, L, d_c)
+    kr = np.zeros((L, d_R))
+    kr[11, 0] = 60.0
+    q_rope = np.zeros((H, d_R))
+    q_rope[:, 0] = 1.0
+    out, _ = _one_seq(orc, _rand(rng, H, d_c, scale=0.1), q_rope, c, kr, B, 1.0, gamma)
+    assert np.allclose(out, gamma * c[11][None], rtol=0, atol=1e-12), "spike"
+    # huge common shift of every score changes nothing (max subtraction)
+    q_lat, q_rope = _rand(rng, H, d_c), _rand(rng, H, d_R)
+    c, kr = _rand(rng, L, d_c), _rand(rng, L, d_R)
+    base, lb = _one_seq(orc, q_lat, q_rope, c, kr, B, 0.8, gamma)
+    kr2 = np.concatenate([kr, np.full((L, 1), 1000.0)], 1)
+    qr2 = np.concatenate([q_rope, np.ones((H, 1))], 1)
+    shifted, ls = _one_seq(orc, q_lat, qr2, c, kr2, B, 0.8, gamma)
+    assert np.isfinite(shifted).all() and np.allclose(shifted, base, rtol=0, atol=1e-12), "shift"
+    assert np.allclose(ls - lb, 800.0, rtol=0, atol=1e-9), "lse shifts by sigma * 1000"
+
+
+def pin_branch_independence(orc, seed=6, H=5, B=4, d_c=32, d_R=8, L=31):
+    """Changing block b' of the latent leaves every other branch's output bit-identical."""
+    rng = np.random.default_rng(seed)
+    d = d_c // B
+    q_lat, q_rope = _rand(rng, H, d_c), _rand(rng, H, d_R)
+    c, kr = _rand(rng, L, d_c), _rand(rng, L, d_R)
+    base, lb = _one_seq(orc, q_lat, q_rope, c, kr, B, 0.6, 0.25)
+    for bp in range(B):
+        c2 = c.copy()
+        c2[:, bp * d:(bp + 1) * d] = _rand(rng, L, d)
+        out, l2 = _one_seq(orc, q_lat, q_rope, c2, kr, B, 0.6, 0.25)
+        for b in range(B):
+            same = np.array_equal(out[:, b * d:(b + 1) * d], base[:, b * d:(b + 1) * d])
+            assert same == (b != bp), f"branch {b} after changing block {bp}"
+            assert np.array_equal(l2[:, b], lb[:, b]) == (b != bp)
+    # and the shared RoPE key moves every branch
+    kr2 = kr.copy()
+    kr2[3] += 1.0
+    out, _ = _one_seq(orc, q_lat, q_rope, c, kr2, B, 0.6, 0.25)
+    for b in range(B):
+        assert not np.array_equal(out[:, b * d:(b + 1) * d], base[:, b * d:(b + 1) * d])
+
+
+def pin_position_permutation(orc, seed=7, H=3, B=2, d_c=12, d_R=4, L=19):
+    """Attention is a set function of the cached positions."""
+    rng = np.random.default_rng(seed)
+    q_lat, q_rope = _rand(rng, H, d_c), _rand(rng, H, d_R)
+    c, kr = _rand(rng, L, d_c), _rand(rng, L, d_R)
+    perm = rng.permutation(L)
+    a, la = _one_seq(orc, q_lat, q_rope, c, kr, B, 0.9, 0.5)
+    b, lb = _one_seq(orc, q_lat, q_rope, c[perm], kr[perm], B, 0.9, 0.5)
+    assert np.allclose(a, b, rtol=0, atol=1e-13) and np.allclose(la, lb, rtol=0, atol=1e-13)
+
+
+def pin_batch_rows_and_paging(orc, seed=8):
+    """Paged (shuffled pages) and contiguous layouts give identical results; empty sequence."""
+    rng = np.random.default_rng(seed)
+    N, H, B, d_c, d_R, P = 3, 4, 2, 8, 4, 4
+    lens = [10, 0, 7]
+    Lmax = 12
+    q_lat, q_rope = _rand(rng, N, H, d_c), _rand(rng, N, H, d_R)
+    c_cont, kr_cont = _rand(rng, N * Lmax, d_c), _rand(rng, N * Lmax, d_R)
+    out_c, lse_c = orc.decode(q_lat, q_rope, c_cont, kr_cont, lens, None, B, 0.7, 0.5, max_seq_len=Lmax)
+    # scatter the same rows into shuffled pages
+    n_pages = 3 * (Lmax // P)
+    perm = rng.permutation(n_pages)
+    pt = np.full((N, Lmax // P), -1)
+    c_pool, kr_pool = np.full((n_pages * P, d_c), np.nan), np.full((n_pages * P, d_R), np.nan)
+    k = 0
+    for s in range(N):
+        for pg in range((lens[s] + P - 1) // P):
+            pt[s, pg] = perm[k]
+            k += 1
+            for r in range(P):
+                j = pg * P + r
+                if j < lens[s]:
+                    c_pool[pt[s, pg] * P + r] = c_cont[s * Lmax + j]
+                    kr_pool[pt[s, pg] * P + r] = kr_cont[s * Lmax + j]
+    out_p, lse_p = orc.decode(q_lat, q_rope, c_pool, kr_pool, lens, pt, B, 0.7, 0.5, page_size=P)
+    assert np.array_equal(out_p, out_c) and np.array_equal(lse_p, lse_c), "paged != contiguous"
+    assert (out_c[1] == 0).all() and np.isneginf(lse_c[1]).all(), "empty sequence"
+    # each sequence alone equals its batch entry
+    for s in (0, 2):
+        o1, l1 = _one_seq(orc, q_lat[s], q_rope[s], c_cont[s * Lmax:s * Lmax + lens[s]],
+                          kr_cont[s * Lmax:s * Lmax + lens[s]], B, 0.7, 0.5)
+        assert np.array_equal(o1, out_c[s]) and np.array_equal(l1, lse_c[s])
+
+
+# --------------------------------------------------------------------------- golden fixtures
+def read_fixture(name):
+    """Parse ``key = expression`` lines (``#`` comments) with math names available."""
+    env = {k: getattr(math, k) for k in ("log", "exp", "sqrt", "inf")}
+    vals = {}
+    for line in (GOLDEN / name).read_text().splitlines():
+        line = line.split("#", 1)[0].strip()
+        if not line:
+            continue
+        key, expr = (x.strip() for x in line.split("=", 1))
+        vals[key] = eval(expr, {"__builtins__": {}}, env)  # fixture text is ours and tiny
+    return vals
+
+
+def pin_golden_hand_worked(orc):
+    """Hand-derived closed-form example (tests/golden/hand_worked_mlra2.txt)."""
+    f = read_fixture("hand_worked_mlra2.txt")
+    q_lat, q_rope = np.array(f["q_lat"], float), np.array(f["q_rope"], float)
+    c, kr = np.array(f["c_kv"], float), np.array(f["k_rope"], float)
+    for tag in ("a", "b"):
+        sigma, gamma = f[f"sigma_{tag}"], f["gamma"]
+        out, lse = _one_seq(orc, q_lat, q_rope, c, kr, 2, sigma, gamma)
+        assert np.allclose(out, f[f"out_{tag}"], rtol=0, atol=1e-14), f"golden out {tag}"
+        assert np.allclose(lse, f[f"lse_{tag}"], rtol=0, atol=1e-14), f"golden lse {tag}"
+        summed, _ = _one_seq(orc, q_lat, q_rope, c, kr, 2, sigma, gamma, out_mode="summed")
+        assert np.allclose(summed[:, 0], f[f"summed_{tag}"], rtol=0, atol=1e-14), f"golden sum {tag}"
+
+
+def pin_golden_rows(orc):
+    """Hand-written page-resolution example (tests/golden/page_rows.txt)."""
+    f = read_fixture("page_rows.txt")
+    for s, L in enumerate(f["seq_lens"]):
+        paged = orc.resolve_rows(L, s, f["page_table"], f["page_size"], 0).tolist()
+        cont = orc.resolve_rows(L, s, None, 0, f["max_seq_len"]).tolist()
+        assert paged == f["paged_rows"][s], f"paged rows of sequence {s}"
+        assert cont == f["contiguous_rows"][s], f"contiguous rows of sequence {s}"
+
+
+ALL_PINS = [
+    pin_absorbed_equals_explicit,
+    pin_summed_equals_explicit_shared_wuv,
+    pin_b1_equals_mqa,
+    pin_brute_force,
+    pin_probabilities,
+    pin_closed_forms,
+    pin_branch_independence,
+    pin_position_permutation,
+    pin_batch_rows_and_paging,
+    pin_golden_hand_worked,
+    pin_golden_rows,
+]
