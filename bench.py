@@ -1,0 +1,413 @@
+"""Decode-attention benchmark: MLRA step-2 decode on synthetic inputs, one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+A step is one decode call (queries of N sequences against their resident latent/RoPE caches):
+prep -> split-KV attention -> combine, all in libmlra.so.  ``value`` is whole-job decode
+tokens/s (one token per sequence per step), device-timed with CUDA events over exactly K steps
+between barriers, max over ranks.  Multi-GPU runs are weak scaling: every rank decodes its own
+batch (seed + rank), with no collective on the data path.
+
+``--impl reference`` times the CPU float64 oracle (the only other implementation of this path)
+on a bounded sample of the same workload and prints the same line with ``"impl": "reference"``.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import pathlib
+import statistics
+import sys
+import threading
+import time
+
+ROOT = pathlib.Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "decode tokens/s and latent-KV HBM GB/s (fraction of B200 peak), 1 GPU"
+DEFAULT_WORKLOAD = "mlra4_n8_l32k"
+L2_BYTES = 126 * 2 ** 20
+PROFILE_DIR = ROOT / "profiles"
+KERNEL_SOURCES = ["mlra_decode_kernel.cuh", "sm100_ptx.cuh", "mlra_plan.cuh"]
+
+
+# ----------------------------------------------------------------------------- work accounting
+def cache_bytes(inp: workloads.Inputs) -> int:
+    """Algorithmic bytes of one attention launch: every cached latent/RoPE element once."""
+    w = inp.workload
+    elem = 2  # the kernel streams bf16
+    return int(inp.seq_lens.to(torch.int64).sum()) * (w.d_latent + w.d_rope) * elem
+
+
+def algorithmic_flops(inp: workloads.Inputs) -> int:
+    """2 H (d_c + d_R) for the scores (RoPE term once per head) + 2 H d_c for the outputs."""
+    w = inp.workload
+    return int(inp.seq_lens.to(torch.int64).sum()) * 2 * w.heads * (2 * w.d_latent + w.d_rope)
+
+
+def measured_peaks() -> dict:
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        h.update((ROOT / "latent_kv_cache_mlra_b200" / "csrc" / name).read_bytes())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary, if it matches the
+    current kernel source; else None."""
+    f = PROFILE_DIR / f"decode_kernel_{workload}.md"
+    if not f.exists():
+        return None
+    vals = {}
+    for line in f.read_text().splitlines():
+        if line.startswith("- ") and ":" in line:
+            k, v = line[2:].split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_hash") != kernel_hash():
+        return None
+    try:
+        return int(float(vals["dram_bytes_per_launch"]))
+    except (KeyError, ValueError):
+        return None
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons with NVML every ``period`` seconds."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index: int, period: float = 0.02):
+        self.samples, self.period, self.ok = [], period, False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.handle = self._handle(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # no NVML (CPU machine): the line carries clocks = null
+            self.ok = False
+
+    def _handle(self, idx):
+        nv = self.nv
+        try:
+            uuid = str(torch.cuda.get_device_properties(idx).uuid)
+            return nv.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(idx)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                try:
+                    reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                except AttributeError:
+                    reasons = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.handle)
+                power = nv.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+                self.samples.append((sm, reasons, power))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return None
+        sms = [s[0] for s in self.samples]
+        bits = 0
+        for s in self.samples:
+            bits |= s[1]
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": self.max_mhz,
+                "reasons": [n for b, n in self.REASONS.items() if bits & b],
+                "samples": len(self.samples), "power_w_median": statistics.median(s[2] for s in self.samples)}
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1:
+        import torch.distributed as dist
+        rank, local = int(os.environ["RANK"]), int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return rank, world, local
+    return 0, 1, 0
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_workload(name: str, rank: int) -> workloads.Workload:
+    w = workloads.get(name)
+    return workloads.Workload(**{**w.__dict__, "seed": w.seed + 7919 * rank})
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def time_oracle(inp: workloads.Inputs, budget_s: float, max_seqs=None):
+    """Runs the oracle on whole sequences (all heads) until the budget is spent; returns
+    (seconds, sequences done, threads used)."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+    except ImportError:
+        threadpool_info = None
+    w = inp.workload
+    order = list(range(w.batch))[: max_seqs or w.batch]
+    t0 = time.perf_counter()
+    done = 0
+    for s in order:
+        oracle.decode(inp.q_lat, inp.q_rope, inp.c_kv, inp.k_rope, inp.seq_lens, inp.page_table,
+                      w.num_branches, w.sigma, w.gamma, page_size=w.page_size,
+                      max_seq_len=inp.max_seq_len, seqs=[s])
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    threads = len(os.sched_getaffinity(0))
+    if threadpool_info:
+        nums = [p.get("num_threads", 0) for p in threadpool_info() if p.get("user_api") == "blas"]
+        if nums:
+            threads = max(nums)
+    return dt, done, threads
+
+
+def time_oracle_heads(inp: workloads.Inputs, seq: int, heads: slice):
+    import oracle
+    w = inp.workload
+    t0 = time.perf_counter()
+    oracle.decode(inp.q_lat, inp.q_rope, inp.c_kv, inp.k_rope, inp.seq_lens, inp.page_table,
+                  w.num_branches, w.sigma, w.gamma, page_size=w.page_size,
+                  max_seq_len=inp.max_seq_len, seqs=[seq], heads=heads)
+    return time.perf_counter() - t0
+
+
+def workload_config(w: workloads.Workload, inp: workloads.Inputs) -> dict:
+    return {"workload": w.name, "batch": w.batch, "heads": w.heads, "branches": w.num_branches,
+            "d_latent": w.d_latent, "d_rope": w.d_rope,
+            "seq_len": w.seq_len if not w.ragged else f"log-uniform[{w.min_seq_len},{w.seq_len}]",
+            "tokens_in_cache": int(inp.seq_lens.sum()), "page_size": w.page_size,
+            "softmax_scale": w.sigma, "branch_scale": w.gamma, "latent_scale": w.latent_scale,
+            "seed": w.seed, "layers": 1,
+            "l2": f"inputs larger than L2 ({cache_bytes(inp) / 1e6:.0f} MB of cache per step vs 126 MiB L2)"
+            if cache_bytes(inp) > L2_BYTES else "L2 flushed between steps"}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank, world = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return 0
+    w = workloads.get(args.workload)
+    inp = workloads.make_inputs(w)
+    H = w.heads
+    # one step = a bounded slice of heads of one sequence, sized so that the whole run stays
+    # within about two minutes
+    probe = time_oracle_heads(inp, 0, slice(0, 1))
+    per_step = 120.0 / max(1, args.steps + args.warmup)
+    nh = int(max(1, min(H, per_step / max(probe, 1e-6))))
+    sl = slice(0, nh)
+    for _ in range(args.warmup):
+        time_oracle_heads(inp, 0, sl)
+    ts = [time_oracle_heads(inp, 0, sl) for _ in range(args.steps)]
+    t_step = sum(ts) / len(ts)
+    frac = nh / (w.batch * H)                      # share of one full decode step
+    value = w.batch * frac / t_step                # tokens/s of a full step at this rate
+    threads = time_oracle(inp, 0.0, max_seqs=1)[2]
+    sample = (f"heads 0..{nh - 1} of sequence 0 (L={int(inp.seq_lens[0])}), "
+              f"{nh}/{w.batch * H} of one decode step per timed step")
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step / frac * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference", "config": workload_config(w, inp),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args):
+    from latent_kv_cache_mlra_b200 import mlra
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = rank_workload(args.workload, rank)
+    inp = workloads.make_inputs(w)
+    pt = None if inp.page_table is None else inp.page_table.to(dev)
+    q, qr = inp.q_lat.to(dev), inp.q_rope.to(dev)
+    c, kr = inp.c_kv.to(dev), inp.k_rope.to(dev)
+    lens = inp.seq_lens.to(dev)
+    dec = mlra.Decoder(q, qr, c, kr, lens, pt, num_branches=w.num_branches,
+                       softmax_scale=w.sigma, branch_scale=w.gamma, max_seq_len=inp.max_seq_len,
+                       page_size=w.page_size, with_lse=False)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = dec.plan.launches
+    nbytes, nflops = cache_bytes(inp), algorithmic_flops(inp)
+    flush = None if nbytes > L2_BYTES else torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(ev=None):
+        if flush is not None:
+            flush.zero_()
+        dec(k1_events=ev)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    rc, flags = dec.status()
+    if rc != 0:
+        raise RuntimeError(f"device status after warm-up: {mlra.status_string(rc)} (flags {flags})")
+
+    k1 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(k1[i])
+        t_stop.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms_total = t_start.elapsed_time(t_stop)
+    k1_ms = [a.elapsed_time(b) for a, b in k1]
+    ms_total = max_over_ranks(ms_total, world, dev)
+    ms_step = ms_total / args.steps
+    k1_avg_ms = max_over_ranks(sum(k1_ms) / len(k1_ms), world, dev)
+    rc, flags = dec.status()
+    if rc != 0:
+        raise RuntimeError(f"device status after timing: {mlra.status_string(rc)} (flags {flags})")
+
+    # end to end through the public API: pinned host queries/lengths in, output back to host
+    h_q, h_qr = inp.q_lat.pin_memory(), inp.q_rope.pin_memory()
+    h_lens = inp.seq_lens.pin_memory()
+    h_out = torch.empty(dec.out.shape, dtype=dec.out.dtype).pin_memory()
+    h2d = h_q.numel() * h_q.element_size() + h_qr.numel() * h_qr.element_size() + h_lens.numel() * 4
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        q.copy_(h_q, non_blocking=True)
+        qr.copy_(h_qr, non_blocking=True)
+        lens.copy_(h_lens, non_blocking=True)
+        step()
+        h_out.copy_(dec.out, non_blocking=True)
+
+    for _ in range(min(args.warmup, 10)):
+        e2e_step()
+    e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e_start.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e_stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_stop), world, dev) / args.steps
+
+    peaks = measured_peaks()
+    achieved_gbs = nbytes / (k1_avg_ms * 1e-3) / 1e9
+    step_gbs = nbytes / (ms_step * 1e-3) / 1e9
+    tflops = nflops / (k1_avg_ms * 1e-3) / 1e12
+    total_seqs = w.batch * world
+    line = {
+        "metric": METRIC, "value": total_seqs / (ms_step * 1e-3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": {**workload_config(w, inp), "parallelism": f"dp{world}"},
+        "latent_gbs": step_gbs * world,
+        "latent_gbs_frac_of_measured": step_gbs / peaks["hbm_gbs"],
+        "latent_gbs_frac_of_8tbs": step_gbs / 8000.0,
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"],
+                     "traffic": recorded_traffic(w.name), "kernel": "mlra_decode_kernel",
+                     "kernel_ms": k1_avg_ms, "algorithmic_bytes_per_launch": nbytes,
+                     "peak_source": f"{peaks['source']} hbm_gbs (copy test)",
+                     "frac_of_8tbs": achieved_gbs / 8000.0,
+                     "tensor_tflops": tflops, "tensor_frac": tflops / peaks["bf16_tflops"]},
+        "e2e": {"value": total_seqs / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "note": "queries and lengths copied in, output copied out each step; "
+                        "the latent/RoPE cache stays resident like model state"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, done, threads = time_oracle(inp, budget_s=20.0)
+        line["cpu_baseline"] = {"value": done / dt, "unit": "tokens/s", "cores": threads,
+                                "kind": "oracle",
+                                "sample": f"{done} of {w.batch} sequences (all heads, full length), "
+                                          f"{dt:.1f} s on the host cores"}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,194 @@
+/*
+ * mlra.h -- C ABI of the B200 (sm_100a) MLRA single-token decode-attention library.
+ *
+ * The operation ("Multi-Head Low-Rank Attention", yunpan.plus page):
+ *   section 1.3  MLA's efficient decode in three steps -- (1) absorb the key up-projection
+ *                into the query, (2) run MQA-style attention of the absorbed query against the
+ *                cached latent vectors, (3) apply the value up-projection.  This library is
+ *                step 2.
+ *   section 2    the per-head NoPE key is a sum of B block projections of the latent, so the
+ *                latent c_t splits into B column blocks c_{t,b} of width d_blk = d_latent / B;
+ *   section 3.1  MLRA moves that sum behind the attention: every branch b runs its own
+ *                attention over its block with its own softmax over positions, and the RoPE
+ *                key k^R_t is shared by all branches;
+ *   section 3.3  the sum of the branch outputs is scaled.
+ *
+ * For sequence s, head h < heads, branch b < B and cached position j < seq_lens[s]:
+ *
+ *   score(j)          = softmax_scale * ( q_lat[s,h, b-block] . c_kv[row(s,j), b-block]
+ *                                       + q_rope[s,h,:]       . k_rope[row(s,j), :] )
+ *   p                 = softmax over j of score                 (one softmax per branch)
+ *   out[s,h, b-block] = branch_scale * sum_j p(j) * c_kv[row(s,j), b-block]
+ *   lse[s,h,b]        = log sum_j exp(score(j))                  (natural log)
+ *
+ * With num_branches = 1 this is plain MLA decode.  MLRA_OUT_SUMMED adds the B branch
+ * outputs instead: out[s,h,:] = sum_b out[s,h,b-block] (width d_blk).
+ *
+ * Rows: with page_table == NULL the cache is contiguous, row(s,j) = s * max_seq_len + j;
+ * otherwise row(s,j) = page_table[s * max_pages_per_seq + j / page_size] * page_size
+ *                      + j % page_size.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named *_host are host memory; every other pointer is CUDA device memory.
+ *   - The caller owns every buffer, including the workspace; the library never allocates
+ *     device memory and keeps no pointer after a call returns.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *     unless stated otherwise; nothing synchronises.
+ *   - Argument errors are returned before any work is queued.  Problems found on the device
+ *     (bad lengths, bad page ids, an internal wait that ran out) never trap: they set bits in
+ *     a status word inside the workspace, read with mlra_read_status().
+ *   - All functions are thread-safe; calls that share a workspace must not overlap on the GPU.
+ */
+#ifndef MLRA_H_
+#define MLRA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* mlra_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  MLRA_OK = 0,
+  MLRA_ERR_INVALID_ARG = 1,  /* null pointer, negative size, inconsistent dims */
+  MLRA_ERR_UNSUPPORTED = 2,  /* valid but not handled (see mlra_decode) */
+  MLRA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+  MLRA_ERR_TIMEOUT = 4,      /* a device-side bounded wait ran out (status word) */
+  MLRA_ERR_WORKSPACE = 5,    /* workspace null, too small or misaligned */
+  MLRA_ERR_BAD_PAGE = 6,     /* a page id outside [0, cache_rows / page_size) (status word) */
+  MLRA_ERR_BAD_LENGTH = 7    /* a sequence length < 0 or beyond the cache (status word) */
+} mlra_status;
+
+typedef enum { MLRA_BF16 = 0, MLRA_F32 = 1 } mlra_dtype;
+typedef enum { MLRA_OUT_BRANCHES = 0, MLRA_OUT_SUMMED = 1 } mlra_out_mode;
+
+/* Device status bits (mlra_read_status). */
+#define MLRA_FLAG_TIMEOUT 0x1u
+#define MLRA_FLAG_BAD_PAGE 0x2u
+#define MLRA_FLAG_BAD_LENGTH 0x4u
+
+typedef struct {
+  float softmax_scale; /* sigma: multiplies the whole score (NoPE + RoPE terms) */
+  float branch_scale;  /* gamma: multiplies every branch output (1/B for the MLRA sum) */
+} mlra_scales;
+
+typedef struct {
+  int batch;              /* N >= 1 sequences, one query token each */
+  int heads;              /* H, 1..64 */
+  int num_branches;       /* B >= 1, divides d_latent */
+  int d_latent;           /* d_c = B * d_blk, <= 512 */
+  int d_rope;             /* d_R, 1..64 */
+  int page_size;          /* P (paged layout, a multiple of 64); ignored when page_table == NULL */
+  int max_pages_per_seq;  /* page_table row pitch (paged layout) */
+  int max_seq_len;        /* contiguous layout: row pitch of a sequence; both layouts: bound on
+                             seq_lens (paged: also <= max_pages_per_seq * page_size) */
+  long long cache_rows;   /* rows in c_kv and k_rope (paged: the pool; contiguous: >= N * max_seq_len) */
+  long long c_row_stride; /* elements between consecutive c_kv rows (>= d_latent) */
+  long long kr_row_stride;/* elements between consecutive k_rope rows (>= d_rope); c_kv and
+                             k_rope may be two column ranges of one row (e.g. 576-wide rows) */
+  mlra_dtype dtype;       /* element type of q_lat, q_rope, c_kv, k_rope */
+  mlra_out_mode out_mode;
+  int num_ranges;         /* 0: one work range per SM (per branch group); > 0 forces the number
+                             of equal tile ranges the batch is cut into (split-K control) */
+} mlra_dims;
+
+/* Bytes of workspace mlra_decode needs for `dims` (and the device's SM count when
+ * dims->num_ranges == 0, queried on the current device).  Host only, synchronous.
+ * Errors: MLRA_ERR_INVALID_ARG / MLRA_ERR_UNSUPPORTED as mlra_decode; MLRA_ERR_CUDA when the
+ * SM count is needed and no device is available. */
+mlra_status mlra_workspace_size(const mlra_dims* dims, size_t* bytes_host);
+
+/* Step 2 of MLRA decode (see the top of this file).
+ *   q_lat      [N, H, d_latent]   dims->dtype, contiguous: the absorbed queries q~ (section 1.3,
+ *                                 step 1 output), branch b in columns [b*d_blk, (b+1)*d_blk)
+ *   q_rope     [N, H, d_rope]     dims->dtype, contiguous: the RoPE queries q^R
+ *   c_kv       [cache_rows, *]    dims->dtype, row pitch c_row_stride: latent cache c^KV
+ *   k_rope     [cache_rows, *]    dims->dtype, row pitch kr_row_stride: shared RoPE key cache k^R
+ *   seq_lens   [N]                int32, read on the device
+ *   page_table [N, max_pages_per_seq] int32 page ids, or NULL for the contiguous layout
+ *   B          must equal dims->num_branches (kept in the signature as a guard)
+ *   scales     host pointer to {sigma, gamma}
+ *   out        fp32 [N, H, d_latent] (MLRA_OUT_BRANCHES) or [N, H, d_latent / B] (SUMMED)
+ *   lse        fp32 [N, H, B] or NULL
+ *   workspace  >= mlra_workspace_size bytes, 256-byte aligned, caller-owned scratch
+ * An empty sequence (seq_lens[s] == 0) gives out = 0 and lse = -inf.
+ * bf16 inputs with d_blk in {64, 128, 256, 512}, d_rope == 64, 16-byte aligned rows and
+ * base pointers are read in place.  Other shapes (and fp32 inputs) are first repacked into
+ * padded bf16 copies inside the workspace (a full copy of the cache per call: meant for
+ * small problems).  MLRA_ERR_UNSUPPORTED: H > 64, d_latent > 512, d_rope > 64, page_size not
+ * a multiple of 64, misaligned bf16 rows.  Launch failures return MLRA_ERR_CUDA. */
+mlra_status mlra_decode(const void* q_lat, const void* q_rope, const void* c_kv, const void* k_rope,
+                        const int32_t* seq_lens, const int32_t* page_table, int B,
+                        const mlra_scales* scales, float* out, float* lse, const mlra_dims* dims,
+                        void* workspace, size_t ws_bytes, mlra_stream_t stream);
+
+/* Same as mlra_decode, and records the caller's CUDA events `k1_begin` / `k1_end` (cudaEvent_t,
+ * either may be NULL) on `stream` immediately before and after the split-KV attention kernel,
+ * so that its duration can be timed alone (cudaEventElapsedTime).  Errors as mlra_decode;
+ * a failing cudaEventRecord returns MLRA_ERR_CUDA. */
+typedef struct CUevent_st* mlra_event_t; /* same type as cudaEvent_t */
+mlra_status mlra_decode_profiled(const void* q_lat, const void* q_rope, const void* c_kv,
+                                 const void* k_rope, const int32_t* seq_lens,
+                                 const int32_t* page_table, int B, const mlra_scales* scales,
+                                 float* out, float* lse, const mlra_dims* dims, void* workspace,
+                                 size_t ws_bytes, mlra_stream_t stream, mlra_event_t k1_begin,
+                                 mlra_event_t k1_end);
+
+/* What mlra_decode will do for `dims` (same rules and SM-count query as mlra_workspace_size).
+ * Host only, synchronous. */
+typedef struct {
+  int repack;             /* 1: inputs are first copied into padded bf16 buffers */
+  int launches;           /* kernels launched per mlra_decode call */
+  int num_ranges;         /* equal work ranges the batch's KV tiles are cut into */
+  int ctas;               /* CTAs of the attention kernel (ranges x branch groups) */
+  int kernel_branch_width;/* branch width after padding (64, 128, 256 or 512) */
+  int branches_per_cta;   /* 1 or 2 */
+  long long partial_slots;/* partial-result slots in the workspace (num_ranges + N - 1) */
+  size_t workspace_bytes;
+} mlra_plan_info;
+mlra_status mlra_query_plan(const mlra_dims* dims, mlra_plan_info* info_host);
+
+/* Reads the status word that the last mlra_decode on `workspace` left, after synchronising
+ * `stream`.  *flags_host receives the MLRA_FLAG_* bits; the return value is MLRA_OK when no
+ * bit is set, else the status of the most serious bit (timeout, bad page, bad length). */
+mlra_status mlra_read_status(const void* workspace, mlra_stream_t stream, uint32_t* flags_host);
+
+/* Test hook for the indexing logic (bit-exact): writes the cache row of every position
+ * j < min(seq_lens[s], row_pitch) into rows_out[s * row_pitch + j] (int64, device), computed
+ * by the same device function the decode kernel uses to address its TMA tiles.  Entries
+ * past a sequence's length are left untouched.  Same dims rules as mlra_decode. */
+mlra_status mlra_debug_resolve_rows(const int32_t* seq_lens, const int32_t* page_table,
+                                    const mlra_dims* dims, int64_t* rows_out, int row_pitch,
+                                    mlra_stream_t stream);
+
+/* Host replica of the split plan (the same __host__ __device__ code the kernels run): for
+ * tile counts tiles_host[N] cut into min(num_ranges, total tiles) equal ranges, writes for every
+ * sequence the first range touching it and the number of ranges (partial results) it is split
+ * into (0 for an empty sequence).
+ * Host only, synchronous; for tests and tooling. */
+mlra_status mlra_plan_host(const int32_t* tiles_host, int n, int num_ranges,
+                           int32_t* first_range_host, int32_t* num_parts_host);
+
+/* Host replica of the per-CTA segment walk of the attention kernel: for tile counts
+ * tiles_host[N] and num_ranges CTAs (per branch group), lists every (range, sequence, first
+ * tile, tile count) segment that the kernel's CTAs r = 0 .. num_ranges-1 process, in CTA order.
+ * At most max_segments are written to the four *_host arrays; *count_host receives the total.
+ * Host only, synchronous; for tests and tooling. */
+mlra_status mlra_plan_segments_host(const int32_t* tiles_host, int n, int num_ranges,
+                                    int32_t* range_host, int32_t* seq_host, int32_t* tile0_host,
+                                    int32_t* ntiles_host, int max_segments, int* count_host);
+
+/* Human-readable name of a status code (static string). */
+const char* mlra_status_string(mlra_status s);
+
+/* Library version, e.g. 0x000100 for 0.1.0. */
+int mlra_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLRA_H_ */

@@ -1,0 +1,409 @@
+// mlra_api.cu -- the C ABI declared in include/mlra.h: argument checks, the split plan,
+// the workspace layout, TMA tensor maps and the launch sequence K3? -> K0 -> K1 -> K2.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "mlra.h"
+#include "mlra_internal.h"
+#include "mlra_plan.cuh"
+
+namespace {
+
+using namespace mlra;
+
+constexpr size_t kAlign = 256;
+constexpr uint64_t kTimeoutNs = 1000ull * 1000ull * 1000ull;  // 1 s bound on every device wait
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Plan {
+  bool repack = false;
+  Variant variant = kV128x2;
+  int dblk_k = 0;      // padded branch width seen by the kernel
+  int G = 2;           // branches per CTA
+  int n_groups = 1;    // CTAs per range
+  int dck = 0;         // B * dblk_k
+  int R = 0;           // work ranges
+  int64_t slots = 0;   // partial slots = R + N - 1
+  int limit = 0;       // bound on seq_lens
+  size_t off_lens = 0, off_prefix = 0, off_ml = 0, off_o = 0;
+  size_t off_rq = 0, off_rqr = 0, off_rc = 0, off_rkr = 0, total = 0;
+};
+
+int device_sm_count(mlra_status* st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { *st = MLRA_ERR_CUDA; return 0; }
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+    *st = MLRA_ERR_CUDA;
+    return 0;
+  }
+  *st = MLRA_OK;
+  return sms;
+}
+
+mlra_status check_dims(const mlra_dims* d, bool paged) {
+  if (!d) return MLRA_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->heads < 1 || d->num_branches < 1 || d->d_latent < 1 || d->d_rope < 1)
+    return MLRA_ERR_INVALID_ARG;
+  if (d->d_latent % d->num_branches != 0) return MLRA_ERR_INVALID_ARG;
+  if (d->max_seq_len < 0 || d->cache_rows < 0 || d->num_ranges < 0) return MLRA_ERR_INVALID_ARG;
+  if (d->c_row_stride < d->d_latent || d->kr_row_stride < d->d_rope) return MLRA_ERR_INVALID_ARG;
+  if (d->dtype != MLRA_BF16 && d->dtype != MLRA_F32) return MLRA_ERR_INVALID_ARG;
+  if (d->out_mode != MLRA_OUT_BRANCHES && d->out_mode != MLRA_OUT_SUMMED) return MLRA_ERR_INVALID_ARG;
+  if (paged) {
+    if (d->page_size < 1 || d->max_pages_per_seq < 1) return MLRA_ERR_INVALID_ARG;
+    if ((int64_t)d->page_size * d->max_pages_per_seq > INT_MAX) return MLRA_ERR_INVALID_ARG;
+  } else {
+    if ((int64_t)d->batch * d->max_seq_len > d->cache_rows) return MLRA_ERR_INVALID_ARG;
+  }
+  if (d->heads > 64 || d->d_latent > 512 || d->d_rope > 64) return MLRA_ERR_UNSUPPORTED;
+  if (paged && d->page_size % kTile != 0) return MLRA_ERR_UNSUPPORTED;
+  if (d->cache_rows > (int64_t)INT_MAX - 2 * kTile) return MLRA_ERR_UNSUPPORTED;
+  if (d->num_branches > 64) return MLRA_ERR_UNSUPPORTED;
+  return MLRA_OK;
+}
+
+// Kernel variant and workspace layout.  sms == 0 requires dims->num_ranges > 0.
+mlra_status make_plan(const mlra_dims* d, bool paged, int sms, Plan* pl) {
+  mlra_status st = check_dims(d, paged);
+  if (st != MLRA_OK) return st;
+  const int B = d->num_branches, dblk = d->d_latent / B;
+  int dk = dblk <= 64 ? 64 : dblk <= 128 ? 128 : dblk <= 256 ? 256 : 512;
+  if (dk == 64 && B % 2 != 0) dk = 128;
+  if (B * dk > 512) return MLRA_ERR_UNSUPPORTED;
+  const bool inplace_shape = (dk == dblk) && d->d_rope == 64;
+  const bool inplace_align = d->c_row_stride % 8 == 0 && d->kr_row_stride % 8 == 0;
+  if (d->dtype == MLRA_BF16 && inplace_shape && !inplace_align) return MLRA_ERR_UNSUPPORTED;
+  pl->repack = !(d->dtype == MLRA_BF16 && inplace_shape);
+  pl->dblk_k = dk;
+  if (dk == 64) { pl->variant = kV64x2; pl->G = 2; }
+  else if (dk == 128) { pl->variant = (B % 2 == 0) ? kV128x2 : kV128x1; pl->G = (B % 2 == 0) ? 2 : 1; }
+  else if (dk == 256) { pl->variant = kV256x1; pl->G = 1; }
+  else { pl->variant = kV512x1; pl->G = 1; }
+  pl->n_groups = B / pl->G;
+  pl->dck = B * dk;
+  if (d->num_ranges > 0) pl->R = d->num_ranges;
+  else {
+    if (sms <= 0) return MLRA_ERR_CUDA;
+    pl->R = sms / pl->n_groups > 0 ? sms / pl->n_groups : 1;
+  }
+  if ((int64_t)pl->R * pl->n_groups > INT_MAX / 2) return MLRA_ERR_INVALID_ARG;
+  pl->slots = (int64_t)pl->R + d->batch - 1;
+  pl->limit = paged ? d->max_pages_per_seq * d->page_size : d->max_seq_len;
+  if (!paged) pl->limit = d->max_seq_len;
+  else if (d->max_seq_len > 0 && d->max_seq_len < pl->limit) pl->limit = d->max_seq_len;
+
+  const int64_t N = d->batch, H = d->heads;
+  size_t off = kAlign;  // status word + padding
+  pl->off_lens = off; off = align_up(off + 4 * N);
+  pl->off_prefix = off; off = align_up(off + 4 * (N + 1));
+  pl->off_ml = off; off = align_up(off + (size_t)pl->slots * H * B * 2 * sizeof(float));
+  pl->off_o = off; off = align_up(off + (size_t)pl->slots * H * pl->dck * sizeof(float));
+  if (pl->repack) {
+    pl->off_rq = off; off = align_up(off + (size_t)N * H * pl->dck * 2);
+    pl->off_rqr = off; off = align_up(off + (size_t)N * H * 64 * 2);
+    pl->off_rc = off; off = align_up(off + (size_t)d->cache_rows * pl->dck * 2);
+    pl->off_rkr = off; off = align_up(off + (size_t)d->cache_rows * 64 * 2);
+  }
+  pl->total = off;
+  return MLRA_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link needed).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor map with 64 x 64 boxes and 128-byte swizzle.  dims/strides in elements.
+bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+              const uint64_t* strides_elems) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[3], gstride[2];
+  cuuint32_t box[3] = {64, 64, 1}, estr[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) gdim[i] = dims[i];
+  for (int i = 0; i + 1 < rank; ++i) gstride[i] = strides_elems[i] * 2;
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gdim, gstride, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int mlra_version(void) { return 0x000100; }
+
+const char* mlra_status_string(mlra_status s) {
+  switch (s) {
+    case MLRA_OK: return "MLRA_OK";
+    case MLRA_ERR_INVALID_ARG: return "MLRA_ERR_INVALID_ARG: invalid argument";
+    case MLRA_ERR_UNSUPPORTED: return "MLRA_ERR_UNSUPPORTED: shape or layout not supported";
+    case MLRA_ERR_CUDA: return "MLRA_ERR_CUDA: a CUDA call failed";
+    case MLRA_ERR_TIMEOUT: return "MLRA_ERR_TIMEOUT: a device-side wait ran out";
+    case MLRA_ERR_WORKSPACE: return "MLRA_ERR_WORKSPACE: workspace null, too small or misaligned";
+    case MLRA_ERR_BAD_PAGE: return "MLRA_ERR_BAD_PAGE: page id outside the cache pool";
+    case MLRA_ERR_BAD_LENGTH: return "MLRA_ERR_BAD_LENGTH: sequence length outside the cache";
+  }
+  return "MLRA: unknown status";
+}
+
+mlra_status mlra_workspace_size(const mlra_dims* dims, size_t* bytes_host) {
+  if (!dims || !bytes_host) return MLRA_ERR_INVALID_ARG;
+  const bool paged = dims->max_pages_per_seq > 0 && dims->page_size > 0;
+  int sms = 0;
+  if (dims->num_ranges == 0) {
+    mlra_status st;
+    sms = device_sm_count(&st);
+    if (st != MLRA_OK) return st;
+  }
+  Plan pl;
+  mlra_status st = make_plan(dims, paged, sms, &pl);
+  if (st != MLRA_OK) return st;
+  *bytes_host = pl.total;
+  return MLRA_OK;
+}
+
+mlra_status mlra_query_plan(const mlra_dims* dims, mlra_plan_info* info) {
+  if (!dims || !info) return MLRA_ERR_INVALID_ARG;
+  const bool paged = dims->max_pages_per_seq > 0 && dims->page_size > 0;
+  int sms = 0;
+  if (dims->num_ranges == 0) {
+    mlra_status st;
+    sms = device_sm_count(&st);
+    if (st != MLRA_OK) return st;
+  }
+  Plan pl;
+  mlra_status st = make_plan(dims, paged, sms, &pl);
+  if (st != MLRA_OK) return st;
+  info->repack = pl.repack ? 1 : 0;
+  info->launches = 3 + (pl.repack ? 1 : 0);
+  info->num_ranges = pl.R;
+  info->ctas = pl.R * pl.n_groups;
+  info->kernel_branch_width = pl.dblk_k;
+  info->branches_per_cta = pl.G;
+  info->partial_slots = pl.slots;
+  info->workspace_bytes = pl.total;
+  return MLRA_OK;
+}
+
+mlra_status mlra_decode(const void* q_lat, const void* q_rope, const void* c_kv, const void* k_rope,
+                        const int32_t* seq_lens, const int32_t* page_table, int B,
+                        const mlra_scales* scales, float* out, float* lse, const mlra_dims* dims,
+                        void* workspace, size_t ws_bytes, mlra_stream_t stream) {
+  return mlra_decode_profiled(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table, B, scales, out,
+                              lse, dims, workspace, ws_bytes, stream, nullptr, nullptr);
+}
+
+mlra_status mlra_decode_profiled(const void* q_lat, const void* q_rope, const void* c_kv,
+                                 const void* k_rope, const int32_t* seq_lens,
+                                 const int32_t* page_table, int B, const mlra_scales* scales,
+                                 float* out, float* lse, const mlra_dims* dims, void* workspace,
+                                 size_t ws_bytes, mlra_stream_t stream, mlra_event_t k1_begin,
+                                 mlra_event_t k1_end) {
+  if (!q_lat || !q_rope || !c_kv || !k_rope || !seq_lens || !scales || !out || !dims)
+    return MLRA_ERR_INVALID_ARG;
+  if (B != dims->num_branches) return MLRA_ERR_INVALID_ARG;
+  if (!std::isfinite(scales->softmax_scale) || !std::isfinite(scales->branch_scale))
+    return MLRA_ERR_INVALID_ARG;
+  const bool paged = page_table != nullptr;
+  mlra_status st = check_dims(dims, paged);
+  if (st != MLRA_OK) return st;
+  int sms = 0;
+  if (dims->num_ranges == 0) {
+    sms = device_sm_count(&st);
+    if (st != MLRA_OK) return st;
+  }
+  Plan pl;
+  st = make_plan(dims, paged, sms, &pl);
+  if (st != MLRA_OK) return st;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || ws_bytes < pl.total)
+    return MLRA_ERR_WORKSPACE;
+  if (!pl.repack && !(aligned16(q_lat) && aligned16(q_rope) && aligned16(c_kv) && aligned16(k_rope)))
+    return MLRA_ERR_UNSUPPORTED;
+  if (!aligned16(out)) return MLRA_ERR_UNSUPPORTED;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  int32_t* lens = reinterpret_cast<int32_t*>(ws + pl.off_lens);
+  int32_t* prefix = reinterpret_cast<int32_t*>(ws + pl.off_prefix);
+  float* part_ml = reinterpret_cast<float*>(ws + pl.off_ml);
+  float* part_o = reinterpret_cast<float*>(ws + pl.off_o);
+  const int N = dims->batch, H = dims->heads, dblk = dims->d_latent / B;
+  const int64_t rows = dims->cache_rows;
+
+  const void* kq = q_lat; const void* kqr = q_rope; const void* kc = c_kv; const void* kkr = k_rope;
+  int64_t c_pitch = dims->c_row_stride, kr_pitch = dims->kr_row_stride, q_width = dims->d_latent;
+  if (pl.repack) {
+    RepackParams rp;
+    rp.q_lat = q_lat; rp.q_rope = q_rope; rp.c_kv = c_kv; rp.k_rope = k_rope;
+    rp.q_out = reinterpret_cast<uint16_t*>(ws + pl.off_rq);
+    rp.qr_out = reinterpret_cast<uint16_t*>(ws + pl.off_rqr);
+    rp.c_out = reinterpret_cast<uint16_t*>(ws + pl.off_rc);
+    rp.kr_out = reinterpret_cast<uint16_t*>(ws + pl.off_rkr);
+    rp.N = N; rp.H = H; rp.B = B; rp.d_blk = dblk; rp.dblk_k = pl.dblk_k; rp.d_rope = dims->d_rope;
+    rp.rows = rows; rp.c_row_stride = dims->c_row_stride; rp.kr_row_stride = dims->kr_row_stride;
+    rp.src_f32 = dims->dtype == MLRA_F32;
+    if (launch_repack(rp, s) != cudaSuccess) return MLRA_ERR_CUDA;
+    kq = rp.q_out; kqr = rp.qr_out; kc = rp.c_out; kkr = rp.kr_out;
+    c_pitch = pl.dck; kr_pitch = 64; q_width = pl.dck;
+  }
+
+  CUtensorMap tq, tqr, tc, tkr;
+  {
+    const uint64_t dq[3] = {(uint64_t)q_width, (uint64_t)H, (uint64_t)N};
+    const uint64_t sq[2] = {(uint64_t)q_width, (uint64_t)q_width * H};
+    const uint64_t dqr[3] = {64, (uint64_t)H, (uint64_t)N};
+    const uint64_t sqr[2] = {64, (uint64_t)64 * H};
+    const uint64_t dcm[2] = {(uint64_t)q_width, (uint64_t)rows};
+    const uint64_t scm[1] = {(uint64_t)c_pitch};
+    const uint64_t dkr[2] = {64, (uint64_t)rows};
+    const uint64_t skr[1] = {(uint64_t)kr_pitch};
+    if (!make_map(&tq, kq, 3, dq, sq) || !make_map(&tqr, kqr, 3, dqr, sqr) ||
+        !make_map(&tc, kc, 2, dcm, scm) || !make_map(&tkr, kkr, 2, dkr, skr))
+      return MLRA_ERR_CUDA;
+  }
+
+  if (launch_prep(seq_lens, N, pl.limit, lens, prefix, status, s) != cudaSuccess) return MLRA_ERR_CUDA;
+
+  DecodeParams p;
+  p.lens = lens; p.prefix = prefix; p.page_table = page_table;
+  const bool summed = dims->out_mode == MLRA_OUT_SUMMED;
+  p.out = out; p.lse = lse; p.part_o = part_o; p.part_ml = part_ml; p.status = status;
+  p.N = N; p.H = H; p.B = B; p.d_blk_out = dblk; p.out_width = dims->d_latent; p.dck = pl.dck;
+  p.n_groups = pl.n_groups; p.num_ranges = pl.R;
+  p.page_size = paged ? dims->page_size : 0;
+  p.max_pages = paged ? dims->max_pages_per_seq : 0;
+  p.max_seq_len = dims->max_seq_len;
+  p.n_pages = paged ? rows / dims->page_size : 0;
+  p.oob_row = static_cast<int>(rows);
+  p.scale_log2 = scales->softmax_scale * 1.4426950408889634f;
+  p.gamma = scales->branch_scale;
+  p.write_final = summed ? 0 : 1;
+  p.timeout_ns = kTimeoutNs;
+  if (k1_begin && cudaEventRecord(reinterpret_cast<cudaEvent_t>(k1_begin), s) != cudaSuccess)
+    return MLRA_ERR_CUDA;
+  if (launch_decode(pl.variant, tq, tqr, tc, tkr, p, pl.R * pl.n_groups, s) != cudaSuccess)
+    return MLRA_ERR_CUDA;
+  if (k1_end && cudaEventRecord(reinterpret_cast<cudaEvent_t>(k1_end), s) != cudaSuccess)
+    return MLRA_ERR_CUDA;
+
+  CombineParams cp;
+  cp.prefix = prefix; cp.part_o = part_o; cp.part_ml = part_ml; cp.out = out; cp.lse = lse;
+  cp.N = N; cp.H = H; cp.B = B; cp.dblk_k = pl.dblk_k; cp.dck = pl.dck; cp.d_blk_out = dblk;
+  cp.num_ranges = pl.R; cp.summed = summed ? 1 : 0; cp.final_written = summed ? 0 : 1;
+  cp.gamma = scales->branch_scale;
+  if (launch_combine(cp, s) != cudaSuccess) return MLRA_ERR_CUDA;
+  return MLRA_OK;
+}
+
+mlra_status mlra_read_status(const void* workspace, mlra_stream_t stream, uint32_t* flags_host) {
+  if (!workspace || !flags_host) return MLRA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t f = 0;
+  if (cudaMemcpyAsync(&f, workspace, sizeof(f), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return MLRA_ERR_CUDA;
+  *flags_host = f;
+  if (f & kFlagTimeout) return MLRA_ERR_TIMEOUT;
+  if (f & kFlagBadPage) return MLRA_ERR_BAD_PAGE;
+  if (f & kFlagBadLength) return MLRA_ERR_BAD_LENGTH;
+  return MLRA_OK;
+}
+
+mlra_status mlra_debug_resolve_rows(const int32_t* seq_lens, const int32_t* page_table,
+                                    const mlra_dims* dims, int64_t* rows_out, int row_pitch,
+                                    mlra_stream_t stream) {
+  if (!seq_lens || !rows_out || row_pitch < 0) return MLRA_ERR_INVALID_ARG;
+  const bool paged = page_table != nullptr;
+  mlra_status st = check_dims(dims, paged);
+  if (st != MLRA_OK) return st;
+  const int64_t rows = dims->cache_rows;
+  if (launch_resolve_rows(nullptr, seq_lens, page_table, dims->batch,
+                          paged ? dims->max_pages_per_seq : 0, paged ? dims->page_size : 0,
+                          dims->max_seq_len, paged ? rows / dims->page_size : 0,
+                          static_cast<int>(rows), rows_out, row_pitch,
+                          reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MLRA_ERR_CUDA;
+  return MLRA_OK;
+}
+
+mlra_status mlra_plan_host(const int32_t* tiles_host, int n, int num_ranges,
+                           int32_t* first_range_host, int32_t* num_parts_host) {
+  if (!tiles_host || !first_range_host || !num_parts_host || n < 1 || num_ranges < 1)
+    return MLRA_ERR_INVALID_ARG;
+  std::vector<int32_t> prefix(n + 1, 0);
+  for (int i = 0; i < n; ++i) {
+    if (tiles_host[i] < 0) return MLRA_ERR_INVALID_ARG;
+    const int64_t next = (int64_t)prefix[i] + tiles_host[i];
+    if (next > INT_MAX) return MLRA_ERR_INVALID_ARG;
+    prefix[i + 1] = static_cast<int32_t>(next);
+  }
+  const int64_t total = prefix[n];
+  for (int s = 0; s < n; ++s) {
+    int r0 = 0, np = 0;
+    if (total > 0) seq_parts(prefix.data(), s, total, effective_ranges(num_ranges, total), &r0, &np);
+    first_range_host[s] = r0;
+    num_parts_host[s] = np;
+  }
+  return MLRA_OK;
+}
+
+mlra_status mlra_plan_segments_host(const int32_t* tiles_host, int n, int num_ranges,
+                                    int32_t* range_host, int32_t* seq_host, int32_t* tile0_host,
+                                    int32_t* ntiles_host, int max_segments, int* count_host) {
+  if (!tiles_host || !count_host || n < 1 || num_ranges < 1 || max_segments < 0)
+    return MLRA_ERR_INVALID_ARG;
+  std::vector<int32_t> prefix(n + 1, 0);
+  for (int i = 0; i < n; ++i) {
+    if (tiles_host[i] < 0) return MLRA_ERR_INVALID_ARG;
+    const int64_t next = (int64_t)prefix[i] + tiles_host[i];
+    if (next > INT_MAX) return MLRA_ERR_INVALID_ARG;
+    prefix[i + 1] = static_cast<int32_t>(next);
+  }
+  const int64_t total = prefix[n];
+  const int64_t R = effective_ranges(num_ranges, total);
+  int count = 0;
+  for (int r = 0; r < num_ranges; ++r) {
+    SegmentWalker walk(prefix.data(), n, total, R, r);
+    Segment seg;
+    while (walk.next(seg)) {
+      if (count < max_segments) {
+        if (range_host) range_host[count] = r;
+        if (seq_host) seq_host[count] = seg.seq;
+        if (tile0_host) tile0_host[count] = seg.tile0;
+        if (ntiles_host) ntiles_host[count] = seg.ntiles;
+      }
+      ++count;
+    }
+  }
+  *count_host = count;
+  return MLRA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,78 @@
+// mlra_internal.h -- declarations shared by the host API (mlra_api.cu) and the kernels
+// (mlra_kernels.cu).  Not part of the public C ABI.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace mlra {
+
+constexpr uint32_t kFlagTimeout = 0x1u;
+constexpr uint32_t kFlagBadPage = 0x2u;
+constexpr uint32_t kFlagBadLength = 0x4u;
+
+// Parameters of the split-KV decode kernel (K1).
+struct DecodeParams {
+  const int32_t* lens;        // clamped sequence lengths [N]
+  const int32_t* prefix;      // tile prefix sums [N + 1]
+  const int32_t* page_table;  // [N, max_pages] or nullptr (contiguous)
+  float* out;                 // final output, row width out_width, or nullptr
+  float* lse;                 // [N, H, B] or nullptr
+  float* part_o;              // partial outputs [slots, H, dck]
+  float* part_ml;             // partial (m, l) [slots, H, B, 2]
+  uint32_t* status;           // device status word
+  int N, H, B;
+  int d_blk_out;              // branch width of the caller's output
+  int out_width;              // row width of out (d_latent)
+  int dck;                    // latent width seen by the kernel (B * padded d_blk)
+  int n_groups;               // CTAs per work range (branch groups)
+  int num_ranges;
+  int page_size, max_pages, max_seq_len;
+  int64_t n_pages;            // pages in the pool (paged layout)
+  int oob_row;                // tile row used for an invalid page id (reads zeros)
+  float scale_log2;           // softmax_scale * log2(e)
+  float gamma;                // branch_scale
+  int write_final;            // whole-sequence segments write `out` directly
+  uint64_t timeout_ns;        // bound on every wait inside the kernel
+};
+
+struct CombineParams {
+  const int32_t* prefix;
+  const float* part_o;
+  const float* part_ml;
+  float* out;
+  float* lse;
+  int N, H, B;
+  int dblk_k, dck;            // kernel branch width and latent width
+  int d_blk_out;              // caller branch width
+  int num_ranges;
+  int summed;                 // 1: out[s,h,:d_blk_out] = sum over branches
+  int final_written;          // 1: sequences held in one part were written by K1
+  float gamma;
+};
+
+struct RepackParams {
+  const void* q_lat; const void* q_rope; const void* c_kv; const void* k_rope;
+  uint16_t* q_out; uint16_t* qr_out; uint16_t* c_out; uint16_t* kr_out;
+  int N, H, B, d_blk, dblk_k, d_rope;
+  int64_t rows, c_row_stride, kr_row_stride;
+  int src_f32;
+};
+
+// Kernel variants of K1: (padded branch width, branches per CTA).
+enum Variant { kV64x2 = 0, kV128x2, kV128x1, kV256x1, kV512x1, kNumVariants };
+
+int variant_smem_bytes(Variant v);
+cudaError_t launch_prep(const int32_t* seq_lens, int N, int limit, int32_t* lens_out,
+                        int32_t* prefix, uint32_t* status, cudaStream_t st);
+cudaError_t launch_decode(Variant v, const CUtensorMap& tq, const CUtensorMap& tqr,
+                          const CUtensorMap& tc, const CUtensorMap& tkr, const DecodeParams& p,
+                          int grid, cudaStream_t st);
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t st);
+cudaError_t launch_repack(const RepackParams& p, cudaStream_t st);
+cudaError_t launch_resolve_rows(const int32_t* lens_or_null, const int32_t* seq_lens,
+                                const int32_t* page_table, int N, int max_pages, int page_size,
+                                int max_seq_len, int64_t n_pages, int oob_row, int64_t* rows_out,
+                                int row_pitch, cudaStream_t st);
+
+}  // namespace mlra

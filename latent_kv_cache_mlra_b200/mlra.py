@@ -1,0 +1,270 @@
+"""ctypes binding of libmlra.so (declared in include/mlra.h).
+
+Argument marshalling only: every step of the decode runs in the library's CUDA kernels.
+PyTorch provides device memory and the current stream.  There is no fallback: if the
+library is missing, loading it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import pathlib
+from typing import Optional
+
+import torch
+
+LIB_PATH = pathlib.Path(__file__).resolve().parent / "libmlra.so"
+
+MLRA_OK, MLRA_ERR_INVALID_ARG, MLRA_ERR_UNSUPPORTED, MLRA_ERR_CUDA = 0, 1, 2, 3
+MLRA_ERR_TIMEOUT, MLRA_ERR_WORKSPACE, MLRA_ERR_BAD_PAGE, MLRA_ERR_BAD_LENGTH = 4, 5, 6, 7
+MLRA_BF16, MLRA_F32 = 0, 1
+MLRA_OUT_BRANCHES, MLRA_OUT_SUMMED = 0, 1
+FLAG_TIMEOUT, FLAG_BAD_PAGE, FLAG_BAD_LENGTH = 0x1, 0x2, 0x4
+
+# Every entry point of include/mlra.h.
+EXPORTS = ("mlra_workspace_size", "mlra_decode", "mlra_decode_profiled", "mlra_query_plan",
+           "mlra_read_status", "mlra_debug_resolve_rows", "mlra_plan_host",
+           "mlra_plan_segments_host", "mlra_status_string", "mlra_version")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("heads", ctypes.c_int), ("num_branches", ctypes.c_int),
+                ("d_latent", ctypes.c_int), ("d_rope", ctypes.c_int), ("page_size", ctypes.c_int),
+                ("max_pages_per_seq", ctypes.c_int), ("max_seq_len", ctypes.c_int),
+                ("cache_rows", ctypes.c_longlong), ("c_row_stride", ctypes.c_longlong),
+                ("kr_row_stride", ctypes.c_longlong), ("dtype", ctypes.c_int),
+                ("out_mode", ctypes.c_int), ("num_ranges", ctypes.c_int)]
+
+
+class Scales(ctypes.Structure):
+    _fields_ = [("softmax_scale", ctypes.c_float), ("branch_scale", ctypes.c_float)]
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [("repack", ctypes.c_int), ("launches", ctypes.c_int), ("num_ranges", ctypes.c_int),
+                ("ctas", ctypes.c_int), ("kernel_branch_width", ctypes.c_int),
+                ("branches_per_cta", ctypes.c_int), ("partial_slots", ctypes.c_longlong),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+
+class MlraError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises ImportError when it has not been built."""
+    global _lib
+    if _lib is None:
+        if not LIB_PATH.exists():
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m latent_kv_cache_mlra_b200.build` (needs nvcc)")
+        L = ctypes.CDLL(str(LIB_PATH))
+        vp, i32p, i64p, u32p = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32), \
+            ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_uint32)
+        L.mlra_workspace_size.argtypes = [ctypes.POINTER(Dims), ctypes.POINTER(ctypes.c_size_t)]
+        L.mlra_decode.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.POINTER(Scales),
+                                  vp, vp, ctypes.POINTER(Dims), vp, ctypes.c_size_t, vp]
+        L.mlra_decode_profiled.argtypes = L.mlra_decode.argtypes + [vp, vp]
+        L.mlra_query_plan.argtypes = [ctypes.POINTER(Dims), ctypes.POINTER(PlanInfo)]
+        L.mlra_read_status.argtypes = [vp, vp, u32p]
+        L.mlra_debug_resolve_rows.argtypes = [vp, vp, ctypes.POINTER(Dims), vp, ctypes.c_int, vp]
+        L.mlra_plan_host.argtypes = [i32p, ctypes.c_int, ctypes.c_int, i32p, i32p]
+        L.mlra_plan_segments_host.argtypes = [i32p, ctypes.c_int, ctypes.c_int, i32p, i32p, i32p,
+                                              i32p, ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
+        L.mlra_status_string.argtypes = [ctypes.c_int]
+        L.mlra_status_string.restype = ctypes.c_char_p
+        L.mlra_version.argtypes = []
+        for f in ("mlra_workspace_size", "mlra_decode", "mlra_decode_profiled", "mlra_query_plan",
+                  "mlra_read_status", "mlra_debug_resolve_rows", "mlra_plan_host",
+                  "mlra_plan_segments_host"):
+            getattr(L, f).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().mlra_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != MLRA_OK:
+        raise MlraError(status, what)
+
+
+def make_dims(*, batch, heads, num_branches, d_latent, d_rope, max_seq_len, cache_rows,
+              c_row_stride=None, kr_row_stride=None, page_size=0, max_pages_per_seq=0,
+              dtype="bf16", out_mode="branches", num_ranges=0) -> Dims:
+    return Dims(batch, heads, num_branches, d_latent, d_rope, page_size, max_pages_per_seq,
+                max_seq_len, cache_rows, c_row_stride if c_row_stride is not None else d_latent,
+                kr_row_stride if kr_row_stride is not None else d_rope,
+                MLRA_BF16 if dtype == "bf16" else MLRA_F32,
+                MLRA_OUT_BRANCHES if out_mode == "branches" else MLRA_OUT_SUMMED, num_ranges)
+
+
+def workspace_size(dims: Dims) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().mlra_workspace_size(ctypes.byref(dims), ctypes.byref(n)), "mlra_workspace_size")
+    return int(n.value)
+
+
+def query_plan(dims: Dims) -> PlanInfo:
+    info = PlanInfo()
+    _check(lib().mlra_query_plan(ctypes.byref(dims), ctypes.byref(info)), "mlra_query_plan")
+    return info
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def dims_for(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table, num_branches, *, max_seq_len=None,
+             page_size=0, out_mode="branches", num_ranges=0) -> Dims:
+    """mlra_dims from tensor shapes/strides (q tensors contiguous, cache rows strided)."""
+    N, H, d_c = q_lat.shape
+    d_R = q_rope.shape[-1]
+    if c_kv.stride(-1) != 1 or k_rope.stride(-1) != 1:
+        raise ValueError("cache rows must be contiguous in their last dimension")
+    dtype = {torch.bfloat16: "bf16", torch.float32: "f32"}[q_lat.dtype]
+    if page_table is None:
+        if max_seq_len is None:
+            max_seq_len = c_kv.shape[0] // N
+        return make_dims(batch=N, heads=H, num_branches=num_branches, d_latent=d_c, d_rope=d_R,
+                         max_seq_len=max_seq_len, cache_rows=c_kv.shape[0],
+                         c_row_stride=c_kv.stride(0), kr_row_stride=k_rope.stride(0), dtype=dtype,
+                         out_mode=out_mode, num_ranges=num_ranges)
+    max_pages = page_table.shape[1]
+    return make_dims(batch=N, heads=H, num_branches=num_branches, d_latent=d_c, d_rope=d_R,
+                     max_seq_len=max_seq_len if max_seq_len is not None else max_pages * page_size,
+                     cache_rows=c_kv.shape[0], c_row_stride=c_kv.stride(0),
+                     kr_row_stride=k_rope.stride(0), page_size=page_size,
+                     max_pages_per_seq=max_pages, dtype=dtype, out_mode=out_mode,
+                     num_ranges=num_ranges)
+
+
+def decode(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table=None, *, num_branches: int,
+           softmax_scale: float, branch_scale: Optional[float] = None, out_mode="branches",
+           max_seq_len=None, page_size=0, with_lse=False, out=None, lse=None, workspace=None,
+           num_ranges=0, stream=None):
+    """MLRA step-2 decode attention through ``mlra_decode``.  Returns (out, lse or None).
+
+    q_lat [N, H, d_c], q_rope [N, H, d_R] contiguous; c_kv [rows, >=d_c], k_rope [rows, >=d_R]
+    with unit inner stride (may be two column ranges of one tensor); seq_lens int32 [N];
+    page_table int32 [N, max_pages] or None.  All on the same CUDA device.
+    """
+    gamma = 1.0 / num_branches if branch_scale is None else branch_scale
+    dims = dims_for(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table, num_branches,
+                    max_seq_len=max_seq_len, page_size=page_size, out_mode=out_mode,
+                    num_ranges=num_ranges)
+    N, H, d_c = q_lat.shape
+    width = d_c if out_mode == "branches" else d_c // num_branches
+    dev = q_lat.device
+    if out is None:
+        out = torch.empty(N, H, width, dtype=torch.float32, device=dev)
+    if with_lse and lse is None:
+        lse = torch.empty(N, H, num_branches, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(workspace_size(dims), dtype=torch.uint8, device=dev)
+    st = stream if stream is not None else torch.cuda.current_stream(dev).cuda_stream
+    scales = Scales(softmax_scale, gamma)
+    _check(lib().mlra_decode(_ptr(q_lat), _ptr(q_rope), _ptr(c_kv), _ptr(k_rope), _ptr(seq_lens),
+                             _ptr(page_table), num_branches, ctypes.byref(scales), _ptr(out),
+                             _ptr(lse), ctypes.byref(dims), _ptr(workspace), workspace.numel(),
+                             ctypes.c_void_p(st)), "mlra_decode")
+    return out, lse
+
+
+class Decoder:
+    """Holds the dims, a workspace and outputs for repeated decode calls on fixed shapes."""
+
+    def __init__(self, q_lat, q_rope, c_kv, k_rope, seq_lens, page_table=None, *, num_branches,
+                 softmax_scale, branch_scale=None, out_mode="branches", max_seq_len=None,
+                 page_size=0, with_lse=False, num_ranges=0):
+        self.num_branches = num_branches
+        self.scales = Scales(softmax_scale, 1.0 / num_branches if branch_scale is None else branch_scale)
+        self.dims = dims_for(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table, num_branches,
+                             max_seq_len=max_seq_len, page_size=page_size, out_mode=out_mode,
+                             num_ranges=num_ranges)
+        N, H, d_c = q_lat.shape
+        width = d_c if out_mode == "branches" else d_c // num_branches
+        dev = q_lat.device
+        self.out = torch.empty(N, H, width, dtype=torch.float32, device=dev)
+        self.lse = torch.empty(N, H, num_branches, dtype=torch.float32, device=dev) if with_lse else None
+        self.workspace = torch.empty(workspace_size(self.dims), dtype=torch.uint8, device=dev)
+        self.args = (q_lat, q_rope, c_kv, k_rope, seq_lens, page_table)
+
+        self.plan = query_plan(self.dims)
+
+    def __call__(self, stream=None, args=None, k1_events=None):
+        """One decode call.  ``k1_events`` = (begin, end) torch.cuda.Event pair recorded around
+        the attention kernel on the launch stream."""
+        q_lat, q_rope, c_kv, k_rope, seq_lens, page_table = self.args if args is None else args
+        st = stream if stream is not None else torch.cuda.current_stream(q_lat.device).cuda_stream
+        common = (_ptr(q_lat), _ptr(q_rope), _ptr(c_kv), _ptr(k_rope), _ptr(seq_lens),
+                  _ptr(page_table), self.num_branches, ctypes.byref(self.scales), _ptr(self.out),
+                  _ptr(self.lse), ctypes.byref(self.dims), _ptr(self.workspace),
+                  self.workspace.numel(), ctypes.c_void_p(st))
+        if k1_events is None:
+            _check(lib().mlra_decode(*common), "mlra_decode")
+        else:
+            _check(lib().mlra_decode_profiled(*common, ctypes.c_void_p(k1_events[0].cuda_event),
+                                              ctypes.c_void_p(k1_events[1].cuda_event)),
+                   "mlra_decode_profiled")
+        return self.out
+
+    def status(self, stream=None):
+        """(status code, flag bits) left by the last call; synchronises the stream."""
+        flags = ctypes.c_uint32(0)
+        st = stream if stream is not None else torch.cuda.current_stream(self.out.device).cuda_stream
+        rc = lib().mlra_read_status(_ptr(self.workspace), ctypes.c_void_p(st), ctypes.byref(flags))
+        return rc, flags.value
+
+
+def read_status(workspace: torch.Tensor, stream=None):
+    flags = ctypes.c_uint32(0)
+    st = stream if stream is not None else torch.cuda.current_stream(workspace.device).cuda_stream
+    rc = lib().mlra_read_status(_ptr(workspace), ctypes.c_void_p(st), ctypes.byref(flags))
+    return rc, flags.value
+
+
+def resolve_rows(seq_lens, page_table, dims: Dims, row_pitch: int, stream=None) -> torch.Tensor:
+    """Test hook: cache row of every position, computed by the decode kernel's addressing."""
+    N = dims.batch
+    rows = torch.full((N, row_pitch), -1, dtype=torch.int64, device=seq_lens.device)
+    st = stream if stream is not None else torch.cuda.current_stream(seq_lens.device).cuda_stream
+    _check(lib().mlra_debug_resolve_rows(_ptr(seq_lens), _ptr(page_table), ctypes.byref(dims),
+                                         _ptr(rows), row_pitch, ctypes.c_void_p(st)),
+           "mlra_debug_resolve_rows")
+    return rows
+
+
+def plan_host(tiles, num_ranges: int):
+    """Host replica of the split plan: (first range, number of parts) per sequence."""
+    n = len(tiles)
+    arr = (ctypes.c_int32 * n)(*[int(t) for t in tiles])
+    first, parts = (ctypes.c_int32 * n)(), (ctypes.c_int32 * n)()
+    _check(lib().mlra_plan_host(arr, n, num_ranges, first, parts), "mlra_plan_host")
+    return list(first), list(parts)
+
+
+def plan_segments_host(tiles, num_ranges: int):
+    """Host replica of the kernel's per-CTA segment walk: list of (range, seq, tile0, ntiles)."""
+    n = len(tiles)
+    arr = (ctypes.c_int32 * n)(*[int(t) for t in tiles])
+    count = ctypes.c_int(0)
+    _check(lib().mlra_plan_segments_host(arr, n, num_ranges, None, None, None, None, 0,
+                                         ctypes.byref(count)), "mlra_plan_segments_host")
+    m = count.value
+    bufs = [(ctypes.c_int32 * max(m, 1))() for _ in range(4)]
+    _check(lib().mlra_plan_segments_host(arr, n, num_ranges, *bufs, m, ctypes.byref(count)),
+           "mlra_plan_segments_host")
+    return [tuple(b[i] for b in bufs) for i in range(m)]
+
+
+def default_scales(num_branches: int, d_rope: int, head_dim: int = 128):
+    """(sigma, gamma) = (1/sqrt(d_h + d_R), 1/B)."""
+    return 1.0 / math.sqrt(head_dim + d_rope), 1.0 / num_branches

@@ -85,8 +85,13 @@ def _apply_probs(p: np.ndarray, c_blk: np.ndarray) -> np.ndarray:
 
 
 def _gather(seq_len, s, c_kv, k_rope, page_table, page_size, max_seq_len):
+    """The sequence's cache rows, converted to float64 after gathering (tensor or array)."""
     rows = resolve_rows(seq_len, s, page_table, page_size, max_seq_len)
-    return c_kv[rows], k_rope[rows]
+    if hasattr(c_kv, "detach"):
+        import torch
+        idx = torch.from_numpy(rows)
+        return to_f64(c_kv[idx]), to_f64(k_rope[idx])
+    return to_f64(np.asarray(c_kv)[rows]), to_f64(np.asarray(k_rope)[rows])
 
 
 def decode_heads(q_lat_s, q_rope_s, c_rows, kr_rows, num_branches, sigma, gamma,
@@ -129,7 +134,6 @@ def decode(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table, num_branches, sigm
     subset (default: all).  Returns (out [n, h, ...], lse [n, h, B]) in float64.
     """
     q_lat, q_rope = to_f64(q_lat), to_f64(q_rope)
-    c_kv, k_rope = to_f64(c_kv), to_f64(k_rope)
     lens = np.asarray(seq_lens.tolist() if hasattr(seq_lens, "tolist") else seq_lens, dtype=np.int64)
     pt = None if page_table is None else np.asarray(
         page_table.tolist() if hasattr(page_table, "tolist") else page_table, dtype=np.int64)
