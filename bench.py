@@ -306,6 +306,10 @@ def run_ours(args):
 
     k1 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
+    for a, b in k1:  # torch creates the CUDA event on its first record; the library re-records it
+        a.record(stream)
+        b.record(stream)
+    torch.cuda.synchronize()
     t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         barrier(world)
