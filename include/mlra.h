@@ -145,7 +145,8 @@ typedef struct {
   int num_ranges;         /* equal work ranges the batch's KV tiles are cut into */
   int ctas;               /* CTAs of the attention kernel (ranges x branch groups) */
   int kernel_branch_width;/* branch width after padding (64, 128, 256 or 512) */
-  int branches_per_cta;   /* 1 or 2 */
+  int branches_per_cta;   /* branches whose latent columns one attention CTA reads */
+  int tile;               /* KV positions per tile (64 or 128) */
   long long partial_slots;/* partial-result slots in the workspace (num_ranges + N - 1) */
   size_t workspace_bytes;
 } mlra_plan_info;

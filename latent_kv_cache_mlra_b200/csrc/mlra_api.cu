@@ -25,10 +25,10 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct Plan {
   bool repack = false;
-  Variant variant = kV128x2;
+  Variant variant = kV128;
   int dblk_k = 0;      // padded branch width seen by the kernel
-  int G = 2;           // branches per CTA
-  int n_groups = 1;    // CTAs per range
+  int tile = 0;        // KV positions per tile
+  int n_groups = 1;    // CTAs per range (one per branch)
   int dck = 0;         // B * dblk_k
   int R = 0;           // work ranges
   int64_t slots = 0;   // partial slots = R + N - 1
@@ -76,19 +76,16 @@ mlra_status make_plan(const mlra_dims* d, bool paged, int sms, Plan* pl) {
   mlra_status st = check_dims(d, paged);
   if (st != MLRA_OK) return st;
   const int B = d->num_branches, dblk = d->d_latent / B;
-  int dk = dblk <= 64 ? 64 : dblk <= 128 ? 128 : dblk <= 256 ? 256 : 512;
-  if (dk == 64 && B % 2 != 0) dk = 128;
+  const int dk = dblk <= 64 ? 64 : dblk <= 128 ? 128 : dblk <= 256 ? 256 : 512;
   if (B * dk > 512) return MLRA_ERR_UNSUPPORTED;
   const bool inplace_shape = (dk == dblk) && d->d_rope == 64;
   const bool inplace_align = d->c_row_stride % 8 == 0 && d->kr_row_stride % 8 == 0;
   if (d->dtype == MLRA_BF16 && inplace_shape && !inplace_align) return MLRA_ERR_UNSUPPORTED;
   pl->repack = !(d->dtype == MLRA_BF16 && inplace_shape);
   pl->dblk_k = dk;
-  if (dk == 64) { pl->variant = kV64x2; pl->G = 2; }
-  else if (dk == 128) { pl->variant = (B % 2 == 0) ? kV128x2 : kV128x1; pl->G = (B % 2 == 0) ? 2 : 1; }
-  else if (dk == 256) { pl->variant = kV256x1; pl->G = 1; }
-  else { pl->variant = kV512x1; pl->G = 1; }
-  pl->n_groups = B / pl->G;
+  pl->variant = dk == 64 ? kV64 : dk == 128 ? kV128 : dk == 256 ? kV256 : kV512;
+  pl->tile = variant_tile(pl->variant);
+  pl->n_groups = B;
   pl->dck = B * dk;
   if (d->num_ranges > 0) pl->R = d->num_ranges;
   else {
@@ -205,7 +202,8 @@ mlra_status mlra_query_plan(const mlra_dims* dims, mlra_plan_info* info) {
   info->num_ranges = pl.R;
   info->ctas = pl.R * pl.n_groups;
   info->kernel_branch_width = pl.dblk_k;
-  info->branches_per_cta = pl.G;
+  info->branches_per_cta = 1;
+  info->tile = pl.tile;
   info->partial_slots = pl.slots;
   info->workspace_bytes = pl.total;
   return MLRA_OK;
@@ -289,7 +287,8 @@ mlra_status mlra_decode_profiled(const void* q_lat, const void* q_rope, const vo
       return MLRA_ERR_CUDA;
   }
 
-  if (launch_prep(seq_lens, N, pl.limit, lens, prefix, status, s) != cudaSuccess) return MLRA_ERR_CUDA;
+  if (launch_prep(seq_lens, N, pl.limit, pl.tile, lens, prefix, status, s) != cudaSuccess)
+    return MLRA_ERR_CUDA;
 
   DecodeParams p;
   p.lens = lens; p.prefix = prefix; p.page_table = page_table;
@@ -316,7 +315,8 @@ mlra_status mlra_decode_profiled(const void* q_lat, const void* q_rope, const vo
   CombineParams cp;
   cp.prefix = prefix; cp.part_o = part_o; cp.part_ml = part_ml; cp.out = out; cp.lse = lse;
   cp.N = N; cp.H = H; cp.B = B; cp.dblk_k = pl.dblk_k; cp.dck = pl.dck; cp.d_blk_out = dblk;
-  cp.num_ranges = pl.R; cp.summed = summed ? 1 : 0; cp.final_written = summed ? 0 : 1;
+  cp.num_ranges = pl.R; cp.max_parts = pl.R; cp.summed = summed ? 1 : 0;
+  cp.final_written = summed ? 0 : 1;
   cp.gamma = scales->branch_scale;
   if (launch_combine(cp, s) != cudaSuccess) return MLRA_ERR_CUDA;
   return MLRA_OK;

@@ -5,24 +5,25 @@
 // scores of the absorbed query block against latent block c_b plus the shared RoPE term,
 // an online softmax of its own over positions, and the probability-weighted sum of c_b.
 //
-// One persistent CTA per (work range, branch group).  A work range is a contiguous run of KV
-// tiles (64 positions) of the batch (see mlra_plan.cuh); a branch group is G branches whose
-// latent columns the CTA reads.  Heads are the M = 64 rows of every tcgen05 MMA:
-//   score:  S_b[64 x T]  = Q~_b[64 x d_blk] . C_b^T  +  Q^R[64 x 64] . K^R^T   (TMEM, fp32)
-//   output: O_b[64 x d]  += P_b[64 x T] . C_b[T x d]                             (TMEM, fp32)
-// The RoPE product is accumulated into every branch's score tile by the same MMA chain.
+// One persistent CTA per (work range, branch).  A work range is a contiguous run of KV tiles
+// (T positions each) of the batch (see mlra_plan.cuh).  Heads are the M = 64 rows of every
+// tcgen05 MMA, the tile's T positions the N of the score product:
+//   score:  S[64 x T]     = Q~_b[64 x d] . C_b^T  +  Q^R[64 x 64] . K^R^T     (TMEM, fp32)
+//   output: O[64 x d]    += P[64 x T] . C_b[T x d]                           (TMEM, fp32)
+// The RoPE product is accumulated into the same score tile by the MMA chain.  An MMA costs at
+// least ~57 cycles and N/2 cycles for N >= 128, so T = 128 keeps the score products efficient.
 //
-// TMEM: an M = 64 accumulator occupies 16 of the 32 lanes of each sub-partition; two
-// accumulators share columns in the lower (lanes 0-15) and upper (lanes 16-31) halves.
-//   G = 2: half x holds branch x of the group: O_x in columns [0, d_blk), S_x in two
-//          buffers of 64 columns after it.
-//   G = 1: the single branch is split by half: half x holds output columns
-//          [x d_blk/2, (x+1) d_blk/2) and the scores of tile positions [32x, 32x+32).
-// Softmax thread (warp w < 4, lane l) owns TMEM lane 32w + l: head 16w + (l & 15), half l >> 4.
+// TMEM.  An M = 64 accumulator occupies 16 of the 32 lanes of each sub-partition (rows 16k..16k+15
+// in lanes 32k + [0,16) + 16h for lane half h).  O is cut into chunks of up to 128 columns: chunk
+// j lives in lane half j % 2 at columns 128 (j / 2); score buffers follow in lane half 0.
+//
+// Shared memory: the branch's queries (per segment), an NS-deep ring of cache tiles
+// [latent blocks | RoPE block].  Once the score MMA of a tile has completed, the tile's RoPE block
+// is dead and the softmax writes the bf16 probabilities P of that tile into it.
 //
 // Warp roles (192 threads): warps 0-3 softmax / rescale / epilogue, warp 4 TMA producer,
-// warp 5 MMA issuer and TMEM owner.  Shared memory: the group's queries (resident per
-// segment), an NS-deep ring of cache tiles, NP probability buffers, mbarriers.
+// warp 5 MMA issuer and TMEM owner.  Softmax warp w owns heads 16w..16w+15; the thread pair
+// (l, l ^ 16) shares head 16w + (l & 15) and splits every row's columns between them.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -34,33 +35,33 @@
 
 namespace mlra {
 
-template <int DBLK, int G, int NS, int NP>
+template <int DBLK, int T, int NS>
 struct DecodeCfg {
-  static constexpr int T = kTile;
-  static constexpr int DG = DBLK * G;               // latent columns per CTA
-  static constexpr int NCB = DG / 64;               // 64-column boxes of latent per tile
+  static constexpr int NCB = DBLK / 64;             // 64-column latent blocks
+  static constexpr int TB = T / 64;                 // 64-row sub-boxes per tile
   static constexpr int BOX = 64 * 64 * 2;           // one [64 x 64] bf16 box, 8 KB
-  static constexpr int STAGE = (NCB + 1) * BOX;     // latent boxes + RoPE box
-  static constexpr int QBYTES = (NCB + 1) * BOX;    // query boxes + RoPE-query box
-  static constexpr int PBYTES = G * BOX;            // P_g [64 heads x 64 positions] bf16
-  static constexpr int O_COLS = (G == 2) ? DBLK : DBLK / 2;
-  static constexpr int S_COLS = (G == 2) ? T : T / 2;
-  static constexpr int N_SCORE = S_COLS;
-  static constexpr int N_PV = O_COLS;
-  static constexpr int TMEM_USED = O_COLS + 2 * S_COLS;
+  static constexpr int CBLK = T * 128;              // one 64-column block of a tile (T rows)
+  static constexpr int STAGE = (NCB + 1) * CBLK;    // latent blocks + RoPE block (later P)
+  static constexpr int QBYTES = (NCB + 1) * BOX;    // query blocks + RoPE-query block
+  static constexpr int OCW = DBLK < 128 ? DBLK : 128;   // O chunk width (columns)
+  static constexpr int OCH = DBLK / OCW;                // O chunks
+  static constexpr int O_COLS = ((OCH + 1) / 2) * OCW;  // TMEM columns used by O
+  static constexpr int NSB_TMEM = (512 - O_COLS) / T;
+  static constexpr int NSB = NSB_TMEM < 3 ? NSB_TMEM : (NS < 3 ? NS : 3);  // score buffers
+  static constexpr int NPV = NSB;                   // ring of output-MMA completion barriers
+  static constexpr int TMEM_USED = O_COLS + NSB * T;
   static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 :
                                    TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_STAGE = QBYTES;
-  static constexpr int OFF_P = OFF_STAGE + NS * STAGE;
-  static constexpr int OFF_BAR = OFF_P + NP * PBYTES;
-  static constexpr int NBAR = 2 * NS + 9;
+  static constexpr int OFF_BAR = OFF_STAGE + NS * STAGE;
+  static constexpr int NBAR = 2 * NS + 2 + 2 * NSB + NPV + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM + 1024;    // slack to align the base to 1024 B
-  static_assert(DBLK % 64 == 0 && (G == 1 || G == 2), "branch width must be a multiple of 64");
-  static_assert(G == 2 || DBLK >= 128, "single-branch CTAs need d_blk >= 128");
-  static_assert(N_PV % 8 == 0 && N_PV <= 256, "UMMA N must be a multiple of 8, at most 256");
+  static_assert(DBLK % 64 == 0 && DBLK <= 512, "branch width must be a multiple of 64, <= 512");
+  static_assert(T == 64 || T == 128, "tile of 64 or 128 positions");
+  static_assert(NSB >= 2 && NSB <= NS, "score buffers: at least 2, at most the stage count");
   static_assert(TMEM_USED <= 512, "TMEM budget");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
@@ -93,9 +94,9 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, uint64_
   return __all_sync(kFull, ok);
 }
 
-// First cache row of tile t (positions [64t, 64t+64)) of sequence s.  Shared by the decode
-// kernel and the row-resolution test hook.  An invalid page id flags the status word and
-// returns a row past the end of the cache, where TMA reads zeros.
+// First cache row of the 64-position block t (positions [64t, 64t+64)) of sequence s.  Shared by
+// the decode kernel and the row-resolution test hook.  An invalid page id flags the status word
+// and returns a row past the end of the cache, where TMA reads zeros.
 __device__ __forceinline__ int tile_row(const int32_t* page_table, int max_pages, int page_size,
                                         int max_seq_len, int64_t n_pages, int oob_row, int s,
                                         int t, uint32_t* status) {
@@ -109,38 +110,38 @@ __device__ __forceinline__ int tile_row(const int32_t* page_table, int max_pages
   return pid * page_size + j % page_size;
 }
 
-template <int DBLK, int G, int NS, int NP>
+template <int DBLK, int T, int NS>
 __global__ void __launch_bounds__(192, 1)
 mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
                    const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_kr,
                    const __grid_constant__ DecodeParams p) {
-  using C = DecodeCfg<DBLK, G, NS, NP>;
+  using C = DecodeCfg<DBLK, T, NS>;
+  constexpr int NSB = C::NSB, NPV = C::NPV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase + C::OFF_Q;
   const uint32_t sStage = sbase + C::OFF_STAGE;
-  const uint32_t sP = sbase + C::OFF_P;
   const uint32_t bar0 = sbase + C::OFF_BAR;
   // barrier map
-  const uint32_t bar_stage_full = bar0;                 // [NS]
-  const uint32_t bar_stage_empty = bar0 + 8 * NS;       // [NS]
-  const uint32_t bar_q_full = bar0 + 16 * NS;
-  const uint32_t bar_q_empty = bar_q_full + 8;
-  const uint32_t bar_s_full = bar_q_full + 16;          // [2]
-  const uint32_t bar_p_full = bar_q_full + 32;          // [2]
-  // PV of tile j commits to bar_pv_done[j & 1].  Two barriers keep every waiter within one
-  // phase of the phase it waits for (the commit before on the same barrier, PV of tile j-2, is
-  // known to be complete), which a parity wait needs to be unambiguous.
-  const uint32_t bar_pv_done = bar_q_full + 48;         // [2]
-  const uint32_t bar_final = bar_q_full + 64;
+  const uint32_t bar_stage_full = bar0;                     // [NS]  TMA -> MMA
+  const uint32_t bar_stage_empty = bar0 + 8 * NS;           // [NS]  MMA (PV done) -> TMA
+  const uint32_t bar_q_full = bar0 + 16 * NS;               //       TMA -> MMA
+  const uint32_t bar_q_empty = bar_q_full + 8;              //       MMA (last score) -> TMA
+  const uint32_t bar_s_full = bar_q_full + 16;              // [NSB] MMA (score) -> softmax
+  const uint32_t bar_p_full = bar_s_full + 8 * NSB;         // [NSB] softmax -> MMA
+  // PV of tile j commits to bar_pv_done[j % NPV].  When a thread waits for PV(j), PV(j - NPV)
+  // is known to be complete, so the barrier is within one phase of the one awaited and the
+  // parity wait is unambiguous.
+  const uint32_t bar_pv_done = bar_p_full + 8 * NSB;        // [NPV] MMA (PV) -> softmax
+  const uint32_t bar_final = bar_pv_done + 8 * NPV;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int range = blockIdx.x / p.n_groups;
-  const int group = blockIdx.x % p.n_groups;
+  const int branch = blockIdx.x % p.n_groups;
   const int64_t total = p.prefix[p.N];
   const int64_t R = effective_ranges(p.num_ranges, total);
   const uint64_t tmo = p.timeout_ns;
@@ -152,12 +153,11 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     mbar_init(bar_q_full, 1);
     mbar_init(bar_q_empty, 1);
-    mbar_init(bar_s_full, 1);
-    mbar_init(bar_s_full + 8, 1);
-    mbar_init(bar_p_full, 128);
-    mbar_init(bar_p_full + 8, 128);
-    mbar_init(bar_pv_done, 1);
-    mbar_init(bar_pv_done + 8, 1);
+    for (int k = 0; k < NSB; ++k) {
+      mbar_init(bar_s_full + 8 * k, 1);
+      mbar_init(bar_p_full + 8 * k, 128);
+    }
+    for (int k = 0; k < NPV; ++k) mbar_init(bar_pv_done + 8 * k, 1);
     mbar_init(bar_final, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -176,6 +176,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const int col0 = branch * DBLK;  // first latent column of this CTA's branch
 
   if (warp == 4) {
     // ------------------------------------------------------------------ TMA producer
@@ -183,7 +184,6 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     Segment seg;
     int it = 0, nseg = 0;
     bool ok = true;
-    const int col0 = group * C::DG;
     while (ok && walk.next(seg)) {
       if (nseg > 0) ok = wait_warp(bar_q_empty, (nseg - 1) & 1, tmo, abort_flag, p.status);
       if (!ok) break;
@@ -195,10 +195,18 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         tma_load_3d(sQ + C::NCB * C::BOX, &tm_qr, bar_q_full, 0, 0, seg.seq);
       }
       __syncwarp();
+      const int L = p.lens[seg.seq];
       for (int i = 0; i < seg.ntiles; ++i, ++it) {
-        const int row0 = tile_row(p.page_table, p.max_pages, p.page_size, p.max_seq_len,
-                                  p.n_pages, p.oob_row, seg.seq, seg.tile0 + i,
-                                  lane == 0 ? p.status : nullptr);
+        // cache rows of the tile's 64-position sub-boxes (past the sequence end: zeros)
+        int rows[C::TB];
+#pragma unroll
+        for (int l = 0; l < C::TB; ++l) {
+          const int t64 = (seg.tile0 + i) * C::TB + l;
+          rows[l] = (t64 * kTile < L)
+                        ? tile_row(p.page_table, p.max_pages, p.page_size, p.max_seq_len, p.n_pages,
+                                   p.oob_row, seg.seq, t64, lane == 0 ? p.status : nullptr)
+                        : p.oob_row;
+        }
         const int st = it % NS;
         if (it >= NS) {
           ok = wait_warp(bar_stage_empty + 8 * st, ((it / NS) - 1) & 1, tmo, abort_flag, p.status);
@@ -209,8 +217,12 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           const uint32_t dst = sStage + st * C::STAGE;
           mbar_arrive_expect_tx(full, C::STAGE);
 #pragma unroll
-          for (int k = 0; k < C::NCB; ++k) tma_load_2d(dst + k * C::BOX, &tm_c, full, col0 + 64 * k, row0);
-          tma_load_2d(dst + C::NCB * C::BOX, &tm_kr, full, 0, row0);
+          for (int l = 0; l < C::TB; ++l) {
+#pragma unroll
+            for (int k = 0; k < C::NCB; ++k)
+              tma_load_2d(dst + k * C::CBLK + l * C::BOX, &tm_c, full, col0 + 64 * k, rows[l]);
+            tma_load_2d(dst + C::NCB * C::CBLK + l * C::BOX, &tm_kr, full, 0, rows[l]);
+          }
         }
         __syncwarp();
       }
@@ -224,33 +236,36 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------------ MMA issuer
-    constexpr uint32_t kIdScore = idesc_bf16_f32(64, C::N_SCORE, false, false);
-    constexpr uint32_t kIdPV = idesc_bf16_f32(64, C::N_PV, false, true);
+    // Order: score of tile it, then the output products of every tile <= it - (NSB - 1), so the
+    // tensor core computes scores up to NSB - 1 tiles ahead of the softmax.
+    constexpr uint32_t kIdScore = idesc_bf16_f32(64, T, false, false);
+    constexpr uint32_t kIdPV = idesc_bf16_f32(64, C::OCW, false, true);
     SegmentWalker walk(p.prefix, p.N, total, R, range);
     Segment seg;
-    int it = 0, nseg = 0, prev = -1;
-    bool prev_first = false, ok = true;
+    int it = 0, nseg = 0, pv_next = 0;
+    uint32_t first_mask = 0;  // bit (j % 32): tile j is the first of its segment
+    bool ok = true;
 
-    auto issue_pv = [&](int j, bool first) -> bool {
-      if (!wait_warp(bar_p_full + 8 * (j & 1), (j >> 1) & 1, tmo, abort_flag, p.status)) return false;
+    auto issue_pv = [&](int j) -> bool {
+      if (!wait_warp(bar_p_full + 8 * (j % NSB), (j / NSB) & 1, tmo, abort_flag, p.status)) return false;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t pbuf = sP + (j % NP) * C::PBYTES;
+        const bool first = (first_mask >> (j & 31)) & 1u;
         const uint32_t stg = sStage + (j % NS) * C::STAGE;
+        const uint32_t pa = stg + C::NCB * C::CBLK;  // P lives in the tile's RoPE block
 #pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          const uint32_t d = tmem + ((uint32_t)(16 * x) << 16);
-          const uint32_t a0 = pbuf + (G == 2 ? x * C::BOX : 0);
-          const uint32_t b0 = stg + (G == 2 ? x * (DBLK / 64) : x * (DBLK / 128)) * C::BOX;
+        for (int ch = 0; ch < C::OCH; ++ch) {
+          const uint32_t d = tmem + ((uint32_t)(16 * (ch & 1)) << 16) + (ch >> 1) * C::OCW;
+          const uint32_t b0 = stg + ch * (C::OCW / 64) * C::CBLK;
 #pragma unroll
-          for (int kk = 0; kk < C::T / 16; ++kk) {
-            const uint64_t ad = sw128_desc(a0 + kk * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(b0 + kk * 2048, C::BOX, 1024);
+          for (int kk = 0; kk < T / 16; ++kk) {
+            const uint64_t ad = sw128_desc(pa + (kk >> 2) * C::BOX + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(b0 + kk * 2048, C::CBLK, 1024);
             umma_bf16(d, ad, bd, kIdPV, (kk > 0 || !first) ? 1u : 0u);
           }
         }
         umma_commit(bar_stage_empty + 8 * (j % NS));
-        umma_commit(bar_pv_done + 8 * (j & 1));
+        umma_commit(bar_pv_done + 8 * (j % NPV));
       }
       __syncwarp();
       return true;
@@ -260,71 +275,58 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       for (int i = 0; i < seg.ntiles; ++i, ++it) {
         if (i == 0) {
           // Finish the previous segment first so that its epilogue overlaps this query load.
-          if (prev >= 0) {
-            ok = issue_pv(prev, prev_first);
-            if (!ok) break;
-            prev = -1;
-          }
+          while (ok && pv_next < it) ok = issue_pv(pv_next++);
+          if (!ok) break;
           ok = wait_warp(bar_q_full, nseg & 1, tmo, abort_flag, p.status);
           if (!ok) break;
         }
         ok = wait_warp(bar_stage_full + 8 * (it % NS), (it / NS) & 1, tmo, abort_flag, p.status);
         if (!ok) break;
-        if (it >= 2) {
-          // score buffer (it & 1) is free once the softmax of tile it-2 has read it
-          ok = wait_warp(bar_p_full + 8 * (it & 1), ((it - 2) >> 1) & 1, tmo, abort_flag, p.status);
+        if (it >= NSB) {
+          // score buffer it % NSB is free once the softmax of tile it - NSB has read it
+          ok = wait_warp(bar_p_full + 8 * (it % NSB), ((it - NSB) / NSB) & 1, tmo, abort_flag, p.status);
           if (!ok) break;
         }
         tc_fence_after();
         if (lane == 0) {
           const uint32_t stg = sStage + (it % NS) * C::STAGE;
+          const uint32_t d = tmem + C::O_COLS + (it % NSB) * T;
 #pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            const uint32_t d = tmem + ((uint32_t)(16 * x) << 16) + C::O_COLS + (it & 1) * C::S_COLS;
-            const int box0 = (G == 2) ? x * (DBLK / 64) : 0;
-            const uint32_t brow = (G == 2) ? 0u : (uint32_t)x * 4096u;  // 32 rows of 128 B
-#pragma unroll
-            for (int kb = 0; kb < DBLK / 64; ++kb) {
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t ad = sw128_desc(sQ + (box0 + kb) * C::BOX + kk * 32, 16, 1024);
-                const uint64_t bd = sw128_desc(stg + (box0 + kb) * C::BOX + brow + kk * 32, 16, 1024);
-                umma_bf16(d, ad, bd, kIdScore, (kb | kk) ? 1u : 0u);
-              }
-            }
+          for (int kb = 0; kb < C::NCB; ++kb) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = sw128_desc(sQ + C::NCB * C::BOX + kk * 32, 16, 1024);
-              const uint64_t bd = sw128_desc(stg + C::NCB * C::BOX + brow + kk * 32, 16, 1024);
-              umma_bf16(d, ad, bd, kIdScore, 1u);
+              const uint64_t ad = sw128_desc(sQ + kb * C::BOX + kk * 32, 16, 1024);
+              const uint64_t bd = sw128_desc(stg + kb * C::CBLK + kk * 32, 16, 1024);
+              umma_bf16(d, ad, bd, kIdScore, (kb | kk) ? 1u : 0u);
             }
           }
-          umma_commit(bar_s_full + 8 * (it & 1));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = sw128_desc(sQ + C::NCB * C::BOX + kk * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(stg + C::NCB * C::CBLK + kk * 32, 16, 1024);
+            umma_bf16(d, ad, bd, kIdScore, 1u);
+          }
+          umma_commit(bar_s_full + 8 * (it % NSB));
           if (i == seg.ntiles - 1) umma_commit(bar_q_empty);
         }
         __syncwarp();
-        if (prev >= 0) {
-          ok = issue_pv(prev, prev_first);
-          if (!ok) break;
-        }
-        prev = it;
-        prev_first = (i == 0);
+        if (i == 0) first_mask |= 1u << (it & 31);
+        else first_mask &= ~(1u << (it & 31));
+        while (ok && pv_next <= it - (NSB - 1)) ok = issue_pv(pv_next++);
+        if (!ok) break;
       }
       ++nseg;
     }
-    if (ok && prev >= 0) issue_pv(prev, prev_first);
+    while (ok && pv_next < it) ok = issue_pv(pv_next++);
     // Nothing of ours may still run on the tensor core when TMEM is released.
     if (lane == 0) umma_commit(bar_final);
     __syncwarp();
     wait_warp(bar_final, 0, tmo, abort_flag, p.status, false);
   } else {
     // ------------------------------------------------------------------ softmax warps 0-3
-    const int half = lane >> 4;
-    const int h = 16 * warp + (lane & 15);
-    const int branch = (G == 2) ? group * 2 + half : group;
-    const uint32_t lane_addr = tmem + ((uint32_t)(32 * warp) << 16);
-    const int tok0 = (G == 2) ? 0 : 32 * half;       // first tile position of this thread's scores
-    const int ocol0 = (G == 2) ? 0 : half * (DBLK / 2);  // first output column of this thread
+    const int q = lane >> 4;                   // which half of the row's columns
+    const int h = 16 * warp + (lane & 15);     // head
+    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
     SegmentWalker walk(p.prefix, p.N, total, R, range);
     Segment seg;
     int it = 0;
@@ -334,27 +336,31 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       float m_used = -CUDART_INF_F, l_sum = 0.f;
       for (int i = 0; i < seg.ntiles; ++i, ++it) {
         const int t = seg.tile0 + i;
-        ok = wait_warp(bar_s_full + 8 * (it & 1), (it >> 1) & 1, tmo, abort_flag, p.status);
+        ok = wait_warp(bar_s_full + 8 * (it % NSB), (it / NSB) & 1, tmo, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
-        float v[C::S_COLS];
+        // this thread's scores: positions 64 l + 32 q + [0, 32) of the tile, l < T / 64
+        float v[C::TB][32];
 #pragma unroll
-        for (int c0 = 0; c0 < C::S_COLS; c0 += 32) {
+        for (int l = 0; l < C::TB; ++l) {
           uint32_t r[32];
-          tmem_ld32(lane_addr + C::O_COLS + (it & 1) * C::S_COLS + c0, r);
+          tmem_ld16x2_32(tmem + lane_base + C::O_COLS + (it % NSB) * T + 64 * l, r);
           tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 32; ++k) v[c0 + k] = __uint_as_float(r[k]);
+          for (int k = 0; k < 32; ++k) v[l][k] = __uint_as_float(r[k]);
         }
-        const int valid = min(C::T, L - C::T * t);
+        const int valid = min(T, L - T * t);
         float mx = -CUDART_INF_F;
 #pragma unroll
-        for (int c = 0; c < C::S_COLS; ++c) {
-          const float x = (tok0 + c < valid) ? v[c] * p.scale_log2 : -CUDART_INF_F;
-          v[c] = x;
-          mx = fmaxf(mx, x);
+        for (int l = 0; l < C::TB; ++l) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const float x = (64 * l + 32 * q + k < valid) ? v[l][k] * p.scale_log2 : -CUDART_INF_F;
+            v[l][k] = x;
+            mx = fmaxf(mx, x);
+          }
         }
-        if (G == 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
         bool rescale = false;
         float alpha = 1.f;
         if (i == 0) {
@@ -365,67 +371,68 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           rescale = true;
         }
         l_sum *= alpha;
-        const bool warp_rescale = __any_sync(kFull, rescale);
-        if ((warp_rescale || NP == 1) && it > 0) {
-          // O (rescale) and the single P buffer are only free once PV of tile it-1 is done
-          ok = wait_warp(bar_pv_done + 8 * ((it - 1) & 1), ((it - 1) >> 1) & 1, tmo, abort_flag,
+        if (__any_sync(kFull, rescale)) {
+          // O holds the output products up to tile it-1: wait for them, then scale O
+          ok = wait_warp(bar_pv_done + 8 * ((it - 1) % NPV), ((it - 1) / NPV) & 1, tmo, abort_flag,
                          p.status);
           if (!ok) break;
           tc_fence_after();
-        }
-        if (warp_rescale) {
 #pragma unroll 1
-          for (int c0 = 0; c0 < C::O_COLS; c0 += 32) {
-            uint32_t r[32];
-            tmem_ld32(lane_addr + c0, r);
-            tmem_wait_ld();
+          for (int ch = 0; ch < C::OCH; ++ch) {
+#pragma unroll 1
+            for (int c0 = 0; c0 < C::OCW; c0 += 64) {
+              const uint32_t a = tmem + ((uint32_t)(32 * warp + 16 * (ch & 1)) << 16) +
+                                 (ch >> 1) * C::OCW + c0;
+              uint32_t r[32];
+              tmem_ld16x2_32(a, r);
+              tmem_wait_ld();
 #pragma unroll
-            for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
-            tmem_st32(lane_addr + c0, r);
+              for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
+              tmem_st16x2_32(a, r);
+            }
           }
           tmem_wait_st();
         }
-        // probabilities -> bf16 P tile (K-major, 128-byte swizzle), row h
+        // probabilities -> bf16 P tile in the (consumed) RoPE block: K-major, 128-byte swizzle
+        uint8_t* stg = smem + C::OFF_STAGE + (it % NS) * C::STAGE;
         float sum = 0.f;
-        uint32_t pk[C::S_COLS / 2];
 #pragma unroll
-        for (int c = 0; c < C::S_COLS; c += 2) {
-          const float p0 = ex2_approx(v[c] - m_used);
-          const float p1 = ex2_approx(v[c + 1] - m_used);
-          sum += p0 + p1;
-          pk[c / 2] = pack_bf16x2(p0, p1);
-        }
-        if (G == 1) sum += __shfl_xor_sync(kFull, sum, 16);
-        l_sum += sum;
-        {
-          uint8_t* prow = smem + C::OFF_P + (it % NP) * C::PBYTES + (G == 2 ? half * C::BOX : 0) + h * 128;
+        for (int l = 0; l < C::TB; ++l) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int q = 0; q < C::S_COLS / 8; ++q) {
-            const int chunk = tok0 / 8 + q;
-            uint4 val = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-            *reinterpret_cast<uint4*>(prow + ((chunk ^ (h & 7)) << 4)) = val;
+          for (int k = 0; k < 32; k += 2) {
+            const float p0 = ex2_approx(v[l][k] - m_used);
+            const float p1 = ex2_approx(v[l][k + 1] - m_used);
+            sum += p0 + p1;
+            pk[k / 2] = pack_bf16x2(p0, p1);
+          }
+          uint8_t* prow = stg + C::NCB * C::CBLK + l * C::BOX + h * 128;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int chunk = 4 * q + c;
+            *reinterpret_cast<uint4*>(prow + ((chunk ^ (h & 7)) << 4)) =
+                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
           }
         }
-        if (valid < C::T) {
+        sum += __shfl_xor_sync(kFull, sum, 16);
+        l_sum += sum;
+        if (valid < T) {
           // Ragged last tile: zero the latent rows past the sequence end so that the zero
           // probabilities never multiply a non-finite value left in the cache.
-          ok = wait_warp(bar_stage_full + 8 * (it % NS), (it / NS) & 1, tmo, abort_flag, p.status);
-          if (!ok) break;
-          uint8_t* stg = smem + C::OFF_STAGE + (it % NS) * C::STAGE;
-          for (int k = threadIdx.x; k < C::NCB * 64 * 8; k += 128) {
-            const int row = (k >> 3) & 63;
+          for (int k = threadIdx.x; k < C::NCB * T * 8; k += 128) {
+            const int row = (k >> 3) % T;
             if (row >= valid)
-              *reinterpret_cast<uint4*>(stg + (k >> 9) * C::BOX + row * 128 + (k & 7) * 16) =
+              *reinterpret_cast<uint4*>(stg + (k / (T * 8)) * C::CBLK + row * 128 + (k & 7) * 16) =
                   make_uint4(0u, 0u, 0u, 0u);
           }
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(bar_p_full + 8 * (it & 1));
+        mbar_arrive(bar_p_full + 8 * (it % NSB));
       }
       if (!ok) break;
       // ------------------------------------------------ epilogue of the segment
-      ok = wait_warp(bar_pv_done + 8 * ((it - 1) & 1), ((it - 1) >> 1) & 1, tmo, abort_flag,
+      ok = wait_warp(bar_pv_done + 8 * ((it - 1) % NPV), ((it - 1) / NPV) & 1, tmo, abort_flag,
                      p.status);
       if (!ok) break;
       tc_fence_after();
@@ -445,27 +452,30 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         ncols_out = DBLK;
       }
 #pragma unroll 1
-      for (int c0 = 0; c0 < C::O_COLS; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(lane_addr + c0, r);
-        tmem_wait_ld();
-        if (live) {
-          const int cbase = ocol0 + c0;
-          if (cbase + 32 <= ncols_out && ((reinterpret_cast<uintptr_t>(dst + cbase)) & 15) == 0) {
+      for (int ch = 0; ch < C::OCH; ++ch) {
+#pragma unroll 1
+        for (int c0 = 0; c0 < C::OCW; c0 += 64) {
+          uint32_t r[32];
+          tmem_ld16x2_32(tmem + ((uint32_t)(32 * warp + 16 * (ch & 1)) << 16) + (ch >> 1) * C::OCW + c0, r);
+          tmem_wait_ld();
+          if (live) {
+            const int cbase = ch * C::OCW + c0 + 32 * q;
+            if (cbase + 32 <= ncols_out && ((reinterpret_cast<uintptr_t>(dst + cbase)) & 15) == 0) {
 #pragma unroll
-            for (int k = 0; k < 32; k += 4) {
-              float4 o4 = make_float4(__uint_as_float(r[k]) * scale, __uint_as_float(r[k + 1]) * scale,
-                                      __uint_as_float(r[k + 2]) * scale, __uint_as_float(r[k + 3]) * scale);
-              *reinterpret_cast<float4*>(dst + cbase + k) = o4;
+              for (int k = 0; k < 32; k += 4) {
+                float4 o4 = make_float4(__uint_as_float(r[k]) * scale, __uint_as_float(r[k + 1]) * scale,
+                                        __uint_as_float(r[k + 2]) * scale, __uint_as_float(r[k + 3]) * scale);
+                *reinterpret_cast<float4*>(dst + cbase + k) = o4;
+              }
+            } else {
+#pragma unroll
+              for (int k = 0; k < 32; ++k)
+                if (cbase + k < ncols_out) dst[cbase + k] = __uint_as_float(r[k]) * scale;
             }
-          } else {
-#pragma unroll
-            for (int k = 0; k < 32; ++k)
-              if (cbase + k < ncols_out) dst[cbase + k] = __uint_as_float(r[k]) * scale;
           }
         }
       }
-      if (live && (G == 2 || half == 0)) {
+      if (live && q == 0) {
         if (to_final) {
           if (p.lse) p.lse[((int64_t)seg.seq * p.H + h) * p.B + branch] = (m_used + __log2f(l_sum)) * 0.69314718055994531f;
         } else {

@@ -37,7 +37,7 @@ struct DecodeParams {
 };
 
 struct CombineParams {
-  const int32_t* prefix;
+  const int32_t* prefix;      // tile prefix sums [N + 1]
   const float* part_o;
   const float* part_ml;
   float* out;
@@ -46,6 +46,7 @@ struct CombineParams {
   int dblk_k, dck;            // kernel branch width and latent width
   int d_blk_out;              // caller branch width
   int num_ranges;
+  int max_parts;              // upper bound on the parts of one sequence (shared-memory sizing)
   int summed;                 // 1: out[s,h,:d_blk_out] = sum over branches
   int final_written;          // 1: sequences held in one part were written by K1
   float gamma;
@@ -59,11 +60,12 @@ struct RepackParams {
   int src_f32;
 };
 
-// Kernel variants of K1: (padded branch width, branches per CTA).
-enum Variant { kV64x2 = 0, kV128x2, kV128x1, kV256x1, kV512x1, kNumVariants };
+// Kernel variants of K1, one per padded branch width (one branch per CTA).
+enum Variant { kV64 = 0, kV128, kV256, kV512, kNumVariants };
 
 int variant_smem_bytes(Variant v);
-cudaError_t launch_prep(const int32_t* seq_lens, int N, int limit, int32_t* lens_out,
+int variant_tile(Variant v);  // KV positions per tile (64 or 128)
+cudaError_t launch_prep(const int32_t* seq_lens, int N, int limit, int tile, int32_t* lens_out,
                         int32_t* prefix, uint32_t* status, cudaStream_t st);
 cudaError_t launch_decode(Variant v, const CUtensorMap& tq, const CUtensorMap& tqr,
                           const CUtensorMap& tc, const CUtensorMap& tkr, const DecodeParams& p,

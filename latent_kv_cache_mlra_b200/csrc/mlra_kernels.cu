@@ -15,10 +15,10 @@ namespace mlra {
 
 // ----------------------------------------------------------------------------- K0
 // One block.  seq_lens outside [0, limit] set kFlagBadLength and are clamped; the status word
-// is rewritten first so that it reports this call only.
+// is rewritten so that it reports this call only.  prefix counts tiles of `tile` positions.
 __global__ void __launch_bounds__(1024) mlra_prep_kernel(const int32_t* seq_lens, int N, int limit,
-                                                         int32_t* lens_out, int32_t* prefix,
-                                                         uint32_t* status) {
+                                                         int tile, int32_t* lens_out,
+                                                         int32_t* prefix, uint32_t* status) {
   __shared__ int32_t warp_tot[32];
   __shared__ int32_t carry;
   __shared__ uint32_t flags;
@@ -39,7 +39,7 @@ __global__ void __launch_bounds__(1024) mlra_prep_kernel(const int32_t* seq_lens
         L = L < 0 ? 0 : limit;
       }
       lens_out[i] = L;
-      tiles = (L + kTile - 1) / kTile;
+      tiles = (L + tile - 1) / tile;
     }
     int x = tiles;  // inclusive warp scan
 #pragma unroll
@@ -68,36 +68,44 @@ __global__ void __launch_bounds__(1024) mlra_prep_kernel(const int32_t* seq_lens
   if (tid == 0) *status = flags;
 }
 
-cudaError_t launch_prep(const int32_t* seq_lens, int N, int limit, int32_t* lens_out,
+cudaError_t launch_prep(const int32_t* seq_lens, int N, int limit, int tile, int32_t* lens_out,
                         int32_t* prefix, uint32_t* status, cudaStream_t st) {
-  mlra_prep_kernel<<<1, 1024, 0, st>>>(seq_lens, N, limit, lens_out, prefix, status);
+  mlra_prep_kernel<<<1, 1024, 0, st>>>(seq_lens, N, limit, tile, lens_out, prefix, status);
   return cudaGetLastError();
 }
 
 // ----------------------------------------------------------------------------- K1
-template <int DBLK, int G, int NS, int NP>
+template <int DBLK, int T, int NS>
 static cudaError_t launch_decode_t(const CUtensorMap& tq, const CUtensorMap& tqr,
                                    const CUtensorMap& tc, const CUtensorMap& tkr,
                                    const DecodeParams& p, int grid, cudaStream_t st) {
-  using C = DecodeCfg<DBLK, G, NS, NP>;
-  auto kern = mlra_decode_kernel<DBLK, G, NS, NP>;
+  using C = DecodeCfg<DBLK, T, NS>;
+  auto kern = mlra_decode_kernel<DBLK, T, NS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
   kern<<<grid, 192, C::SMEM_ALLOC, st>>>(tq, tqr, tc, tkr, p);
   return cudaGetLastError();
 }
 
-// (padded branch width, branches per CTA, cache-tile stages, probability buffers)
-#define MLRA_VARIANTS(X)  \
-  X(kV64x2, 64, 2, 4, 2)  \
-  X(kV128x2, 128, 2, 3, 2) \
-  X(kV128x1, 128, 1, 4, 2) \
-  X(kV256x1, 256, 1, 3, 2) \
-  X(kV512x1, 512, 1, 2, 1)
+// (padded branch width, positions per tile, cache-tile stages)
+#define MLRA_VARIANTS(X) \
+  X(kV64, 64, 128, 4)    \
+  X(kV128, 128, 128, 4)  \
+  X(kV256, 256, 128, 2)  \
+  X(kV512, 512, 64, 2)
 
 int variant_smem_bytes(Variant v) {
   switch (v) {
-#define X(id, D, G, NS, NP) case id: return DecodeCfg<D, G, NS, NP>::SMEM_ALLOC;
+#define X(id, D, T, NS) case id: return DecodeCfg<D, T, NS>::SMEM_ALLOC;
+    MLRA_VARIANTS(X)
+#undef X
+    default: return 0;
+  }
+}
+
+int variant_tile(Variant v) {
+  switch (v) {
+#define X(id, D, T, NS) case id: return T;
     MLRA_VARIANTS(X)
 #undef X
     default: return 0;
@@ -108,7 +116,7 @@ cudaError_t launch_decode(Variant v, const CUtensorMap& tq, const CUtensorMap& t
                           const CUtensorMap& tc, const CUtensorMap& tkr, const DecodeParams& p,
                           int grid, cudaStream_t st) {
   switch (v) {
-#define X(id, D, G, NS, NP) case id: return launch_decode_t<D, G, NS, NP>(tq, tqr, tc, tkr, p, grid, st);
+#define X(id, D, T, NS) case id: return launch_decode_t<D, T, NS>(tq, tqr, tc, tkr, p, grid, st);
     MLRA_VARIANTS(X)
 #undef X
     default: return cudaErrorInvalidValue;
@@ -116,26 +124,27 @@ cudaError_t launch_decode(Variant v, const CUtensorMap& tq, const CUtensorMap& t
 }
 
 // ----------------------------------------------------------------------------- K2
-// Grid (H, N), 128 threads.  For sequence s split into parts p (ranges r0 .. r0+np-1, slot
-// r + s), per branch b: m* = max_p m_p, l* = sum_p 2^(m_p - m*) l_p and
+// Grid (H, N, column chunks of 128), 128 threads.  For sequence s split into parts (ranges
+// r0 .. r0+np-1, slot r + s), per branch b: m* = max_p m_p, l* = sum_p 2^(m_p - m*) l_p and
 //   out = gamma * sum_p 2^(m_p - m*) o_p / l*,   lse = (m* + log2 l*) ln 2.
-// Scores are kept in log2 units by K1.
+// Scores are kept in log2 units by K1.  The per-part weights gamma 2^(m_p - m*) / l* of every
+// branch are computed once per block into shared memory.
 __global__ void __launch_bounds__(128) mlra_combine_kernel(const CombineParams p) {
-  const int h = blockIdx.x, s = blockIdx.y;
+  const int h = blockIdx.x, s = blockIdx.y, chunk = blockIdx.z;
   const int64_t total = p.prefix[p.N];
   int r0 = 0, np = 0;
   if (total > 0) seq_parts(p.prefix, s, total, effective_ranges(p.num_ranges, total), &r0, &np);
   if (np == 1 && p.final_written) return;
   const int width = p.summed ? p.d_blk_out : p.B * p.d_blk_out;
+  const int c = chunk * 128 + threadIdx.x;
   float* out_row = p.out + ((int64_t)s * p.H + h) * width;
   if (np == 0) {
-    for (int c = threadIdx.x; c < width; c += blockDim.x) out_row[c] = 0.f;
-    if (p.lse && threadIdx.x < p.B) p.lse[((int64_t)s * p.H + h) * p.B + threadIdx.x] = -CUDART_INF_F;
+    if (c < width) out_row[c] = 0.f;
+    if (p.lse && chunk == 0 && threadIdx.x < p.B)
+      p.lse[((int64_t)s * p.H + h) * p.B + threadIdx.x] = -CUDART_INF_F;
     return;
   }
-  extern __shared__ float sh[];  // mstar[B], linv[B]
-  float* mstar = sh;
-  float* linv = sh + p.B;
+  extern __shared__ float wts[];  // [np][B]
   const int64_t slot0 = (int64_t)r0 + s;
   for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
     float m = -CUDART_INF_F;
@@ -143,46 +152,46 @@ __global__ void __launch_bounds__(128) mlra_combine_kernel(const CombineParams p
     float l = 0.f;
     for (int q = 0; q < np; ++q) {
       const float* ml = p.part_ml + (((slot0 + q) * p.H + h) * p.B + b) * 2;
-      l += exp2f(ml[0] - m) * ml[1];
+      const float w = exp2f(ml[0] - m);
+      wts[q * p.B + b] = w;
+      l += w * ml[1];
     }
-    mstar[b] = m;
-    linv[b] = 1.f / l;
-    if (p.lse) p.lse[((int64_t)s * p.H + h) * p.B + b] = (m + log2f(l)) * 0.69314718055994531f;
+    const float g = p.gamma / l;
+    for (int q = 0; q < np; ++q) wts[q * p.B + b] *= g;
+    if (p.lse && chunk == 0) p.lse[((int64_t)s * p.H + h) * p.B + b] = (m + log2f(l)) * 0.69314718055994531f;
   }
   __syncthreads();
+  if (c >= width) return;
+  const float* po = p.part_o + (slot0 * p.H + h) * p.dck;
+  const int64_t pstride = (int64_t)p.H * p.dck;  // next part of the same (s, h)
   if (!p.summed) {
-    for (int c = threadIdx.x; c < width; c += blockDim.x) {
-      const int b = c / p.d_blk_out, cc = c - b * p.d_blk_out;
-      const int kc = b * p.dblk_k + cc;
-      float acc = 0.f;
-      for (int q = 0; q < np; ++q) {
-        const int64_t base = (slot0 + q) * p.H + h;
-        const float w = exp2f(p.part_ml[(base * p.B + b) * 2] - mstar[b]);
-        acc += w * p.part_o[base * p.dck + kc];
-      }
-      out_row[c] = p.gamma * acc * linv[b];
-    }
+    const int b = c / p.d_blk_out;
+    const float* src = po + b * p.dblk_k + (c - b * p.d_blk_out);
+    float acc = 0.f;
+#pragma unroll 4
+    for (int q = 0; q < np; ++q) acc += wts[q * p.B + b] * src[q * pstride];
+    out_row[c] = acc;
   } else {
-    for (int c = threadIdx.x; c < width; c += blockDim.x) {
-      float tot = 0.f;
-      for (int b = 0; b < p.B; ++b) {
-        const int kc = b * p.dblk_k + c;
-        float acc = 0.f;
-        for (int q = 0; q < np; ++q) {
-          const int64_t base = (slot0 + q) * p.H + h;
-          const float w = exp2f(p.part_ml[(base * p.B + b) * 2] - mstar[b]);
-          acc += w * p.part_o[base * p.dck + kc];
-        }
-        tot += acc * linv[b];
-      }
-      out_row[c] = p.gamma * tot;
+    float acc = 0.f;
+    for (int b = 0; b < p.B; ++b) {
+      const float* src = po + b * p.dblk_k + c;
+#pragma unroll 4
+      for (int q = 0; q < np; ++q) acc += wts[q * p.B + b] * src[q * pstride];
     }
+    out_row[c] = acc;
   }
 }
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t st) {
-  dim3 grid(p.H, p.N);
-  mlra_combine_kernel<<<grid, 128, 2 * p.B * sizeof(float), st>>>(p);
+  const int width = p.summed ? p.d_blk_out : p.B * p.d_blk_out;
+  dim3 grid(p.H, p.N, (width + 127) / 128);
+  const size_t sh = (size_t)p.max_parts * p.B * sizeof(float);
+  if (sh > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(mlra_combine_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);
+    if (e != cudaSuccess) return e;
+  }
+  mlra_combine_kernel<<<grid, 128, sh, st>>>(p);
   return cudaGetLastError();
 }
 

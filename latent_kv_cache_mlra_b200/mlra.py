@@ -43,7 +43,8 @@ class Scales(ctypes.Structure):
 class PlanInfo(ctypes.Structure):
     _fields_ = [("repack", ctypes.c_int), ("launches", ctypes.c_int), ("num_ranges", ctypes.c_int),
                 ("ctas", ctypes.c_int), ("kernel_branch_width", ctypes.c_int),
-                ("branches_per_cta", ctypes.c_int), ("partial_slots", ctypes.c_longlong),
+                ("branches_per_cta", ctypes.c_int), ("tile", ctypes.c_int),
+                ("partial_slots", ctypes.c_longlong),
                 ("workspace_bytes", ctypes.c_size_t)]
 
 
