@@ -21,9 +21,19 @@
 // [latent blocks | RoPE block].  Once the score MMA of a tile has completed, the tile's RoPE block
 // is dead and the softmax writes the bf16 probabilities P of that tile into it.
 //
-// Warp roles (192 threads): warps 0-3 softmax / rescale / epilogue, warp 4 TMA producer,
-// warp 5 MMA issuer and TMEM owner.  Softmax warp w owns heads 16w..16w+15; the thread pair
-// (l, l ^ 16) shares head 16w + (l & 15) and splits every row's columns between them.
+// Warp roles (224 threads): warps 0-3 softmax / rescale / epilogue, warp 4 TMA producer,
+// warp 5 score-MMA issuer and TMEM owner, warp 6 output-MMA issuer.  The two issuers feed the
+// tensor core independently, each blocking on its own barriers.  Softmax warp w owns heads
+// 16w..16w+15; the thread pair (l, l ^ 16) shares head 16w + (l & 15) and splits every row's
+// columns between them.
+//
+// Ordering facts the parity waits rely on (a parity wait is only safe when the barrier is at
+// most one phase past the previous phase awaited):
+//   * the score of tile s is issued only after the output product of tile s - NSB was issued
+//     (bar_pv_issued), so neither issuer can run more than NSB tiles ahead of the other;
+//   * tile s is loaded only after the output product of tile s - NS completed (stage reuse),
+//     so once the score of tile s is done, every output product up to s - NS is done: the
+//     output-completion ring bar_pv_done has NS entries.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -48,14 +58,14 @@ struct DecodeCfg {
   static constexpr int O_COLS = ((OCH + 1) / 2) * OCW;  // TMEM columns used by O
   static constexpr int NSB_TMEM = (512 - O_COLS) / T;
   static constexpr int NSB = NSB_TMEM < 3 ? NSB_TMEM : (NS < 3 ? NS : 3);  // score buffers
-  static constexpr int NPV = NSB;                   // ring of output-MMA completion barriers
+  static constexpr int NPV = NS;                    // ring of output-MMA completion barriers
   static constexpr int TMEM_USED = O_COLS + NSB * T;
   static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 :
                                    TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_STAGE = QBYTES;
   static constexpr int OFF_BAR = OFF_STAGE + NS * STAGE;
-  static constexpr int NBAR = 2 * NS + 2 + 2 * NSB + NPV + 1;
+  static constexpr int NBAR = 2 * NS + 2 + 3 * NSB + NPV + 2;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM + 1024;    // slack to align the base to 1024 B
@@ -110,8 +120,10 @@ __device__ __forceinline__ int tile_row(const int32_t* page_table, int max_pages
   return pid * page_size + j % page_size;
 }
 
+constexpr int kDecodeThreads = 224;
+
 template <int DBLK, int T, int NS>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kDecodeThreads, 1)
 mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
                    const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_kr,
                    const __grid_constant__ DecodeParams p) {
@@ -131,11 +143,10 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const uint32_t bar_q_empty = bar_q_full + 8;              //       MMA (last score) -> TMA
   const uint32_t bar_s_full = bar_q_full + 16;              // [NSB] MMA (score) -> softmax
   const uint32_t bar_p_full = bar_s_full + 8 * NSB;         // [NSB] softmax -> MMA
-  // PV of tile j commits to bar_pv_done[j % NPV].  When a thread waits for PV(j), PV(j - NPV)
-  // is known to be complete, so the barrier is within one phase of the one awaited and the
-  // parity wait is unambiguous.
-  const uint32_t bar_pv_done = bar_p_full + 8 * NSB;        // [NPV] MMA (PV) -> softmax
-  const uint32_t bar_final = bar_pv_done + 8 * NPV;
+  const uint32_t bar_pv_issued = bar_p_full + 8 * NSB;     // [NSB] output issuer -> score issuer
+  const uint32_t bar_pv_done = bar_pv_issued + 8 * NSB;     // [NPV] MMA (PV done) -> softmax
+  const uint32_t bar_final_s = bar_pv_done + 8 * NPV;       // drains of the two issuers
+  const uint32_t bar_final_pv = bar_final_s + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -156,9 +167,11 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     for (int k = 0; k < NSB; ++k) {
       mbar_init(bar_s_full + 8 * k, 1);
       mbar_init(bar_p_full + 8 * k, 128);
+      mbar_init(bar_pv_issued + 8 * k, 1);
     }
     for (int k = 0; k < NPV; ++k) mbar_init(bar_pv_done + 8 * k, 1);
-    mbar_init(bar_final, 1);
+    mbar_init(bar_final_s, 1);
+    mbar_init(bar_final_pv, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -235,58 +248,20 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         wait_warp(bar_stage_full + 8 * (k % NS), (k / NS) & 1, tmo / 8, abort_flag, p.status, false);
     }
   } else if (warp == 5) {
-    // ------------------------------------------------------------------ MMA issuer
-    // Order: score of tile it, then the output products of every tile <= it - (NSB - 1), so the
-    // tensor core computes scores up to NSB - 1 tiles ahead of the softmax.
+    // ------------------------------------------------------------------ score-MMA issuer
     constexpr uint32_t kIdScore = idesc_bf16_f32(64, T, false, false);
-    constexpr uint32_t kIdPV = idesc_bf16_f32(64, C::OCW, false, true);
     SegmentWalker walk(p.prefix, p.N, total, R, range);
     Segment seg;
-    int it = 0, nseg = 0, pv_next = 0;
-    uint32_t first_mask = 0;  // bit (j % 32): tile j is the first of its segment
+    int it = 0, nseg = 0;
     bool ok = true;
-
-    auto issue_pv = [&](int j) -> bool {
-      if (!wait_warp(bar_p_full + 8 * (j % NSB), (j / NSB) & 1, tmo, abort_flag, p.status)) return false;
-      tc_fence_after();
-      if (lane == 0) {
-        const bool first = (first_mask >> (j & 31)) & 1u;
-        const uint32_t stg = sStage + (j % NS) * C::STAGE;
-        const uint32_t pa = stg + C::NCB * C::CBLK;  // P lives in the tile's RoPE block
-#pragma unroll
-        for (int ch = 0; ch < C::OCH; ++ch) {
-          const uint32_t d = tmem + ((uint32_t)(16 * (ch & 1)) << 16) + (ch >> 1) * C::OCW;
-          const uint32_t b0 = stg + ch * (C::OCW / 64) * C::CBLK;
-#pragma unroll
-          for (int kk = 0; kk < T / 16; ++kk) {
-            const uint64_t ad = sw128_desc(pa + (kk >> 2) * C::BOX + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(b0 + kk * 2048, C::CBLK, 1024);
-            umma_bf16(d, ad, bd, kIdPV, (kk > 0 || !first) ? 1u : 0u);
-          }
-        }
-        umma_commit(bar_stage_empty + 8 * (j % NS));
-        umma_commit(bar_pv_done + 8 * (j % NPV));
-      }
-      __syncwarp();
-      return true;
-    };
-
     while (ok && walk.next(seg)) {
-      for (int i = 0; i < seg.ntiles; ++i, ++it) {
-        if (i == 0) {
-          // Finish the previous segment first so that its epilogue overlaps this query load.
-          while (ok && pv_next < it) ok = issue_pv(pv_next++);
-          if (!ok) break;
-          ok = wait_warp(bar_q_full, nseg & 1, tmo, abort_flag, p.status);
-          if (!ok) break;
-        }
+      ok = wait_warp(bar_q_full, nseg & 1, tmo, abort_flag, p.status);
+      for (int i = 0; ok && i < seg.ntiles; ++i, ++it) {
         ok = wait_warp(bar_stage_full + 8 * (it % NS), (it / NS) & 1, tmo, abort_flag, p.status);
+        if (ok && it >= NSB)  // score buffer free and the output product of tile it-NSB issued
+          ok = wait_warp(bar_pv_issued + 8 * (it % NSB), ((it - NSB) / NSB) & 1, tmo, abort_flag,
+                         p.status);
         if (!ok) break;
-        if (it >= NSB) {
-          // score buffer it % NSB is free once the softmax of tile it - NSB has read it
-          ok = wait_warp(bar_p_full + 8 * (it % NSB), ((it - NSB) / NSB) & 1, tmo, abort_flag, p.status);
-          if (!ok) break;
-        }
         tc_fence_after();
         if (lane == 0) {
           const uint32_t stg = sStage + (it % NS) * C::STAGE;
@@ -310,18 +285,50 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           if (i == seg.ntiles - 1) umma_commit(bar_q_empty);
         }
         __syncwarp();
-        if (i == 0) first_mask |= 1u << (it & 31);
-        else first_mask &= ~(1u << (it & 31));
-        while (ok && pv_next <= it - (NSB - 1)) ok = issue_pv(pv_next++);
-        if (!ok) break;
       }
       ++nseg;
     }
-    while (ok && pv_next < it) ok = issue_pv(pv_next++);
     // Nothing of ours may still run on the tensor core when TMEM is released.
-    if (lane == 0) umma_commit(bar_final);
+    if (lane == 0) umma_commit(bar_final_s);
     __syncwarp();
-    wait_warp(bar_final, 0, tmo, abort_flag, p.status, false);
+    wait_warp(bar_final_s, 0, tmo, abort_flag, p.status, false);
+  } else if (warp == 6) {
+    // ------------------------------------------------------------------ output-MMA issuer
+    constexpr uint32_t kIdPV = idesc_bf16_f32(64, C::OCW, false, true);
+    SegmentWalker walk(p.prefix, p.N, total, R, range);
+    Segment seg;
+    int j = 0;
+    bool ok = true;
+    while (ok && walk.next(seg)) {
+      for (int i = 0; i < seg.ntiles; ++i, ++j) {
+        ok = wait_warp(bar_p_full + 8 * (j % NSB), (j / NSB) & 1, tmo, abort_flag, p.status);
+        if (!ok) break;
+        tc_fence_after();
+        if (lane == 0) {
+          const bool first = (i == 0);  // the segment's first product overwrites O
+          const uint32_t stg = sStage + (j % NS) * C::STAGE;
+          const uint32_t pa = stg + C::NCB * C::CBLK;  // P lives in the tile's RoPE block
+#pragma unroll
+          for (int ch = 0; ch < C::OCH; ++ch) {
+            const uint32_t d = tmem + ((uint32_t)(16 * (ch & 1)) << 16) + (ch >> 1) * C::OCW;
+            const uint32_t b0 = stg + ch * (C::OCW / 64) * C::CBLK;
+#pragma unroll
+            for (int kk = 0; kk < T / 16; ++kk) {
+              const uint64_t ad = sw128_desc(pa + (kk >> 2) * C::BOX + (kk & 3) * 32, 16, 1024);
+              const uint64_t bd = sw128_desc(b0 + kk * 2048, C::CBLK, 1024);
+              umma_bf16(d, ad, bd, kIdPV, (kk > 0 || !first) ? 1u : 0u);
+            }
+          }
+          umma_commit(bar_stage_empty + 8 * (j % NS));
+          umma_commit(bar_pv_done + 8 * (j % NPV));
+          mbar_arrive(bar_pv_issued + 8 * (j % NSB));
+        }
+        __syncwarp();
+      }
+    }
+    if (lane == 0) umma_commit(bar_final_pv);
+    __syncwarp();
+    wait_warp(bar_final_pv, 0, tmo, abort_flag, p.status, false);
   } else {
     // ------------------------------------------------------------------ softmax warps 0-3
     const int q = lane >> 4;                   // which half of the row's columns

@@ -83,7 +83,7 @@ static cudaError_t launch_decode_t(const CUtensorMap& tq, const CUtensorMap& tqr
   auto kern = mlra_decode_kernel<DBLK, T, NS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
-  kern<<<grid, 192, C::SMEM_ALLOC, st>>>(tq, tqr, tc, tkr, p);
+  kern<<<grid, kDecodeThreads, C::SMEM_ALLOC, st>>>(tq, tqr, tc, tkr, p);
   return cudaGetLastError();
 }
 
