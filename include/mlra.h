@@ -59,7 +59,9 @@ typedef enum {
   MLRA_ERR_TIMEOUT = 4,      /* a device-side bounded wait ran out (status word) */
   MLRA_ERR_WORKSPACE = 5,    /* workspace null, too small or misaligned */
   MLRA_ERR_BAD_PAGE = 6,     /* a page id outside [0, cache_rows / page_size) (status word) */
-  MLRA_ERR_BAD_LENGTH = 7    /* a sequence length < 0 or beyond the cache (status word) */
+  MLRA_ERR_BAD_LENGTH = 7,   /* a sequence length < 0 or beyond the cache (status word) */
+  MLRA_ERR_SCRATCH_LIMIT = 8 /* mlra_decode_static_scratch: the problem needs more scratch than
+                                MLRA_STATIC_SCRATCH_BYTES */
 } mlra_status;
 
 typedef enum { MLRA_BF16 = 0, MLRA_F32 = 1 } mlra_dtype;
@@ -151,6 +153,29 @@ typedef struct {
   size_t workspace_bytes;
 } mlra_plan_info;
 mlra_status mlra_query_plan(const mlra_dims* dims, mlra_plan_info* info_host);
+
+/* mlra_decode for callers that cannot hand the library any device memory: hosts that own every
+ * device allocation through their own pool and give plug-ins no allocator, or serving paths that
+ * must not allocate at all.  It takes the same arguments as mlra_decode minus the workspace and
+ * uses instead a scratch array built into the library (MLRA_STATIC_SCRATCH_BYTES, allocated on a
+ * device when the library's kernels are loaded there and kept until the process exits).  It
+ * allocates nothing and frees nothing.  (This entry point is an addition of this library; the
+ * method's pages have no counterpart.)
+ *   - The first call on each device does a one-time set-up: with that device current it looks up
+ *     the scratch array's device address.  Make that first call before any stream capture.
+ *   - Every call on a device shares the one array, which keeps the last call's contents (nothing
+ *     in it has to start at zero: each call rewrites what it later reads).  Calls that overlap on
+ *     the GPU (other streams, other host threads) race on it: serialise them.
+ *   - Problems whose workspace (mlra_workspace_size) exceeds MLRA_STATIC_SCRATCH_BYTES, including
+ *     every problem that needs the fp32 / padded repack copies, return MLRA_ERR_SCRATCH_LIMIT
+ *     before any work is queued.  Other errors as mlra_decode.  The device status word of these
+ *     calls is not readable through mlra_read_status. */
+#define MLRA_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+mlra_status mlra_decode_static_scratch(const void* q_lat, const void* q_rope, const void* c_kv,
+                                       const void* k_rope, const int32_t* seq_lens,
+                                       const int32_t* page_table, int B, const mlra_scales* scales,
+                                       float* out, float* lse, const mlra_dims* dims,
+                                       mlra_stream_t stream);
 
 /* Reads the status word that the last mlra_decode on `workspace` left, after synchronising
  * `stream`.  *flags_host receives the MLRA_FLAG_* bits; the return value is MLRA_OK when no

@@ -149,6 +149,13 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// Scratch of mlra_decode_static_scratch.  In host code the name stands for the array only as a
+// symbol: its device address comes from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) unsigned char g_static_scratch[MLRA_STATIC_SCRATCH_BYTES];
+constexpr int kMaxDevices = 256;
+std::mutex g_static_scratch_mu;
+void* g_static_scratch_addr[kMaxDevices] = {};
+
 }  // namespace
 
 extern "C" {
@@ -165,6 +172,9 @@ const char* mlra_status_string(mlra_status s) {
     case MLRA_ERR_WORKSPACE: return "MLRA_ERR_WORKSPACE: workspace null, too small or misaligned";
     case MLRA_ERR_BAD_PAGE: return "MLRA_ERR_BAD_PAGE: page id outside the cache pool";
     case MLRA_ERR_BAD_LENGTH: return "MLRA_ERR_BAD_LENGTH: sequence length outside the cache";
+    case MLRA_ERR_SCRATCH_LIMIT:
+      return "MLRA_ERR_SCRATCH_LIMIT: the problem needs more scratch than the library's built-in "
+             "buffer (MLRA_STATIC_SCRATCH_BYTES); use mlra_decode with a workspace";
   }
   return "MLRA: unknown status";
 }
@@ -320,6 +330,39 @@ mlra_status mlra_decode_profiled(const void* q_lat, const void* q_rope, const vo
   cp.gamma = scales->branch_scale;
   if (launch_combine(cp, s) != cudaSuccess) return MLRA_ERR_CUDA;
   return MLRA_OK;
+}
+
+mlra_status mlra_decode_static_scratch(const void* q_lat, const void* q_rope, const void* c_kv,
+                                       const void* k_rope, const int32_t* seq_lens,
+                                       const int32_t* page_table, int B, const mlra_scales* scales,
+                                       float* out, float* lse, const mlra_dims* dims,
+                                       mlra_stream_t stream) {
+  if (!dims) return MLRA_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLRA_ERR_CUDA;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+    if (!g_static_scratch_addr[dev]) {
+      void* addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, g_static_scratch) != cudaSuccess || !addr) return MLRA_ERR_CUDA;
+      g_static_scratch_addr[dev] = addr;
+    }
+    scratch = g_static_scratch_addr[dev];
+  }
+  const bool paged = page_table != nullptr;
+  int sms = 0;
+  mlra_status st = MLRA_OK;
+  if (dims->num_ranges == 0) {
+    sms = device_sm_count(&st);
+    if (st != MLRA_OK) return st;
+  }
+  Plan pl;
+  st = make_plan(dims, paged, sms, &pl);
+  if (st != MLRA_OK) return st;
+  if (pl.total > MLRA_STATIC_SCRATCH_BYTES) return MLRA_ERR_SCRATCH_LIMIT;
+  return mlra_decode(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table, B, scales, out, lse, dims,
+                     scratch, MLRA_STATIC_SCRATCH_BYTES, stream);
 }
 
 mlra_status mlra_read_status(const void* workspace, mlra_stream_t stream, uint32_t* flags_host) {

@@ -17,12 +17,15 @@ LIB_PATH = pathlib.Path(__file__).resolve().parent / "libmlra.so"
 
 MLRA_OK, MLRA_ERR_INVALID_ARG, MLRA_ERR_UNSUPPORTED, MLRA_ERR_CUDA = 0, 1, 2, 3
 MLRA_ERR_TIMEOUT, MLRA_ERR_WORKSPACE, MLRA_ERR_BAD_PAGE, MLRA_ERR_BAD_LENGTH = 4, 5, 6, 7
+MLRA_ERR_SCRATCH_LIMIT = 8
+STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 MLRA_BF16, MLRA_F32 = 0, 1
 MLRA_OUT_BRANCHES, MLRA_OUT_SUMMED = 0, 1
 FLAG_TIMEOUT, FLAG_BAD_PAGE, FLAG_BAD_LENGTH = 0x1, 0x2, 0x4
 
 # Every entry point of include/mlra.h.
 EXPORTS = ("mlra_workspace_size", "mlra_decode", "mlra_decode_profiled", "mlra_query_plan",
+           "mlra_decode_static_scratch",
            "mlra_read_status", "mlra_debug_resolve_rows", "mlra_plan_host",
            "mlra_plan_segments_host", "mlra_status_string", "mlra_version")
 
@@ -72,6 +75,7 @@ def lib() -> ctypes.CDLL:
                                   vp, vp, ctypes.POINTER(Dims), vp, ctypes.c_size_t, vp]
         L.mlra_decode_profiled.argtypes = L.mlra_decode.argtypes + [vp, vp]
         L.mlra_query_plan.argtypes = [ctypes.POINTER(Dims), ctypes.POINTER(PlanInfo)]
+        L.mlra_decode_static_scratch.argtypes = L.mlra_decode.argtypes[:11] + [vp]
         L.mlra_read_status.argtypes = [vp, vp, u32p]
         L.mlra_debug_resolve_rows.argtypes = [vp, vp, ctypes.POINTER(Dims), vp, ctypes.c_int, vp]
         L.mlra_plan_host.argtypes = [i32p, ctypes.c_int, ctypes.c_int, i32p, i32p]
@@ -81,6 +85,7 @@ def lib() -> ctypes.CDLL:
         L.mlra_status_string.restype = ctypes.c_char_p
         L.mlra_version.argtypes = []
         for f in ("mlra_workspace_size", "mlra_decode", "mlra_decode_profiled", "mlra_query_plan",
+                  "mlra_decode_static_scratch",
                   "mlra_read_status", "mlra_debug_resolve_rows", "mlra_plan_host",
                   "mlra_plan_segments_host"):
             getattr(L, f).restype = ctypes.c_int
@@ -176,6 +181,31 @@ def decode(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table=None, *, num_branch
                              _ptr(page_table), num_branches, ctypes.byref(scales), _ptr(out),
                              _ptr(lse), ctypes.byref(dims), _ptr(workspace), workspace.numel(),
                              ctypes.c_void_p(st)), "mlra_decode")
+    return out, lse
+
+
+def decode_static_scratch(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table=None, *,
+                          num_branches: int, softmax_scale: float,
+                          branch_scale: Optional[float] = None, out_mode="branches",
+                          max_seq_len=None, page_size=0, out=None, lse=None, num_ranges=0,
+                          stream=None):
+    """``mlra_decode_static_scratch``: the decode without a workspace argument; the library uses
+    its built-in scratch array.  ``out`` / ``lse`` are allocated here when not given (the C entry
+    point itself allocates nothing).  Returns (out, lse or None)."""
+    gamma = 1.0 / num_branches if branch_scale is None else branch_scale
+    dims = dims_for(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table, num_branches,
+                    max_seq_len=max_seq_len, page_size=page_size, out_mode=out_mode,
+                    num_ranges=num_ranges)
+    N, H, d_c = q_lat.shape
+    width = d_c if out_mode == "branches" else d_c // num_branches
+    if out is None:
+        out = torch.empty(N, H, width, dtype=torch.float32, device=q_lat.device)
+    st = stream if stream is not None else torch.cuda.current_stream(q_lat.device).cuda_stream
+    scales = Scales(softmax_scale, gamma)
+    _check(lib().mlra_decode_static_scratch(
+        _ptr(q_lat), _ptr(q_rope), _ptr(c_kv), _ptr(k_rope), _ptr(seq_lens), _ptr(page_table),
+        num_branches, ctypes.byref(scales), _ptr(out), _ptr(lse), ctypes.byref(dims),
+        ctypes.c_void_p(st)), "mlra_decode_static_scratch")
     return out, lse
 
 

@@ -29,7 +29,7 @@ def test_library_loads_and_exports_every_declared_symbol():
 
 
 def test_status_strings():
-    for code in range(8):
+    for code in range(9):
         s = mlra.status_string(code)
         assert s.startswith("MLRA_")
     assert "unknown" in mlra.status_string(99)
