@@ -181,6 +181,12 @@ def max_over_ranks(x: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def weak_scaling_value(batch_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job decode tokens/s: every rank decodes its own batch (one token per sequence) per
+    step, and the step time is the maximum over ranks."""
+    return batch_per_rank * world / (ms_per_step * 1e-3)
+
+
 def rank_workload(name: str, rank: int) -> workloads.Workload:
     w = workloads.get(name)
     return workloads.Workload(**{**w.__dict__, "seed": w.seed + 7919 * rank})
@@ -362,7 +368,7 @@ def run_ours(args):
     tflops = nflops / (k1_avg_ms * 1e-3) / 1e12
     total_seqs = w.batch * world
     line = {
-        "metric": METRIC, "value": total_seqs / (ms_step * 1e-3), "unit": "tokens/s",
+        "metric": METRIC, "value": weak_scaling_value(w.batch, world, ms_step), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": {**workload_config(w, inp), "parallelism": f"dp{world}"},
