@@ -18,8 +18,8 @@
 // j lives in lane half j % 2 at columns 128 (j / 2); score buffers follow in lane half 0.
 //
 // Shared memory: the branch's queries (per segment), an NS-deep ring of cache tiles
-// [latent blocks | RoPE block].  Once the score MMA of a tile has completed, the tile's RoPE block
-// is dead and the softmax writes the bf16 probabilities P of that tile into it.
+// [latent blocks | RoPE block].  The bf16 probabilities P of a tile overwrite the front of the
+// tile's own score buffer in TMEM, from where the output MMA reads them as its A operand.
 //
 // Warp roles (224 threads): warps 0-3 softmax / rescale / epilogue, warp 4 TMA producer,
 // warp 5 score-MMA issuer and TMEM owner, warp 6 output-MMA issuer.  The two issuers feed the
@@ -29,8 +29,9 @@
 //
 // Ordering facts the parity waits rely on (a parity wait is only safe when the barrier is at
 // most one phase past the previous phase awaited):
-//   * the score of tile s is issued only after the output product of tile s - NSB was issued
-//     (bar_pv_issued), so neither issuer can run more than NSB tiles ahead of the other;
+//   * the score of tile s is issued only after the output product of tile s - NSB completed
+//     (its P sits in the score buffer being reused), so neither issuer can run more than NSB
+//     tiles ahead of the other;
 //   * tile s is loaded only after the output product of tile s - NS completed (stage reuse),
 //     so once the score of tile s is done, every output product up to s - NS is done: the
 //     output-completion ring bar_pv_done has NS entries.
@@ -65,7 +66,7 @@ struct DecodeCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_STAGE = QBYTES;
   static constexpr int OFF_BAR = OFF_STAGE + NS * STAGE;
-  static constexpr int NBAR = 2 * NS + 2 + 3 * NSB + NPV + 2;
+  static constexpr int NBAR = 2 * NS + 2 + 2 * NSB + NPV + 2;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM + 1024;    // slack to align the base to 1024 B
@@ -143,8 +144,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const uint32_t bar_q_empty = bar_q_full + 8;              //       MMA (last score) -> TMA
   const uint32_t bar_s_full = bar_q_full + 16;              // [NSB] MMA (score) -> softmax
   const uint32_t bar_p_full = bar_s_full + 8 * NSB;         // [NSB] softmax -> MMA
-  const uint32_t bar_pv_issued = bar_p_full + 8 * NSB;     // [NSB] output issuer -> score issuer
-  const uint32_t bar_pv_done = bar_pv_issued + 8 * NSB;     // [NPV] MMA (PV done) -> softmax
+  const uint32_t bar_pv_done = bar_p_full + 8 * NSB;       // [NPV] MMA (PV done) -> softmax, score issuer
   const uint32_t bar_final_s = bar_pv_done + 8 * NPV;       // drains of the two issuers
   const uint32_t bar_final_pv = bar_final_s + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -153,9 +153,9 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int range = blockIdx.x / p.n_groups;
   const int branch = blockIdx.x % p.n_groups;
-  const int64_t total = p.prefix[p.N];
-  const int64_t R = effective_ranges(p.num_ranges, total);
   const uint64_t tmo = p.timeout_ns;
+  // The combine kernel may be scheduled now; it waits for this grid before reading anything.
+  pdl_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int k = 0; k < NS; ++k) {
@@ -167,7 +167,6 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     for (int k = 0; k < NSB; ++k) {
       mbar_init(bar_s_full + 8 * k, 1);
       mbar_init(bar_p_full + 8 * k, 128);
-      mbar_init(bar_pv_issued + 8 * k, 1);
     }
     for (int k = 0; k < NPV; ++k) mbar_init(bar_pv_done + 8 * k, 1);
     mbar_init(bar_final_s, 1);
@@ -190,6 +189,10 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int col0 = branch * DBLK;  // first latent column of this CTA's branch
+  // Everything above overlapped the prep kernel; its lengths and tile prefix are needed now.
+  pdl_wait_prerequisites();
+  const int64_t total = p.prefix[p.N];
+  const int64_t R = effective_ranges(p.num_ranges, total);
 
   if (warp == 4) {
     // ------------------------------------------------------------------ TMA producer
@@ -258,9 +261,9 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       ok = wait_warp(bar_q_full, nseg & 1, tmo, abort_flag, p.status);
       for (int i = 0; ok && i < seg.ntiles; ++i, ++it) {
         ok = wait_warp(bar_stage_full + 8 * (it % NS), (it / NS) & 1, tmo, abort_flag, p.status);
-        if (ok && it >= NSB)  // score buffer free and the output product of tile it-NSB issued
-          ok = wait_warp(bar_pv_issued + 8 * (it % NSB), ((it - NSB) / NSB) & 1, tmo, abort_flag,
-                         p.status);
+        if (ok && it >= NSB)  // score buffer free: the output product of tile it-NSB read its P
+          ok = wait_warp(bar_pv_done + 8 * ((it - NSB) % NPV), ((it - NSB) / NPV) & 1, tmo,
+                         abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
         if (lane == 0) {
@@ -307,21 +310,22 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         if (lane == 0) {
           const bool first = (i == 0);  // the segment's first product overwrites O
           const uint32_t stg = sStage + (j % NS) * C::STAGE;
-          const uint32_t pa = stg + C::NCB * C::CBLK;  // P lives in the tile's RoPE block
+          const uint32_t pa = tmem + C::O_COLS + (j % NSB) * T;  // P: front of the score buffer
 #pragma unroll
           for (int ch = 0; ch < C::OCH; ++ch) {
+            // A from TMEM must sit in the accumulator's lanes: chunks in lane half 1 read the
+            // copy of P that the softmax writes there
             const uint32_t d = tmem + ((uint32_t)(16 * (ch & 1)) << 16) + (ch >> 1) * C::OCW;
             const uint32_t b0 = stg + ch * (C::OCW / 64) * C::CBLK;
 #pragma unroll
             for (int kk = 0; kk < T / 16; ++kk) {
-              const uint64_t ad = sw128_desc(pa + (kk >> 2) * C::BOX + (kk & 3) * 32, 16, 1024);
               const uint64_t bd = sw128_desc(b0 + kk * 2048, C::CBLK, 1024);
-              umma_bf16(d, ad, bd, kIdPV, (kk > 0 || !first) ? 1u : 0u);
+              umma_bf16_ts(d, pa + ((uint32_t)(16 * (ch & 1)) << 16) + kk * 8, bd, kIdPV,
+                           (kk > 0 || !first) ? 1u : 0u);
             }
           }
           umma_commit(bar_stage_empty + 8 * (j % NS));
           umma_commit(bar_pv_done + 8 * (j % NPV));
-          mbar_arrive(bar_pv_issued + 8 * (j % NSB));
         }
         __syncwarp();
       }
@@ -400,8 +404,9 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           }
           tmem_wait_st();
         }
-        // probabilities -> bf16 P tile in the (consumed) RoPE block: K-major, 128-byte swizzle
-        uint8_t* stg = smem + C::OFF_STAGE + (it % NS) * C::STAGE;
+        // probabilities -> bf16 P over the front of this tile's score buffer: position
+        // 64 l + 32 q + k goes to column (64 l + 32 q + k) / 2, two positions per column
+        const uint32_t pcol = tmem + lane_base + C::O_COLS + (it % NSB) * T;
         float sum = 0.f;
 #pragma unroll
         for (int l = 0; l < C::TB; ++l) {
@@ -413,17 +418,14 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             sum += p0 + p1;
             pk[k / 2] = pack_bf16x2(p0, p1);
           }
-          uint8_t* prow = stg + C::NCB * C::CBLK + l * C::BOX + h * 128;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int chunk = 4 * q + c;
-            *reinterpret_cast<uint4*>(prow + ((chunk ^ (h & 7)) << 4)) =
-                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-          }
+          tmem_st16x2_16(pcol + 32 * l, pk);
+          if (C::OCH > 1) tmem_st16x2_16(pcol + (16u << 16) + 32 * l, pk);  // copy in lane half 1
         }
+        tmem_wait_st();
         sum += __shfl_xor_sync(kFull, sum, 16);
         l_sum += sum;
         if (valid < T) {
+          uint8_t* stg = smem + C::OFF_STAGE + (it % NS) * C::STAGE;
           // Ragged last tile: zero the latent rows past the sequence end so that the zero
           // probabilities never multiply a non-finite value left in the cache.
           for (int k = threadIdx.x; k < C::NCB * T * 8; k += 128) {
@@ -432,8 +434,8 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
               *reinterpret_cast<uint4*>(stg + (k / (T * 8)) * C::CBLK + row * 128 + (k & 7) * 16) =
                   make_uint4(0u, 0u, 0u, 0u);
           }
+          fence_proxy_async_smem();  // the zeros are read by the output MMA (async proxy)
         }
-        fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(bar_p_full + 8 * (it % NSB));
       }

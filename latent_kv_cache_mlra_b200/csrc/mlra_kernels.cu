@@ -8,6 +8,7 @@
 #include <math_constants.h>
 
 #include "mlra_decode_kernel.cuh"
+#include "sm100_ptx.cuh"
 #include "mlra_internal.h"
 #include "mlra_plan.cuh"
 
@@ -23,6 +24,7 @@ __global__ void __launch_bounds__(1024) mlra_prep_kernel(const int32_t* seq_lens
   __shared__ int32_t carry;
   __shared__ uint32_t flags;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  pdl_launch_dependents();  // the decode kernel may start its prologue now
   if (tid == 0) {
     carry = 0;
     flags = 0;
@@ -83,8 +85,17 @@ static cudaError_t launch_decode_t(const CUtensorMap& tq, const CUtensorMap& tqr
   auto kern = mlra_decode_kernel<DBLK, T, NS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kDecodeThreads, C::SMEM_ALLOC, st>>>(tq, tqr, tc, tkr, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kDecodeThreads);
+  cfg.dynamicSmemBytes = C::SMEM_ALLOC;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap with the prep kernel
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tq, tqr, tc, tkr, p);
 }
 
 // (padded branch width, positions per tile, cache-tile stages)
@@ -131,6 +142,7 @@ cudaError_t launch_decode(Variant v, const CUtensorMap& tq, const CUtensorMap& t
 // branch are computed once per block into shared memory.
 __global__ void __launch_bounds__(128) mlra_combine_kernel(const CombineParams p) {
   const int h = blockIdx.x, s = blockIdx.y, chunk = blockIdx.z;
+  pdl_wait_prerequisites();  // the decode kernel's partials must be complete and visible
   const int64_t total = p.prefix[p.N];
   int r0 = 0, np = 0;
   if (total > 0) seq_parts(p.prefix, s, total, effective_ranges(p.num_ranges, total), &r0, &np);
@@ -144,22 +156,41 @@ __global__ void __launch_bounds__(128) mlra_combine_kernel(const CombineParams p
       p.lse[((int64_t)s * p.H + h) * p.B + threadIdx.x] = -CUDART_INF_F;
     return;
   }
-  extern __shared__ float wts[];  // [np][B]
+  extern __shared__ float sh[];  // m[np][B] (then the weights), l[np][B], m*[B], l*[B]
+  float* wts = sh;
+  float* lpart = sh + np * p.B;
+  float* mstar = lpart + np * p.B;
+  float* lstar = mstar + p.B;
   const int64_t slot0 = (int64_t)r0 + s;
+  const int n_ml = np * p.B;
+  // 1. every (part, branch) state in parallel
+  for (int k = threadIdx.x; k < n_ml; k += blockDim.x) {
+    const int q = k / p.B, b = k - q * p.B;
+    const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + (((slot0 + q) * p.H + h) * p.B + b) * 2);
+    wts[k] = ml.x;
+    lpart[k] = ml.y;
+  }
+  __syncthreads();
+  // 2. per branch: m* = max_p m_p
   for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
     float m = -CUDART_INF_F;
-    for (int q = 0; q < np; ++q) m = fmaxf(m, p.part_ml[(((slot0 + q) * p.H + h) * p.B + b) * 2]);
-    float l = 0.f;
-    for (int q = 0; q < np; ++q) {
-      const float* ml = p.part_ml + (((slot0 + q) * p.H + h) * p.B + b) * 2;
-      const float w = exp2f(ml[0] - m);
-      wts[q * p.B + b] = w;
-      l += w * ml[1];
-    }
-    const float g = p.gamma / l;
-    for (int q = 0; q < np; ++q) wts[q * p.B + b] *= g;
-    if (p.lse && chunk == 0) p.lse[((int64_t)s * p.H + h) * p.B + b] = (m + log2f(l)) * 0.69314718055994531f;
+    for (int q = 0; q < np; ++q) m = fmaxf(m, wts[q * p.B + b]);
+    mstar[b] = m;
   }
+  __syncthreads();
+  // 3. w_p = 2^(m_p - m*) (unnormalised), in parallel
+  for (int k = threadIdx.x; k < n_ml; k += blockDim.x) wts[k] = exp2f(wts[k] - mstar[k % p.B]);
+  __syncthreads();
+  // 4. l* = sum_p w_p l_p, then fold gamma / l* into the weights
+  for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
+    float l = 0.f;
+    for (int q = 0; q < np; ++q) l += wts[q * p.B + b] * lpart[q * p.B + b];
+    lstar[b] = l;
+    if (p.lse && chunk == 0)
+      p.lse[((int64_t)s * p.H + h) * p.B + b] = (mstar[b] + log2f(l)) * 0.69314718055994531f;
+  }
+  __syncthreads();
+  for (int k = threadIdx.x; k < n_ml; k += blockDim.x) wts[k] *= p.gamma / lstar[k % p.B];
   __syncthreads();
   if (c >= width) return;
   const float* po = p.part_o + (slot0 * p.H + h) * p.dck;
@@ -184,15 +215,23 @@ __global__ void __launch_bounds__(128) mlra_combine_kernel(const CombineParams p
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t st) {
   const int width = p.summed ? p.d_blk_out : p.B * p.d_blk_out;
-  dim3 grid(p.H, p.N, (width + 127) / 128);
-  const size_t sh = (size_t)p.max_parts * p.B * sizeof(float);
+  const size_t sh = (2 * (size_t)p.max_parts * p.B + 2 * p.B) * sizeof(float);
   if (sh > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(mlra_combine_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);
     if (e != cudaSuccess) return e;
   }
-  mlra_combine_kernel<<<grid, 128, sh, st>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.H, p.N, (width + 127) / 128);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = sh;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap the decode tail
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, mlra_combine_kernel, p);
 }
 
 // ----------------------------------------------------------------------------- K3
