@@ -33,7 +33,8 @@ struct Plan {
   int R = 0;           // work ranges
   int64_t slots = 0;   // partial slots = R + N - 1
   int limit = 0;       // bound on seq_lens
-  size_t off_lens = 0, off_prefix = 0, off_ml = 0, off_o = 0;
+  size_t off_lens = 0, off_prefix = 0, off_ranges = 0, off_segs = 0, off_seqs = 0;
+  size_t off_ml = 0, off_o = 0;
   size_t off_rq = 0, off_rqr = 0, off_rc = 0, off_rkr = 0, total = 0;
 };
 
@@ -102,6 +103,9 @@ mlra_status make_plan(const mlra_dims* d, bool paged, int sms, Plan* pl) {
   size_t off = kAlign;  // status word + padding
   pl->off_lens = off; off = align_up(off + 4 * N);
   pl->off_prefix = off; off = align_up(off + 4 * (N + 1));
+  pl->off_ranges = off; off = align_up(off + sizeof(RangeInfo) * (size_t)pl->R);
+  pl->off_segs = off; off = align_up(off + sizeof(SegDesc) * (size_t)pl->slots);
+  pl->off_seqs = off; off = align_up(off + sizeof(SeqInfo) * (size_t)N);
   pl->off_ml = off; off = align_up(off + (size_t)pl->slots * H * B * 2 * sizeof(float));
   pl->off_o = off; off = align_up(off + (size_t)pl->slots * H * pl->dck * sizeof(float));
   if (pl->repack) {
@@ -262,6 +266,9 @@ mlra_status mlra_decode_profiled(const void* q_lat, const void* q_rope, const vo
   int32_t* prefix = reinterpret_cast<int32_t*>(ws + pl.off_prefix);
   float* part_ml = reinterpret_cast<float*>(ws + pl.off_ml);
   float* part_o = reinterpret_cast<float*>(ws + pl.off_o);
+  RangeInfo* ranges = reinterpret_cast<RangeInfo*>(ws + pl.off_ranges);
+  SegDesc* segs = reinterpret_cast<SegDesc*>(ws + pl.off_segs);
+  SeqInfo* seqs = reinterpret_cast<SeqInfo*>(ws + pl.off_seqs);
   const int N = dims->batch, H = dims->heads, dblk = dims->d_latent / B;
   const int64_t rows = dims->cache_rows;
 
@@ -297,14 +304,20 @@ mlra_status mlra_decode_profiled(const void* q_lat, const void* q_rope, const vo
       return MLRA_ERR_CUDA;
   }
 
-  if (launch_prep(seq_lens, N, pl.limit, pl.tile, lens, prefix, status, s) != cudaSuccess)
-    return MLRA_ERR_CUDA;
+  const bool summed = dims->out_mode == MLRA_OUT_SUMMED;
+  const int out_width = summed ? dblk : dims->d_latent;  // floats per (sequence, head) row of out
+  PrepParams pp;
+  pp.seq_lens = seq_lens; pp.N = N; pp.limit = pl.limit; pp.tile = pl.tile; pp.num_ranges = pl.R;
+  pp.lens = lens; pp.prefix = prefix; pp.ranges = ranges; pp.segs = segs; pp.seqs = seqs;
+  pp.status = status;
+  pp.out = out; pp.lse = lse; pp.H = H; pp.B = B; pp.out_width = out_width;
+  if (launch_prep(pp, s) != cudaSuccess) return MLRA_ERR_CUDA;
 
   DecodeParams p;
-  p.lens = lens; p.prefix = prefix; p.page_table = page_table;
-  const bool summed = dims->out_mode == MLRA_OUT_SUMMED;
+  p.ranges = ranges; p.segs = segs;
+  p.page_table = page_table;
   p.out = out; p.lse = lse; p.part_o = part_o; p.part_ml = part_ml; p.status = status;
-  p.N = N; p.H = H; p.B = B; p.d_blk_out = dblk; p.out_width = dims->d_latent; p.dck = pl.dck;
+  p.N = N; p.H = H; p.B = B; p.d_blk_out = dblk; p.out_width = out_width; p.dck = pl.dck;
   p.n_groups = pl.n_groups; p.num_ranges = pl.R;
   p.page_size = paged ? dims->page_size : 0;
   p.max_pages = paged ? dims->max_pages_per_seq : 0;
@@ -323,9 +336,17 @@ mlra_status mlra_decode_profiled(const void* q_lat, const void* q_rope, const vo
     return MLRA_ERR_CUDA;
 
   CombineParams cp;
-  cp.prefix = prefix; cp.part_o = part_o; cp.part_ml = part_ml; cp.out = out; cp.lse = lse;
+  cp.seqs = seqs; cp.part_o = part_o; cp.part_ml = part_ml; cp.out = out; cp.lse = lse;
   cp.N = N; cp.H = H; cp.B = B; cp.dblk_k = pl.dblk_k; cp.dck = pl.dck; cp.d_blk_out = dblk;
-  cp.num_ranges = pl.R; cp.max_parts = pl.R; cp.summed = summed ? 1 : 0;
+  cp.summed = summed ? 1 : 0;
+  // about R / N parts per sequence (all R for one sequence): enough warps per head that each folds
+  // at most one batch of loads
+  {
+    const int est_parts = (pl.R + N - 1) / N + 1;
+    int G = 1;
+    while (G < 8 && G * 8 < est_parts) G *= 2;
+    cp.groups = G;
+  }
   cp.final_written = summed ? 0 : 1;
   cp.gamma = scales->branch_scale;
   if (launch_combine(cp, s) != cudaSuccess) return MLRA_ERR_CUDA;

@@ -123,6 +123,28 @@ __device__ __forceinline__ int tile_row(const int32_t* page_table, int max_pages
 
 constexpr int kDecodeThreads = 224;
 
+// The segments of one work range, read from the prep kernel's descriptors one ahead of use.
+struct SegCursor {
+  const SegDesc* segs;
+  int first, count, i;
+  int4 nxt;
+  __device__ __forceinline__ SegCursor(const SegDesc* s, RangeInfo ri)
+      : segs(s), first(ri.first), count(ri.count), i(0) {
+    if (count > 0) nxt = __ldcg(reinterpret_cast<const int4*>(segs + first));
+  }
+  __device__ __forceinline__ bool next(Segment& seg, int& len) {
+    if (i >= count) return false;
+    const int4 d = nxt;
+    if (++i < count) nxt = __ldcg(reinterpret_cast<const int4*>(segs + first + i));
+    seg.seq = d.x;
+    seg.tile0 = d.y;
+    seg.ntiles = d.z;
+    seg.whole = d.w < 0;
+    len = d.w & 0x7fffffff;
+    return true;
+  }
+};
+
 template <int DBLK, int T, int NS>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
 mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
@@ -189,18 +211,23 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int col0 = branch * DBLK;  // first latent column of this CTA's branch
-  // Everything above overlapped the prep kernel; its lengths and tile prefix are needed now.
+  // Everything above overlapped the prep kernel; its segment descriptors are needed now.
   pdl_wait_prerequisites();
-  const int64_t total = p.prefix[p.N];
-  const int64_t R = effective_ranges(p.num_ranges, total);
+  RangeInfo rinfo;
+  {
+    const int2 r2 = __ldcg(reinterpret_cast<const int2*>(p.ranges + range));
+    rinfo.first = r2.x;
+    rinfo.count = r2.y;
+  }
 
   if (warp == 4) {
     // ------------------------------------------------------------------ TMA producer
-    SegmentWalker walk(p.prefix, p.N, total, R, range);
+    SegCursor walk(p.segs, rinfo);
     Segment seg;
+    int L = 0;
     int it = 0, nseg = 0;
     bool ok = true;
-    while (ok && walk.next(seg)) {
+    while (ok && walk.next(seg, L)) {
       if (nseg > 0) ok = wait_warp(bar_q_empty, (nseg - 1) & 1, tmo, abort_flag, p.status);
       if (!ok) break;
       if (lane == 0) {
@@ -211,7 +238,6 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         tma_load_3d(sQ + C::NCB * C::BOX, &tm_qr, bar_q_full, 0, 0, seg.seq);
       }
       __syncwarp();
-      const int L = p.lens[seg.seq];
       for (int i = 0; i < seg.ntiles; ++i, ++it) {
         // cache rows of the tile's 64-position sub-boxes (past the sequence end: zeros)
         int rows[C::TB];
@@ -253,11 +279,12 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   } else if (warp == 5) {
     // ------------------------------------------------------------------ score-MMA issuer
     constexpr uint32_t kIdScore = idesc_bf16_f32(64, T, false, false);
-    SegmentWalker walk(p.prefix, p.N, total, R, range);
+    SegCursor walk(p.segs, rinfo);
     Segment seg;
+    int L = 0;
     int it = 0, nseg = 0;
     bool ok = true;
-    while (ok && walk.next(seg)) {
+    while (ok && walk.next(seg, L)) {
       ok = wait_warp(bar_q_full, nseg & 1, tmo, abort_flag, p.status);
       for (int i = 0; ok && i < seg.ntiles; ++i, ++it) {
         ok = wait_warp(bar_stage_full + 8 * (it % NS), (it / NS) & 1, tmo, abort_flag, p.status);
@@ -298,11 +325,12 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   } else if (warp == 6) {
     // ------------------------------------------------------------------ output-MMA issuer
     constexpr uint32_t kIdPV = idesc_bf16_f32(64, C::OCW, false, true);
-    SegmentWalker walk(p.prefix, p.N, total, R, range);
+    SegCursor walk(p.segs, rinfo);
     Segment seg;
+    int L = 0;
     int j = 0;
     bool ok = true;
-    while (ok && walk.next(seg)) {
+    while (ok && walk.next(seg, L)) {
       for (int i = 0; i < seg.ntiles; ++i, ++j) {
         ok = wait_warp(bar_p_full + 8 * (j % NSB), (j / NSB) & 1, tmo, abort_flag, p.status);
         if (!ok) break;
@@ -338,12 +366,12 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int q = lane >> 4;                   // which half of the row's columns
     const int h = 16 * warp + (lane & 15);     // head
     const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-    SegmentWalker walk(p.prefix, p.N, total, R, range);
+    SegCursor walk(p.segs, rinfo);
     Segment seg;
+    int L = 0;
     int it = 0;
     bool ok = true;
-    while (ok && walk.next(seg)) {
-      const int L = p.lens[seg.seq];
+    while (ok && walk.next(seg, L)) {
       float m_used = -CUDART_INF_F, l_sum = 0.f;
       for (int i = 0; i < seg.ntiles; ++i, ++it) {
         const int t = seg.tile0 + i;
@@ -502,6 +530,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   __syncthreads();
   tc_fence_after();
   if (warp == 5) tmem_dealloc(tmem, C::TMEM_COLS);
+
 }
 
 }  // namespace mlra

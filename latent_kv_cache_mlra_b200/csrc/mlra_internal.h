@@ -11,10 +11,35 @@ constexpr uint32_t kFlagTimeout = 0x1u;
 constexpr uint32_t kFlagBadPage = 0x2u;
 constexpr uint32_t kFlagBadLength = 0x4u;
 
+// The split plan as the prep kernel writes it for the decode and combine kernels.
+//   RangeInfo[r]  : descriptors segs[first, first + count) of work range r, in tile order
+//   SegDesc       : one (range, sequence) overlap; its partial slot is r + seq
+//   SeqInfo[s]    : ranges r0 .. r0 + nparts - 1 hold sequence s (its partial slots r0 + p + s)
+struct alignas(8) RangeInfo { int32_t first, count; };
+struct alignas(16) SegDesc {
+  int32_t seq, tile0, ntiles;  // tile0: first tile counted inside the sequence
+  int32_t len_whole;           // bits 0-30: sequence length; bit 31: the segment is the whole sequence
+};
+struct alignas(8) SeqInfo { int32_t r0, nparts; };
+
+struct PrepParams {
+  const int32_t* seq_lens;    // caller lengths [N]
+  int N, limit, tile, num_ranges;
+  int32_t* lens;              // clamped lengths [N]
+  int32_t* prefix;            // tile prefix sums [N + 1]
+  RangeInfo* ranges;          // [num_ranges]
+  SegDesc* segs;              // [num_ranges + N - 1]
+  SeqInfo* seqs;              // [N]
+  uint32_t* status;           // rewritten
+  float* out;                 // rows of empty sequences are zeroed ...
+  float* lse;                 // ... and their lse set to -inf (nullable)
+  int H, B, out_width;        // out: [N, H, out_width], lse: [N, H, B]
+};
+
 // Parameters of the split-KV decode kernel (K1).
 struct DecodeParams {
-  const int32_t* lens;        // clamped sequence lengths [N]
-  const int32_t* prefix;      // tile prefix sums [N + 1]
+  const RangeInfo* ranges;    // [num_ranges] (prep kernel)
+  const SegDesc* segs;
   const int32_t* page_table;  // [N, max_pages] or nullptr (contiguous)
   float* out;                 // final output, row width out_width, or nullptr
   float* lse;                 // [N, H, B] or nullptr
@@ -37,7 +62,7 @@ struct DecodeParams {
 };
 
 struct CombineParams {
-  const int32_t* prefix;      // tile prefix sums [N + 1]
+  const SeqInfo* seqs;        // [N] (prep kernel)
   const float* part_o;
   const float* part_ml;
   float* out;
@@ -45,8 +70,7 @@ struct CombineParams {
   int N, H, B;
   int dblk_k, dck;            // kernel branch width and latent width
   int d_blk_out;              // caller branch width
-  int num_ranges;
-  int max_parts;              // upper bound on the parts of one sequence (shared-memory sizing)
+  int groups;                 // part groups per head (1, 2, 4 or 8): parts are split across warps
   int summed;                 // 1: out[s,h,:d_blk_out] = sum over branches
   int final_written;          // 1: sequences held in one part were written by K1
   float gamma;
@@ -65,8 +89,7 @@ enum Variant { kV64 = 0, kV128, kV256, kV512, kNumVariants };
 
 int variant_smem_bytes(Variant v);
 int variant_tile(Variant v);  // KV positions per tile (64 or 128)
-cudaError_t launch_prep(const int32_t* seq_lens, int N, int limit, int tile, int32_t* lens_out,
-                        int32_t* prefix, uint32_t* status, cudaStream_t st);
+cudaError_t launch_prep(const PrepParams& p, cudaStream_t st);
 cudaError_t launch_decode(Variant v, const CUtensorMap& tq, const CUtensorMap& tqr,
                           const CUtensorMap& tc, const CUtensorMap& tkr, const DecodeParams& p,
                           int grid, cudaStream_t st);

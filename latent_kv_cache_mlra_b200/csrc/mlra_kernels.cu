@@ -1,5 +1,6 @@
 // mlra_kernels.cu -- device kernels of the MLRA decode library and their launchers.
-//   K0 mlra_prep_kernel      lengths -> clamped lengths, tile prefix sums, status word reset
+//   K0 mlra_prep_kernel      lengths -> clamped lengths, tile prefix sums, segment
+//                            descriptors, empty-sequence outputs, status word reset
 //   K1 mlra_decode_kernel    split-KV decode attention (mlra_decode_kernel.cuh)
 //   K2 mlra_combine_kernel   merges the partial softmax states of split sequences
 //   K3 mlra_repack_kernel    fp32 / odd-width inputs -> padded bf16 copies in the workspace
@@ -8,6 +9,7 @@
 #include <math_constants.h>
 
 #include "mlra_decode_kernel.cuh"
+#include "mlra_merge.cuh"
 #include "sm100_ptx.cuh"
 #include "mlra_internal.h"
 #include "mlra_plan.cuh"
@@ -17,13 +19,23 @@ namespace mlra {
 // ----------------------------------------------------------------------------- K0
 // One block.  seq_lens outside [0, limit] set kFlagBadLength and are clamped; the status word
 // is rewritten so that it reports this call only.  prefix counts tiles of `tile` positions.
-__global__ void __launch_bounds__(1024) mlra_prep_kernel(const int32_t* seq_lens, int N, int limit,
-                                                         int tile, int32_t* lens_out,
-                                                         int32_t* prefix, uint32_t* status) {
+// Then the split plan for the decode and combine kernels: per work range its segment
+// descriptors (range r's first descriptor sits at r + its first sequence, which keeps the
+// ranges' descriptor blocks disjoint) and per sequence the ranges holding it.  Empty sequences
+// get out = 0, lse = -inf here.  For up to kPrepSmemSeqs sequences the prefix and the lengths
+// are also kept in shared memory, where the per-range searches read them.
+constexpr int kPrepSmemSeqs = 4096;
+
+__global__ void __launch_bounds__(1024) mlra_prep_kernel(const PrepParams p) {
   __shared__ int32_t warp_tot[32];
   __shared__ int32_t carry;
   __shared__ uint32_t flags;
+  extern __shared__ int32_t sh_plan[];  // [N + 1] prefix, [N] lens (when N <= kPrepSmemSeqs)
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int N = p.N;
+  const bool in_smem = N <= kPrepSmemSeqs;
+  int32_t* prefix = in_smem ? sh_plan : p.prefix;
+  int32_t* lens = in_smem ? sh_plan + N + 1 : p.lens;
   pdl_launch_dependents();  // the decode kernel may start its prologue now
   if (tid == 0) {
     carry = 0;
@@ -35,13 +47,13 @@ __global__ void __launch_bounds__(1024) mlra_prep_kernel(const int32_t* seq_lens
     const int i = base + tid;
     int tiles = 0;
     if (i < N) {
-      int L = seq_lens[i];
-      if (L < 0 || L > limit) {
+      int L = p.seq_lens[i];
+      if (L < 0 || L > p.limit) {
         atomicOr(&flags, kFlagBadLength);
-        L = L < 0 ? 0 : limit;
+        L = L < 0 ? 0 : p.limit;
       }
-      lens_out[i] = L;
-      tiles = (L + tile - 1) / tile;
+      lens[i] = L;
+      tiles = (L + p.tile - 1) / p.tile;
     }
     int x = tiles;  // inclusive warp scan
 #pragma unroll
@@ -67,12 +79,46 @@ __global__ void __launch_bounds__(1024) mlra_prep_kernel(const int32_t* seq_lens
     if (tid == 1023) carry = incl;
     __syncthreads();
   }
-  if (tid == 0) *status = flags;
+  // prefix and lens written above are visible to the whole block after the last __syncthreads
+  const int64_t total = prefix[N];
+  const int64_t R = effective_ranges(p.num_ranges, total);
+  for (int r = tid; r < p.num_ranges; r += blockDim.x) {
+    RangeInfo ri{0, 0};
+    if (r < R && total > 0) {
+      SegmentWalker walk(prefix, N, total, R, r);
+      Segment seg;
+      ri.first = -1;
+      while (walk.next(seg)) {
+        if (ri.first < 0) ri.first = r + seg.seq;
+        SegDesc d;
+        d.seq = seg.seq;
+        d.tile0 = seg.tile0;
+        d.ntiles = seg.ntiles;
+        d.len_whole = lens[seg.seq] | (seg.whole ? (int32_t)0x80000000u : 0);
+        p.segs[ri.first + ri.count] = d;
+        ++ri.count;
+      }
+    }
+    p.ranges[r] = ri;
+  }
+  for (int sq = tid; sq < N; sq += blockDim.x) {
+    SeqInfo si{0, 0};
+    if (total > 0) seq_parts(prefix, sq, total, R, &si.r0, &si.nparts);
+    p.seqs[sq] = si;
+  }
+  for (int sq = wid; sq < N; sq += 32) {  // empty sequences (a warp each): out = 0, lse = -inf
+    if (lens[sq] != 0) continue;
+    float* row = p.out + (int64_t)sq * p.H * p.out_width;
+    for (int i = lane; i < p.H * p.out_width; i += 32) row[i] = 0.f;
+    if (p.lse)
+      for (int i = lane; i < p.H * p.B; i += 32) p.lse[(int64_t)sq * p.H * p.B + i] = -CUDART_INF_F;
+  }
+  if (tid == 0) *p.status = flags;
 }
 
-cudaError_t launch_prep(const int32_t* seq_lens, int N, int limit, int tile, int32_t* lens_out,
-                        int32_t* prefix, uint32_t* status, cudaStream_t st) {
-  mlra_prep_kernel<<<1, 1024, 0, st>>>(seq_lens, N, limit, tile, lens_out, prefix, status);
+cudaError_t launch_prep(const PrepParams& p, cudaStream_t st) {
+  const size_t sh = p.N <= kPrepSmemSeqs ? (2 * (size_t)p.N + 1) * sizeof(int32_t) : 0;
+  mlra_prep_kernel<<<1, 1024, sh, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -135,96 +181,77 @@ cudaError_t launch_decode(Variant v, const CUtensorMap& tq, const CUtensorMap& t
 }
 
 // ----------------------------------------------------------------------------- K2
-// Grid (H, N, column chunks of 128), 128 threads.  For sequence s split into parts (ranges
-// r0 .. r0+np-1, slot r + s), per branch b: m* = max_p m_p, l* = sum_p 2^(m_p - m*) l_p and
-//   out = gamma * sum_p 2^(m_p - m*) o_p / l*,   lse = (m* + log2 l*) ln 2.
-// Scores are kept in log2 units by K1.  The per-part weights gamma 2^(m_p - m*) / l* of every
-// branch are computed once per block into shared memory.
-__global__ void __launch_bounds__(128) mlra_combine_kernel(const CombineParams p) {
-  const int h = blockIdx.x, s = blockIdx.y, chunk = blockIdx.z;
+// Merge of split sequences.  For sequence s split into np parts (ranges r0 .. r0+np-1; part p
+// in slot r0 + p + s), per head h and branch b the parts are folded as in mlra_merge.cuh;
+// summed mode adds the branches' gamma o* / l*.  Launched with programmatic stream
+// serialization: its blocks may be scheduled during the decode kernel and wait for it.
+// Grid (N, ceil(H / HG), column chunks of 128), 256 threads = 8 warps = HG heads x G part groups.
+// Lane t of a warp covers 4 columns (128 per warp); part group g takes parts g, g+G, ...; the G
+// group states of a head are merged in shared memory.  Empty sequences were written by K0.
+constexpr int kCombineWarps = 8;
+
+__global__ void __launch_bounds__(kCombineWarps * 32) mlra_combine_kernel(const CombineParams p) {
+  __shared__ MergeState part[kCombineWarps][32];
+  const int s = blockIdx.x;
+  const int G = p.groups, HG = kCombineWarps / G;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y * HG + warp / G, g = warp % G;
+  const bool live_h = h < p.H;
+  // padded column of this lane: branch mode over [0, dck), summed mode over [0, dblk_k)
+  const int k = blockIdx.z * 128 + 4 * lane;
+  const bool live = live_h && k < (p.summed ? p.dblk_k : p.dck);
   pdl_wait_prerequisites();  // the decode kernel's partials must be complete and visible
-  const int64_t total = p.prefix[p.N];
-  int r0 = 0, np = 0;
-  if (total > 0) seq_parts(p.prefix, s, total, effective_ranges(p.num_ranges, total), &r0, &np);
-  if (np == 1 && p.final_written) return;
+  const int2 si = __ldcg(reinterpret_cast<const int2*>(p.seqs + s));  // (r0, nparts)
+  const int np = si.y;
+  if (np == 0 || (np == 1 && p.final_written)) return;  // written by K0 / by the decode kernel
   const int width = p.summed ? p.d_blk_out : p.B * p.d_blk_out;
-  const int c = chunk * 128 + threadIdx.x;
   float* out_row = p.out + ((int64_t)s * p.H + h) * width;
-  if (np == 0) {
-    if (c < width) out_row[c] = 0.f;
-    if (p.lse && chunk == 0 && threadIdx.x < p.B)
-      p.lse[((int64_t)s * p.H + h) * p.B + threadIdx.x] = -CUDART_INF_F;
-    return;
-  }
-  extern __shared__ float sh[];  // m[np][B] (then the weights), l[np][B], m*[B], l*[B]
-  float* wts = sh;
-  float* lpart = sh + np * p.B;
-  float* mstar = lpart + np * p.B;
-  float* lstar = mstar + p.B;
-  const int64_t slot0 = (int64_t)r0 + s;
-  const int n_ml = np * p.B;
-  // 1. every (part, branch) state in parallel
-  for (int k = threadIdx.x; k < n_ml; k += blockDim.x) {
-    const int q = k / p.B, b = k - q * p.B;
-    const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + (((slot0 + q) * p.H + h) * p.B + b) * 2);
-    wts[k] = ml.x;
-    lpart[k] = ml.y;
-  }
-  __syncthreads();
-  // 2. per branch: m* = max_p m_p
-  for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
-    float m = -CUDART_INF_F;
-    for (int q = 0; q < np; ++q) m = fmaxf(m, wts[q * p.B + b]);
-    mstar[b] = m;
-  }
-  __syncthreads();
-  // 3. w_p = 2^(m_p - m*) (unnormalised), in parallel
-  for (int k = threadIdx.x; k < n_ml; k += blockDim.x) wts[k] = exp2f(wts[k] - mstar[k % p.B]);
-  __syncthreads();
-  // 4. l* = sum_p w_p l_p, then fold gamma / l* into the weights
-  for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
-    float l = 0.f;
-    for (int q = 0; q < np; ++q) l += wts[q * p.B + b] * lpart[q * p.B + b];
-    lstar[b] = l;
-    if (p.lse && chunk == 0)
-      p.lse[((int64_t)s * p.H + h) * p.B + b] = (mstar[b] + log2f(l)) * 0.69314718055994531f;
-  }
-  __syncthreads();
-  for (int k = threadIdx.x; k < n_ml; k += blockDim.x) wts[k] *= p.gamma / lstar[k % p.B];
-  __syncthreads();
-  if (c >= width) return;
-  const float* po = p.part_o + (slot0 * p.H + h) * p.dck;
-  const int64_t pstride = (int64_t)p.H * p.dck;  // next part of the same (s, h)
-  if (!p.summed) {
-    const int b = c / p.d_blk_out;
-    const float* src = po + b * p.dblk_k + (c - b * p.d_blk_out);
-    float acc = 0.f;
-#pragma unroll 4
-    for (int q = 0; q < np; ++q) acc += wts[q * p.B + b] * src[q * pstride];
-    out_row[c] = acc;
-  } else {
-    float acc = 0.f;
-    for (int b = 0; b < p.B; ++b) {
-      const float* src = po + b * p.dblk_k + c;
-#pragma unroll 4
-      for (int q = 0; q < np; ++q) acc += wts[q * p.B + b] * src[q * pstride];
+  const int64_t slot0 = (int64_t)si.x + s;
+  const int b_lo = p.summed ? 0 : k / p.dblk_k;
+  const int b_hi = p.summed ? p.B : b_lo + 1;
+  MergeState tot = merge_empty();
+  tot.acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int b = b_lo; b < b_hi; ++b) {  // block-uniform trip count (1 in branch mode)
+    const int kb = p.summed ? b * p.dblk_k + k : k;
+    MergeState st = merge_empty();
+    if (live) st = fold_parts(p.part_ml, p.part_o, p.H, p.B, p.dck, slot0, np, g, G, h, b, kb);
+    if (G > 1) {
+      part[warp][lane] = st;
+      __syncthreads();
+      if (g == 0)
+        for (int j = 1; j < G; ++j) {
+          const MergeState o = part[warp + j][lane];
+          merge_into(st, o.m, o.l, o.acc);
+        }
+      __syncthreads();  // part[] is rewritten by the next branch
     }
-    out_row[c] = acc;
+    if (!live || g != 0) continue;
+    if (p.lse && (p.summed ? (blockIdx.z == 0 && lane == 0) : (k - b * p.dblk_k == 0)))
+      p.lse[((int64_t)s * p.H + h) * p.B + b] = merged_lse(st);
+    if (p.summed) {
+      const float sc = p.gamma / st.l;
+      tot.acc.x += st.acc.x * sc; tot.acc.y += st.acc.y * sc;
+      tot.acc.z += st.acc.z * sc; tot.acc.w += st.acc.w * sc;
+    } else {
+      const int kk = k - b * p.dblk_k;
+      if (kk < p.d_blk_out) store_merged(out_row + b * p.d_blk_out + kk, st, p.gamma, p.d_blk_out - kk);
+    }
+  }
+  if (p.summed && live && g == 0 && k < p.d_blk_out) {
+    tot.l = 1.f;
+    store_merged(out_row + k, tot, 1.f, p.d_blk_out - k);
   }
 }
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t st) {
-  const int width = p.summed ? p.d_blk_out : p.B * p.d_blk_out;
-  const size_t sh = (2 * (size_t)p.max_parts * p.B + 2 * p.B) * sizeof(float);
-  if (sh > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(mlra_combine_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);
-    if (e != cudaSuccess) return e;
-  }
+  if (p.groups < 1 || p.groups > kCombineWarps || kCombineWarps % p.groups != 0)
+    return cudaErrorInvalidValue;
+  const int HG = kCombineWarps / p.groups;
+  const int kspan = p.summed ? p.dblk_k : p.dck;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.H, p.N, (width + 127) / 128);
-  cfg.blockDim = dim3(128);
-  cfg.dynamicSmemBytes = sh;
+  cfg.gridDim = dim3(p.N, (p.H + HG - 1) / HG, (kspan + 127) / 128);
+  cfg.blockDim = dim3(kCombineWarps * 32);
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap the decode tail

@@ -7,8 +7,8 @@
 // sequence, whole sequences and the head of another: each (range, sequence) overlap is a
 // segment with its own partial softmax state, stored in partial slot r + s (slots are unique
 // because both r and s never decrease along the tile order).  A sequence split over several
-// ranges is merged by the combine kernel.  The plan depends only on the logical lengths, never
-// on physical page ids.  When the batch has fewer tiles than ranges, the number of ranges is
+// ranges is merged inside the decode kernel, by the CTA that finishes the last of its parts.
+// The plan depends only on the logical lengths, never on physical page ids.  When the batch has fewer tiles than ranges, the number of ranges is
 // cut to the tile count (effective_ranges) so that every range holds at least one tile and the
 // ranges covering one sequence are consecutive.
 #pragma once
@@ -55,12 +55,13 @@ struct SegmentWalker {
   int n;
   int64_t g, end;
   int s;
-  // A range index r >= R (a CTA beyond the effective ranges) walks nothing.
+  // A range index r >= R (a CTA beyond the effective ranges) walks nothing.  first_seq >= 0 is
+  // the sequence holding the range's first tile when the caller knows it (saves the search).
   __host__ __device__ SegmentWalker(const int32_t* prefix_, int n_, int64_t total, int64_t R,
-                                    int64_t r)
+                                    int64_t r, int first_seq = -1)
       : prefix(prefix_), n(n_), g(r < R ? range_begin(r, total, R) : total),
         end(r < R ? range_begin(r + 1, total, R) : total), s(0) {
-    if (g < end) s = seq_of_tile(prefix, n, g);
+    if (g < end) s = first_seq >= 0 ? first_seq : seq_of_tile(prefix, n, g);
   }
   __host__ __device__ bool next(Segment& seg) {
     if (g >= end) return false;

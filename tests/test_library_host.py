@@ -43,11 +43,13 @@ def dims(**kw):
 
 
 def test_workspace_size_layout():
-    # status 256 + lens + prefix + (R + N - 1) slots of (m, l) and partial outputs
+    # status 256 + lens + prefix + plan (a range record per range, a segment descriptor per
+    # slot, a sequence record per sequence) + (R + N - 1) slots of (m, l) and partial outputs
     n = mlra.workspace_size(dims())
-    slots, H, B, dck = 74 + 8 - 1, 64, 4, 512
-    expect_min = 256 + slots * H * B * 2 * 4 + slots * H * dck * 4
-    assert expect_min <= n <= expect_min + 5 * 256 + 64
+    slots, H, B, dck, R, N = 74 + 8 - 1, 64, 4, 512, 74, 8
+    plan = 8 * R + 16 * slots + 8 * N
+    expect_min = 256 + plan + slots * H * B * 2 * 4 + slots * H * dck * 4
+    assert expect_min <= n <= expect_min + 8 * 256 + 64
     # fp32 input adds padded bf16 copies of queries and cache
     n32 = mlra.workspace_size(dims(dtype="f32"))
     assert n32 - n >= 8 * 32768 * (512 + 64) * 2
