@@ -150,6 +150,7 @@ typedef struct {
   int branches_per_cta;   /* branches whose latent columns one attention CTA reads */
   int tile;               /* KV positions per tile (64 or 128) */
   long long partial_slots;/* partial-result slots in the workspace (num_ranges + N - 1) */
+  int segment_cost_tiles; /* plan balance: tiles a sequence start costs a CTA (mlra_plan_host) */
   size_t workspace_bytes;
 } mlra_plan_info;
 mlra_status mlra_query_plan(const mlra_dims* dims, mlra_plan_info* info_host);
@@ -190,12 +191,17 @@ mlra_status mlra_debug_resolve_rows(const int32_t* seq_lens, const int32_t* page
                                     const mlra_dims* dims, int64_t* rows_out, int row_pitch,
                                     mlra_stream_t stream);
 
-/* Host replica of the split plan (the same __host__ __device__ code the kernels run): for
- * tile counts tiles_host[N] cut into min(num_ranges, total tiles) equal ranges, writes for every
- * sequence the first range touching it and the number of ranges (partial results) it is split
- * into (0 for an empty sequence).
+/* Host replica of the split plan (the same __host__ __device__ code the kernels run): tile
+ * counts tiles_host[N] are cut into min(num_ranges, total tiles) contiguous ranges that balance
+ * tiles plus seg_cost tiles per non-empty sequence (each range r starts at the virtual position
+ * floor(r V / R) of the virtual length V = sum of (tiles + seg_cost) over non-empty sequences;
+ * a position inside a sequence's seg_cost leading slots maps to the sequence's first tile).  The
+ * attention kernel uses seg_cost = mlra_plan_info.segment_cost_tiles; 0 gives equal ranges.
+ * Writes for every sequence the first range touching it and the number of ranges (partial
+ * results) it is split into (0 for an empty sequence).  Errors: MLRA_ERR_INVALID_ARG for a
+ * negative tile count or seg_cost, num_ranges < 1, n < 1, or a virtual length past INT_MAX.
  * Host only, synchronous; for tests and tooling. */
-mlra_status mlra_plan_host(const int32_t* tiles_host, int n, int num_ranges,
+mlra_status mlra_plan_host(const int32_t* tiles_host, int n, int num_ranges, int seg_cost,
                            int32_t* first_range_host, int32_t* num_parts_host);
 
 /* Host replica of the per-CTA segment walk of the attention kernel: for tile counts
@@ -203,7 +209,7 @@ mlra_status mlra_plan_host(const int32_t* tiles_host, int n, int num_ranges,
  * tile, tile count) segment that the kernel's CTAs r = 0 .. num_ranges-1 process, in CTA order.
  * At most max_segments are written to the four *_host arrays; *count_host receives the total.
  * Host only, synchronous; for tests and tooling. */
-mlra_status mlra_plan_segments_host(const int32_t* tiles_host, int n, int num_ranges,
+mlra_status mlra_plan_segments_host(const int32_t* tiles_host, int n, int num_ranges, int seg_cost,
                                     int32_t* range_host, int32_t* seq_host, int32_t* tile0_host,
                                     int32_t* ntiles_host, int max_segments, int* count_host);
 

@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <array>
 #include <mutex>
 #include <vector>
 
@@ -33,10 +34,16 @@ struct Plan {
   int R = 0;           // work ranges
   int64_t slots = 0;   // partial slots = R + N - 1
   int limit = 0;       // bound on seq_lens
-  size_t off_lens = 0, off_prefix = 0, off_ranges = 0, off_segs = 0, off_seqs = 0;
+  int seg_cost = 0;    // tiles a sequence start costs a CTA (plan balance)
+  bool self_plan = false;  // the decode kernel plans its ranges (no prep kernel)
+  size_t off_scratch = 0, off_ranges = 0, off_segs = 0, off_seqs = 0, off_flags = 0;
   size_t off_ml = 0, off_o = 0;
   size_t off_rq = 0, off_rqr = 0, off_rc = 0, off_rkr = 0, total = 0;
 };
+
+// Tiles of streaming that a sequence start inside a work range costs a CTA (the segment's
+// epilogue and the next queries' load), measured at 2 to 3.5 tiles on B200.
+constexpr int kSegmentCostTiles = 3;
 
 int device_sm_count(mlra_status* st) {
   int dev = 0;
@@ -98,11 +105,16 @@ mlra_status make_plan(const mlra_dims* d, bool paged, int sms, Plan* pl) {
   pl->limit = paged ? d->max_pages_per_seq * d->page_size : d->max_seq_len;
   if (!paged) pl->limit = d->max_seq_len;
   else if (d->max_seq_len > 0 && d->max_seq_len < pl->limit) pl->limit = d->max_seq_len;
+  pl->seg_cost = kSegmentCostTiles;
+  // the plan's (virtual) tile prefix must fit int32
+  if ((int64_t)d->batch * ((pl->limit + pl->tile - 1) / pl->tile + pl->seg_cost) > INT_MAX)
+    return MLRA_ERR_INVALID_ARG;
 
   const int64_t N = d->batch, H = d->heads;
   size_t off = kAlign;  // status word + padding
-  pl->off_lens = off; off = align_up(off + 4 * N);
-  pl->off_prefix = off; off = align_up(off + 4 * (N + 1));
+  pl->self_plan = N <= kSelfPlanMaxSeqs;
+  pl->off_scratch = off; off = align_up(off + 4 * (5 * (size_t)N + 2));
+  pl->off_flags = off; off = align_up(off + 4 * ((size_t)pl->R * pl->n_groups + 1));
   pl->off_ranges = off; off = align_up(off + sizeof(RangeInfo) * (size_t)pl->R);
   pl->off_segs = off; off = align_up(off + sizeof(SegDesc) * (size_t)pl->slots);
   pl->off_seqs = off; off = align_up(off + sizeof(SeqInfo) * (size_t)N);
@@ -212,13 +224,14 @@ mlra_status mlra_query_plan(const mlra_dims* dims, mlra_plan_info* info) {
   mlra_status st = make_plan(dims, paged, sms, &pl);
   if (st != MLRA_OK) return st;
   info->repack = pl.repack ? 1 : 0;
-  info->launches = 3 + (pl.repack ? 1 : 0);
+  info->launches = (pl.self_plan ? 2 : 3) + (pl.repack ? 1 : 0);
   info->num_ranges = pl.R;
   info->ctas = pl.R * pl.n_groups;
   info->kernel_branch_width = pl.dblk_k;
   info->branches_per_cta = 1;
   info->tile = pl.tile;
   info->partial_slots = pl.slots;
+  info->segment_cost_tiles = pl.seg_cost;
   info->workspace_bytes = pl.total;
   return MLRA_OK;
 }
@@ -262,8 +275,7 @@ mlra_status mlra_decode_profiled(const void* q_lat, const void* q_rope, const vo
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
-  int32_t* lens = reinterpret_cast<int32_t*>(ws + pl.off_lens);
-  int32_t* prefix = reinterpret_cast<int32_t*>(ws + pl.off_prefix);
+  int32_t* plan_scratch = reinterpret_cast<int32_t*>(ws + pl.off_scratch);
   float* part_ml = reinterpret_cast<float*>(ws + pl.off_ml);
   float* part_o = reinterpret_cast<float*>(ws + pl.off_o);
   RangeInfo* ranges = reinterpret_cast<RangeInfo*>(ws + pl.off_ranges);
@@ -306,17 +318,25 @@ mlra_status mlra_decode_profiled(const void* q_lat, const void* q_rope, const vo
 
   const bool summed = dims->out_mode == MLRA_OUT_SUMMED;
   const int out_width = summed ? dblk : dims->d_latent;  // floats per (sequence, head) row of out
-  PrepParams pp;
-  pp.seq_lens = seq_lens; pp.N = N; pp.limit = pl.limit; pp.tile = pl.tile; pp.num_ranges = pl.R;
-  pp.lens = lens; pp.prefix = prefix; pp.ranges = ranges; pp.segs = segs; pp.seqs = seqs;
-  pp.status = status;
-  pp.out = out; pp.lse = lse; pp.H = H; pp.B = B; pp.out_width = out_width;
-  if (launch_prep(pp, s) != cudaSuccess) return MLRA_ERR_CUDA;
+  const int grid = pl.R * pl.n_groups;
+  uint32_t* cta_flags = reinterpret_cast<uint32_t*>(ws + pl.off_flags);  // [grid] + prep's slot
+  if (!pl.self_plan) {
+    PrepParams pp;
+    pp.seq_lens = seq_lens; pp.N = N; pp.limit = pl.limit; pp.tile = pl.tile; pp.num_ranges = pl.R;
+    pp.seg_cost = pl.seg_cost; pp.scratch = plan_scratch;
+    pp.ranges = ranges; pp.segs = segs; pp.seqs = seqs;
+    pp.flags = cta_flags + grid;
+    pp.out = out; pp.lse = lse; pp.H = H; pp.B = B; pp.out_width = out_width;
+    if (launch_prep(pp, s) != cudaSuccess) return MLRA_ERR_CUDA;
+  }
 
   DecodeParams p;
   p.ranges = ranges; p.segs = segs;
+  p.self_plan = pl.self_plan ? 1 : 0;
+  p.seq_lens = seq_lens; p.limit = pl.limit; p.tile = pl.tile; p.seg_cost = pl.seg_cost;
+  p.seqs = seqs; p.cta_flags = cta_flags;
   p.page_table = page_table;
-  p.out = out; p.lse = lse; p.part_o = part_o; p.part_ml = part_ml; p.status = status;
+  p.out = out; p.lse = lse; p.part_o = part_o; p.part_ml = part_ml;
   p.N = N; p.H = H; p.B = B; p.d_blk_out = dblk; p.out_width = out_width; p.dck = pl.dck;
   p.n_groups = pl.n_groups; p.num_ranges = pl.R;
   p.page_size = paged ? dims->page_size : 0;
@@ -330,12 +350,13 @@ mlra_status mlra_decode_profiled(const void* q_lat, const void* q_rope, const vo
   p.timeout_ns = kTimeoutNs;
   if (k1_begin && cudaEventRecord(reinterpret_cast<cudaEvent_t>(k1_begin), s) != cudaSuccess)
     return MLRA_ERR_CUDA;
-  if (launch_decode(pl.variant, tq, tqr, tc, tkr, p, pl.R * pl.n_groups, s) != cudaSuccess)
+  if (launch_decode(pl.variant, tq, tqr, tc, tkr, p, grid, s) != cudaSuccess)
     return MLRA_ERR_CUDA;
   if (k1_end && cudaEventRecord(reinterpret_cast<cudaEvent_t>(k1_end), s) != cudaSuccess)
     return MLRA_ERR_CUDA;
 
   CombineParams cp;
+  cp.cta_flags = cta_flags; cp.n_flag_slots = grid + (pl.self_plan ? 0 : 1); cp.status = status;
   cp.seqs = seqs; cp.part_o = part_o; cp.part_ml = part_ml; cp.out = out; cp.lse = lse;
   cp.N = N; cp.H = H; cp.B = B; cp.dblk_k = pl.dblk_k; cp.dck = pl.dck; cp.d_blk_out = dblk;
   cp.summed = summed ? 1 : 0;
@@ -417,54 +438,73 @@ mlra_status mlra_debug_resolve_rows(const int32_t* seq_lens, const int32_t* page
   return MLRA_OK;
 }
 
-mlra_status mlra_plan_host(const int32_t* tiles_host, int n, int num_ranges,
-                           int32_t* first_range_host, int32_t* num_parts_host) {
-  if (!tiles_host || !first_range_host || !num_parts_host || n < 1 || num_ranges < 1)
-    return MLRA_ERR_INVALID_ARG;
-  std::vector<int32_t> prefix(n + 1, 0);
+namespace {
+// The plan of the prep kernel, on the host: per sequence the first and last range holding it,
+// and the segments in range order (optional).
+mlra_status host_plan(const int32_t* tiles, int n, int num_ranges, int seg_cost,
+                      std::vector<int32_t>* first_r, std::vector<int32_t>* last_r,
+                      std::vector<std::array<int32_t, 4>>* segs) {
+  if (!tiles || n < 1 || num_ranges < 1 || seg_cost < 0) return MLRA_ERR_INVALID_ARG;
+  std::vector<int32_t> prefix(n + 1, 0), vprefix(n + 1, 0);
   for (int i = 0; i < n; ++i) {
-    if (tiles_host[i] < 0) return MLRA_ERR_INVALID_ARG;
-    const int64_t next = (int64_t)prefix[i] + tiles_host[i];
-    if (next > INT_MAX) return MLRA_ERR_INVALID_ARG;
+    if (tiles[i] < 0) return MLRA_ERR_INVALID_ARG;
+    const int64_t next = (int64_t)prefix[i] + tiles[i];
+    const int64_t vnext = (int64_t)vprefix[i] + tiles[i] + (tiles[i] > 0 ? seg_cost : 0);
+    if (vnext > INT_MAX) return MLRA_ERR_INVALID_ARG;
     prefix[i + 1] = static_cast<int32_t>(next);
+    vprefix[i + 1] = static_cast<int32_t>(vnext);
   }
-  const int64_t total = prefix[n];
+  PlanView pv;
+  pv.prefix = prefix.data();
+  pv.vprefix = vprefix.data();
+  pv.n = n;
+  pv.total = prefix[n];
+  pv.vtotal = vprefix[n];
+  pv.R = effective_ranges(num_ranges, pv.total);
+  pv.cost = seg_cost;
+  first_r->assign(n, 0);
+  last_r->assign(n, -1);
+  if (pv.total == 0) return MLRA_OK;
+  for (int64_t r = 0; r < pv.R; ++r) {
+    SegmentWalker walk(prefix.data(), n, range_start(pv, r), range_start(pv, r + 1));
+    Segment seg;
+    while (walk.next(seg)) {
+      if (seg.tile0 == 0) (*first_r)[seg.seq] = static_cast<int32_t>(r);
+      if (seg.tile0 + seg.ntiles == tiles[seg.seq]) (*last_r)[seg.seq] = static_cast<int32_t>(r);
+      if (segs) segs->push_back({static_cast<int32_t>(r), seg.seq, seg.tile0, seg.ntiles});
+    }
+  }
+  return MLRA_OK;
+}
+}  // namespace
+
+mlra_status mlra_plan_host(const int32_t* tiles_host, int n, int num_ranges, int seg_cost,
+                           int32_t* first_range_host, int32_t* num_parts_host) {
+  if (!first_range_host || !num_parts_host) return MLRA_ERR_INVALID_ARG;
+  std::vector<int32_t> first_r, last_r;
+  const mlra_status st = host_plan(tiles_host, n, num_ranges, seg_cost, &first_r, &last_r, nullptr);
+  if (st != MLRA_OK) return st;
   for (int s = 0; s < n; ++s) {
-    int r0 = 0, np = 0;
-    if (total > 0) seq_parts(prefix.data(), s, total, effective_ranges(num_ranges, total), &r0, &np);
-    first_range_host[s] = r0;
-    num_parts_host[s] = np;
+    first_range_host[s] = first_r[s];
+    num_parts_host[s] = last_r[s] - first_r[s] + 1;
   }
   return MLRA_OK;
 }
 
-mlra_status mlra_plan_segments_host(const int32_t* tiles_host, int n, int num_ranges,
+mlra_status mlra_plan_segments_host(const int32_t* tiles_host, int n, int num_ranges, int seg_cost,
                                     int32_t* range_host, int32_t* seq_host, int32_t* tile0_host,
                                     int32_t* ntiles_host, int max_segments, int* count_host) {
-  if (!tiles_host || !count_host || n < 1 || num_ranges < 1 || max_segments < 0)
-    return MLRA_ERR_INVALID_ARG;
-  std::vector<int32_t> prefix(n + 1, 0);
-  for (int i = 0; i < n; ++i) {
-    if (tiles_host[i] < 0) return MLRA_ERR_INVALID_ARG;
-    const int64_t next = (int64_t)prefix[i] + tiles_host[i];
-    if (next > INT_MAX) return MLRA_ERR_INVALID_ARG;
-    prefix[i + 1] = static_cast<int32_t>(next);
-  }
-  const int64_t total = prefix[n];
-  const int64_t R = effective_ranges(num_ranges, total);
-  int count = 0;
-  for (int r = 0; r < num_ranges; ++r) {
-    SegmentWalker walk(prefix.data(), n, total, R, r);
-    Segment seg;
-    while (walk.next(seg)) {
-      if (count < max_segments) {
-        if (range_host) range_host[count] = r;
-        if (seq_host) seq_host[count] = seg.seq;
-        if (tile0_host) tile0_host[count] = seg.tile0;
-        if (ntiles_host) ntiles_host[count] = seg.ntiles;
-      }
-      ++count;
-    }
+  if (!count_host || max_segments < 0) return MLRA_ERR_INVALID_ARG;
+  std::vector<int32_t> first_r, last_r;
+  std::vector<std::array<int32_t, 4>> segs;
+  const mlra_status st = host_plan(tiles_host, n, num_ranges, seg_cost, &first_r, &last_r, &segs);
+  if (st != MLRA_OK) return st;
+  const int count = static_cast<int>(segs.size());
+  for (int i = 0; i < count && i < max_segments; ++i) {
+    if (range_host) range_host[i] = segs[i][0];
+    if (seq_host) seq_host[i] = segs[i][1];
+    if (tile0_host) tile0_host[i] = segs[i][2];
+    if (ntiles_host) ntiles_host[i] = segs[i][3];
   }
   *count_host = count;
   return MLRA_OK;

@@ -67,8 +67,11 @@ struct DecodeCfg {
   static constexpr int OFF_STAGE = QBYTES;
   static constexpr int OFF_BAR = OFF_STAGE + NS * STAGE;
   static constexpr int NBAR = 2 * NS + 2 + 2 * NSB + NPV + 2;
-  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM = OFF_MISC + 16;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // TMEM address, abort flag, status bits
+  static constexpr int OFF_PLAN = OFF_MISC + 16;       // in-kernel plan (self_plan)
+  static constexpr int PLAN_BYTES = 16 * (kSelfPlanMaxSeqs + 1) +            // segment list
+                                    4 * (3 * kSelfPlanMaxSeqs + 2) + 8;       // lens, prefixes, count
+  static constexpr int SMEM = OFF_PLAN + PLAN_BYTES;
   static constexpr int SMEM_ALLOC = SMEM + 1024;    // slack to align the base to 1024 B
   static_assert(DBLK % 64 == 0 && DBLK <= 512, "branch width must be a multiple of 64, <= 512");
   static_assert(T == 64 || T == 128, "tile of 64 or 128 positions");
@@ -123,19 +126,112 @@ __device__ __forceinline__ int tile_row(const int32_t* page_table, int max_pages
 
 constexpr int kDecodeThreads = 224;
 
-// The segments of one work range, read from the prep kernel's descriptors one ahead of use.
+// In-kernel plan for N <= kSelfPlanMaxSeqs (all threads call it): warp 0 clamps the lengths and
+// scans the real and virtual tile prefixes (mlra_plan.cuh) into shared memory; thread 0 lists the
+// segments of this CTA's range and, in the CTAs of branch 0, records for the combine kernel the
+// ranges holding each sequence's first and last tile; CTA 0 writes the empty sequences' records
+// and outputs.  Returns the segment count.
+__device__ __noinline__ int plan_in_kernel(const DecodeParams& p, int range, int branch,
+                                           uint8_t* plan, uint32_t* flags) {
+  int4* list = reinterpret_cast<int4*>(plan);                       // [kSelfPlanMaxSeqs + 1]
+  int32_t* lens = reinterpret_cast<int32_t*>(list + kSelfPlanMaxSeqs + 1);
+  int32_t* prefix = lens + kSelfPlanMaxSeqs;                          // [N + 1]
+  int32_t* vprefix = prefix + kSelfPlanMaxSeqs + 1;                   // [N + 1]
+  int32_t* count = vprefix + kSelfPlanMaxSeqs + 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, N = p.N;
+  if (warp == 0) {
+    int L[2];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int i = 32 * c + lane;
+      L[c] = i < N ? __ldcg(p.seq_lens + i) : 0;
+    }
+    int carry_t = 0, carry_v = 0;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int i = 32 * c + lane;
+      int Lc = L[c];
+      if (i < N && (Lc < 0 || Lc > p.limit)) {
+        atomicOr(flags, kFlagBadLength);
+        Lc = Lc < 0 ? 0 : p.limit;
+      }
+      int t = i < N ? (Lc + p.tile - 1) / p.tile : 0;
+      int v = t > 0 ? t + p.seg_cost : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int yt = __shfl_up_sync(kFull, t, o), yv = __shfl_up_sync(kFull, v, o);
+        if (lane >= o) {
+          t += yt;
+          v += yv;
+        }
+      }
+      if (i < N) {
+        lens[i] = Lc;
+        prefix[i + 1] = t + carry_t;
+        vprefix[i + 1] = v + carry_v;
+      }
+      carry_t += __shfl_sync(kFull, t, 31);
+      carry_v += __shfl_sync(kFull, v, 31);
+    }
+    if (lane == 0) prefix[0] = vprefix[0] = 0;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    PlanView pv;
+    pv.prefix = prefix;
+    pv.vprefix = vprefix;
+    pv.n = N;
+    pv.total = prefix[N];
+    pv.vtotal = vprefix[N];
+    pv.R = effective_ranges(p.num_ranges, pv.total);
+    pv.cost = p.seg_cost;
+    int n = 0;
+    if (range < pv.R && pv.total > 0) {
+      SegmentWalker walk(prefix, N, range_start(pv, range), range_start(pv, range + 1));
+      Segment seg;
+      while (walk.next(seg)) {
+        list[n++] = make_int4(seg.seq, seg.tile0, seg.ntiles,
+                              lens[seg.seq] | (seg.whole ? (int32_t)0x80000000u : 0));
+        if (branch == 0) {
+          if (seg.tile0 == 0) p.seqs[seg.seq].r0 = range;
+          if (seg.tile0 + seg.ntiles == prefix[seg.seq + 1] - prefix[seg.seq]) p.seqs[seg.seq].r1 = range;
+        }
+      }
+    }
+    *count = n;
+  }
+  if (blockIdx.x == 0 && warp >= 1) {
+    for (int sq = warp - 1; sq < N; sq += kDecodeThreads / 32 - 1) {  // empty: out = 0, lse = -inf
+      if (lens[sq] != 0) continue;
+      if (lane == 0) p.seqs[sq] = SeqInfo{0, -1};
+      float* row = p.out + (int64_t)sq * p.H * p.out_width;
+      for (int i = lane; i < p.H * p.out_width; i += 32) row[i] = 0.f;
+      if (p.lse)
+        for (int i = lane; i < p.H * p.B; i += 32) p.lse[(int64_t)sq * p.H * p.B + i] = -CUDART_INF_F;
+    }
+  }
+  __syncthreads();
+  return *count;
+}
+
+// The segments of one work range, read one ahead of use: from the prep kernel's descriptors in
+// global memory, or from the CTA's own list in shared memory.
 struct SegCursor {
-  const SegDesc* segs;
-  int first, count, i;
+  const int4* segs;
+  bool global;
+  int count, i;
   int4 nxt;
-  __device__ __forceinline__ SegCursor(const SegDesc* s, RangeInfo ri)
-      : segs(s), first(ri.first), count(ri.count), i(0) {
-    if (count > 0) nxt = __ldcg(reinterpret_cast<const int4*>(segs + first));
+  __device__ __forceinline__ int4 load(int k) const {
+    return global ? __ldcg(segs + k) : segs[k];
+  }
+  __device__ __forceinline__ SegCursor(const int4* list, bool in_global, int n)
+      : segs(list), global(in_global), count(n), i(0) {
+    if (count > 0) nxt = load(0);
   }
   __device__ __forceinline__ bool next(Segment& seg, int& len) {
     if (i >= count) return false;
     const int4 d = nxt;
-    if (++i < count) nxt = __ldcg(reinterpret_cast<const int4*>(segs + first + i));
+    if (++i < count) nxt = load(i);
     seg.seq = d.x;
     seg.tile0 = d.y;
     seg.ntiles = d.z;
@@ -171,6 +267,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const uint32_t bar_final_pv = bar_final_s + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  uint32_t* flags = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC + 12);  // this CTA's status bits
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int range = blockIdx.x / p.n_groups;
@@ -194,12 +291,15 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     mbar_init(bar_final_s, 1);
     mbar_init(bar_final_pv, 1);
     *abort_flag = 0;
+    *flags = 0;
     fence_barrier_init();
   }
   if (warp == 5) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
+  if (p.self_plan && warp == 0 && 32 * lane < p.N)
+    prefetch_l2(p.seq_lens + 32 * lane);  // warms L2 and the TLB for the plan below
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_qr);
@@ -211,24 +311,30 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int col0 = branch * DBLK;  // first latent column of this CTA's branch
-  // Everything above overlapped the prep kernel; its segment descriptors are needed now.
+  // Everything above overlapped the previous kernel on the stream (the prep kernel, or the
+  // previous call's combine); the lengths or the prep kernel's plan are read only after it.
   pdl_wait_prerequisites();
-  RangeInfo rinfo;
-  {
+  const int4* seg_list;
+  int seg_count;
+  if (p.self_plan) {
+    seg_count = plan_in_kernel(p, range, branch, smem + C::OFF_PLAN, flags);
+    seg_list = reinterpret_cast<const int4*>(smem + C::OFF_PLAN);
+  } else {
     const int2 r2 = __ldcg(reinterpret_cast<const int2*>(p.ranges + range));
-    rinfo.first = r2.x;
-    rinfo.count = r2.y;
+    seg_list = reinterpret_cast<const int4*>(p.segs + r2.x);
+    seg_count = r2.y;
   }
+  const bool list_global = !p.self_plan;
 
   if (warp == 4) {
     // ------------------------------------------------------------------ TMA producer
-    SegCursor walk(p.segs, rinfo);
+    SegCursor walk(seg_list, list_global, seg_count);
     Segment seg;
     int L = 0;
     int it = 0, nseg = 0;
     bool ok = true;
     while (ok && walk.next(seg, L)) {
-      if (nseg > 0) ok = wait_warp(bar_q_empty, (nseg - 1) & 1, tmo, abort_flag, p.status);
+      if (nseg > 0) ok = wait_warp(bar_q_empty, (nseg - 1) & 1, tmo, abort_flag, flags);
       if (!ok) break;
       if (lane == 0) {
         mbar_arrive_expect_tx(bar_q_full, C::QBYTES);
@@ -246,12 +352,12 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           const int t64 = (seg.tile0 + i) * C::TB + l;
           rows[l] = (t64 * kTile < L)
                         ? tile_row(p.page_table, p.max_pages, p.page_size, p.max_seq_len, p.n_pages,
-                                   p.oob_row, seg.seq, t64, lane == 0 ? p.status : nullptr)
+                                   p.oob_row, seg.seq, t64, lane == 0 ? flags : nullptr)
                         : p.oob_row;
         }
         const int st = it % NS;
         if (it >= NS) {
-          ok = wait_warp(bar_stage_empty + 8 * st, ((it / NS) - 1) & 1, tmo, abort_flag, p.status);
+          ok = wait_warp(bar_stage_empty + 8 * st, ((it / NS) - 1) & 1, tmo, abort_flag, flags);
           if (!ok) break;
         }
         if (lane == 0) {
@@ -272,25 +378,25 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     if (!ok) {
       // Aborting: let the copies already issued land before the CTA can exit.
-      if (nseg > 0) wait_warp(bar_q_full, (nseg - 1) & 1, tmo / 8, abort_flag, p.status, false);
+      if (nseg > 0) wait_warp(bar_q_full, (nseg - 1) & 1, tmo / 8, abort_flag, flags, false);
       for (int k = (it > NS ? it - NS : 0); k < it; ++k)
-        wait_warp(bar_stage_full + 8 * (k % NS), (k / NS) & 1, tmo / 8, abort_flag, p.status, false);
+        wait_warp(bar_stage_full + 8 * (k % NS), (k / NS) & 1, tmo / 8, abort_flag, flags, false);
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------------ score-MMA issuer
     constexpr uint32_t kIdScore = idesc_bf16_f32(64, T, false, false);
-    SegCursor walk(p.segs, rinfo);
+    SegCursor walk(seg_list, list_global, seg_count);
     Segment seg;
     int L = 0;
     int it = 0, nseg = 0;
     bool ok = true;
     while (ok && walk.next(seg, L)) {
-      ok = wait_warp(bar_q_full, nseg & 1, tmo, abort_flag, p.status);
+      ok = wait_warp(bar_q_full, nseg & 1, tmo, abort_flag, flags);
       for (int i = 0; ok && i < seg.ntiles; ++i, ++it) {
-        ok = wait_warp(bar_stage_full + 8 * (it % NS), (it / NS) & 1, tmo, abort_flag, p.status);
+        ok = wait_warp(bar_stage_full + 8 * (it % NS), (it / NS) & 1, tmo, abort_flag, flags);
         if (ok && it >= NSB)  // score buffer free: the output product of tile it-NSB read its P
           ok = wait_warp(bar_pv_done + 8 * ((it - NSB) % NPV), ((it - NSB) / NPV) & 1, tmo,
-                         abort_flag, p.status);
+                         abort_flag, flags);
         if (!ok) break;
         tc_fence_after();
         if (lane == 0) {
@@ -321,18 +427,18 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // Nothing of ours may still run on the tensor core when TMEM is released.
     if (lane == 0) umma_commit(bar_final_s);
     __syncwarp();
-    wait_warp(bar_final_s, 0, tmo, abort_flag, p.status, false);
+    wait_warp(bar_final_s, 0, tmo, abort_flag, flags, false);
   } else if (warp == 6) {
     // ------------------------------------------------------------------ output-MMA issuer
     constexpr uint32_t kIdPV = idesc_bf16_f32(64, C::OCW, false, true);
-    SegCursor walk(p.segs, rinfo);
+    SegCursor walk(seg_list, list_global, seg_count);
     Segment seg;
     int L = 0;
     int j = 0;
     bool ok = true;
     while (ok && walk.next(seg, L)) {
       for (int i = 0; i < seg.ntiles; ++i, ++j) {
-        ok = wait_warp(bar_p_full + 8 * (j % NSB), (j / NSB) & 1, tmo, abort_flag, p.status);
+        ok = wait_warp(bar_p_full + 8 * (j % NSB), (j / NSB) & 1, tmo, abort_flag, flags);
         if (!ok) break;
         tc_fence_after();
         if (lane == 0) {
@@ -360,13 +466,13 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     if (lane == 0) umma_commit(bar_final_pv);
     __syncwarp();
-    wait_warp(bar_final_pv, 0, tmo, abort_flag, p.status, false);
+    wait_warp(bar_final_pv, 0, tmo, abort_flag, flags, false);
   } else {
     // ------------------------------------------------------------------ softmax warps 0-3
     const int q = lane >> 4;                   // which half of the row's columns
     const int h = 16 * warp + (lane & 15);     // head
     const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-    SegCursor walk(p.segs, rinfo);
+    SegCursor walk(seg_list, list_global, seg_count);
     Segment seg;
     int L = 0;
     int it = 0;
@@ -375,7 +481,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       float m_used = -CUDART_INF_F, l_sum = 0.f;
       for (int i = 0; i < seg.ntiles; ++i, ++it) {
         const int t = seg.tile0 + i;
-        ok = wait_warp(bar_s_full + 8 * (it % NSB), (it / NSB) & 1, tmo, abort_flag, p.status);
+        ok = wait_warp(bar_s_full + 8 * (it % NSB), (it / NSB) & 1, tmo, abort_flag, flags);
         if (!ok) break;
         tc_fence_after();
         // this thread's scores: positions 64 l + 32 q + [0, 32) of the tile, l < T / 64
@@ -413,7 +519,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         if (__any_sync(kFull, rescale)) {
           // O holds the output products up to tile it-1: wait for them, then scale O
           ok = wait_warp(bar_pv_done + 8 * ((it - 1) % NPV), ((it - 1) / NPV) & 1, tmo, abort_flag,
-                         p.status);
+                         flags);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll 1
@@ -470,7 +576,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       if (!ok) break;
       // ------------------------------------------------ epilogue of the segment
       ok = wait_warp(bar_pv_done + 8 * ((it - 1) % NPV), ((it - 1) / NPV) & 1, tmo, abort_flag,
-                     p.status);
+                     flags);
       if (!ok) break;
       tc_fence_after();
       const bool to_final = seg.whole && p.write_final;
@@ -530,7 +636,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   __syncthreads();
   tc_fence_after();
   if (warp == 5) tmem_dealloc(tmem, C::TMEM_COLS);
-
+  if (threadIdx.x == 0) p.cta_flags[blockIdx.x] = *flags;  // folded into the status word by K2
 }
 
 }  // namespace mlra

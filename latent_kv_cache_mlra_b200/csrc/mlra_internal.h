@@ -10,27 +10,29 @@ namespace mlra {
 constexpr uint32_t kFlagTimeout = 0x1u;
 constexpr uint32_t kFlagBadPage = 0x2u;
 constexpr uint32_t kFlagBadLength = 0x4u;
+// Up to this many sequences the decode kernel plans its work range itself (no prep kernel).
+constexpr int kSelfPlanMaxSeqs = 64;
 
 // The split plan as the prep kernel writes it for the decode and combine kernels.
 //   RangeInfo[r]  : descriptors segs[first, first + count) of work range r, in tile order
 //   SegDesc       : one (range, sequence) overlap; its partial slot is r + seq
-//   SeqInfo[s]    : ranges r0 .. r0 + nparts - 1 hold sequence s (its partial slots r0 + p + s)
+//   SeqInfo[s]    : ranges r0 .. r1 hold sequence s (its partial slots r + s); empty: r1 = r0 - 1
 struct alignas(8) RangeInfo { int32_t first, count; };
 struct alignas(16) SegDesc {
   int32_t seq, tile0, ntiles;  // tile0: first tile counted inside the sequence
   int32_t len_whole;           // bits 0-30: sequence length; bit 31: the segment is the whole sequence
 };
-struct alignas(8) SeqInfo { int32_t r0, nparts; };
+struct alignas(8) SeqInfo { int32_t r0, r1; };
 
 struct PrepParams {
   const int32_t* seq_lens;    // caller lengths [N]
   int N, limit, tile, num_ranges;
-  int32_t* lens;              // clamped lengths [N]
-  int32_t* prefix;            // tile prefix sums [N + 1]
+  int seg_cost;               // tiles a sequence start costs a CTA (plan balance)
+  int32_t* scratch;           // [5 N + 2] plan arrays when N is too large for shared memory
   RangeInfo* ranges;          // [num_ranges]
   SegDesc* segs;              // [num_ranges + N - 1]
   SeqInfo* seqs;              // [N]
-  uint32_t* status;           // rewritten
+  uint32_t* flags;            // this kernel's status bits (one of the combine kernel's slots)
   float* out;                 // rows of empty sequences are zeroed ...
   float* lse;                 // ... and their lse set to -inf (nullable)
   int H, B, out_width;        // out: [N, H, out_width], lse: [N, H, B]
@@ -38,14 +40,19 @@ struct PrepParams {
 
 // Parameters of the split-KV decode kernel (K1).
 struct DecodeParams {
+  // the plan: from the prep kernel (self_plan == 0) or made by each CTA from seq_lens
   const RangeInfo* ranges;    // [num_ranges] (prep kernel)
   const SegDesc* segs;
+  int self_plan;              // 1: N <= kSelfPlanMaxSeqs, plan in-kernel
+  const int32_t* seq_lens;    // caller lengths [N] (self_plan)
+  int limit, tile, seg_cost;  // length bound, positions per tile, plan balance (self_plan)
+  SeqInfo* seqs;              // [N] written by CTA 0 for the combine kernel (self_plan)
+  uint32_t* cta_flags;        // [grid] status bits of each CTA, written at exit
   const int32_t* page_table;  // [N, max_pages] or nullptr (contiguous)
   float* out;                 // final output, row width out_width, or nullptr
   float* lse;                 // [N, H, B] or nullptr
   float* part_o;              // partial outputs [slots, H, dck]
   float* part_ml;             // partial (m, l) [slots, H, B, 2]
-  uint32_t* status;           // device status word
   int N, H, B;
   int d_blk_out;              // branch width of the caller's output
   int out_width;              // row width of out (d_latent)
@@ -62,7 +69,10 @@ struct DecodeParams {
 };
 
 struct CombineParams {
-  const SeqInfo* seqs;        // [N] (prep kernel)
+  const SeqInfo* seqs;        // [N] (prep kernel, or the decode kernel's CTA 0)
+  const uint32_t* cta_flags;  // [n_flag_slots] status bits of the decode CTAs (and the prep kernel)
+  int n_flag_slots;
+  uint32_t* status;           // the call's status word = OR of the slots
   const float* part_o;
   const float* part_ml;
   float* out;

@@ -1,8 +1,10 @@
 // mlra_kernels.cu -- device kernels of the MLRA decode library and their launchers.
-//   K0 mlra_prep_kernel      lengths -> clamped lengths, tile prefix sums, segment
-//                            descriptors, empty-sequence outputs, status word reset
-//   K1 mlra_decode_kernel    split-KV decode attention (mlra_decode_kernel.cuh)
-//   K2 mlra_combine_kernel   merges the partial softmax states of split sequences
+//   K0 mlra_prep_kernel      (more than kSelfPlanMaxSeqs sequences) clamped lengths, the
+//                            split plan as segment descriptors, empty-sequence outputs
+//   K1 mlra_decode_kernel    split-KV decode attention (mlra_decode_kernel.cuh); plans its own
+//                            work range for up to kSelfPlanMaxSeqs sequences
+//   K2 mlra_combine_kernel   merges the partial softmax states of split sequences and writes
+//                            the call's status word
 //   K3 mlra_repack_kernel    fp32 / odd-width inputs -> padded bf16 copies in the workspace
 //   mlra_resolve_rows_kernel test hook for the cache-row addressing of K1
 #include <cuda_bf16.h>
@@ -17,35 +19,43 @@
 namespace mlra {
 
 // ----------------------------------------------------------------------------- K0
-// One block.  seq_lens outside [0, limit] set kFlagBadLength and are clamped; the status word
-// is rewritten so that it reports this call only.  prefix counts tiles of `tile` positions.
-// Then the split plan for the decode and combine kernels: per work range its segment
-// descriptors (range r's first descriptor sits at r + its first sequence, which keeps the
-// ranges' descriptor blocks disjoint) and per sequence the ranges holding it.  Empty sequences
-// get out = 0, lse = -inf here.  For up to kPrepSmemSeqs sequences the prefix and the lengths
-// are also kept in shared memory, where the per-range searches read them.
-constexpr int kPrepSmemSeqs = 4096;
+// One block, for batches of more than kSelfPlanMaxSeqs sequences (smaller ones are planned by
+// the decode kernel itself).  seq_lens outside [0, limit] set kFlagBadLength (in the kernel's
+// status slot) and are clamped.  Tiles of `tile` positions are counted per
+// sequence and scanned into the real and the virtual prefix of the split plan (mlra_plan.cuh).
+// Then, per work range, its segment descriptors (range r's first descriptor sits at r + its first
+// sequence, which keeps the ranges' descriptor blocks disjoint), per sequence the ranges holding
+// it, and for empty sequences out = 0, lse = -inf.  The plan's arrays live in shared memory for
+// up to kPrepSmemSeqs sequences, else in the workspace (p.scratch).
+constexpr int kPrepSmemSeqs = 2400;  // 5 N + 2 ints <= 48 KB
 
 __global__ void __launch_bounds__(1024) mlra_prep_kernel(const PrepParams p) {
-  __shared__ int32_t warp_tot[32];
-  __shared__ int32_t carry;
+  __shared__ int32_t warp_tot[2][32];
+  __shared__ int32_t carry[2];
   __shared__ uint32_t flags;
-  extern __shared__ int32_t sh_plan[];  // [N + 1] prefix, [N] lens (when N <= kPrepSmemSeqs)
+  extern __shared__ int32_t sh_plan[];
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int N = p.N;
-  const bool in_smem = N <= kPrepSmemSeqs;
-  int32_t* prefix = in_smem ? sh_plan : p.prefix;
-  int32_t* lens = in_smem ? sh_plan + N + 1 : p.lens;
+  int32_t* base = N <= kPrepSmemSeqs ? sh_plan : p.scratch;
+  int32_t* prefix = base;               // [N + 1]
+  int32_t* vprefix = base + (N + 1);    // [N + 1]
+  int32_t* lens = base + 2 * (N + 1);   // [N]
+  int32_t* first_r = lens + N;          // [N] range holding the sequence's first tile
+  int32_t* last_r = first_r + N;        // [N] range holding its last tile
+  // Launched with programmatic stream serialization: the block may be resident before the
+  // previous kernel on the stream (the previous call's combine) has finished.  Nothing is read
+  // or written before that kernel's results are complete and visible.
+  pdl_wait_prerequisites();
   pdl_launch_dependents();  // the decode kernel may start its prologue now
   if (tid == 0) {
-    carry = 0;
+    carry[0] = carry[1] = 0;
     flags = 0;
-    prefix[0] = 0;
+    prefix[0] = vprefix[0] = 0;
   }
   __syncthreads();
-  for (int base = 0; base < N; base += 1024) {
-    const int i = base + tid;
-    int tiles = 0;
+  for (int b0 = 0; b0 < N; b0 += 1024) {
+    const int i = b0 + tid;
+    int x[2] = {0, 0};  // tiles, virtual tiles
     if (i < N) {
       int L = p.seq_lens[i];
       if (L < 0 || L > p.limit) {
@@ -53,39 +63,57 @@ __global__ void __launch_bounds__(1024) mlra_prep_kernel(const PrepParams p) {
         L = L < 0 ? 0 : p.limit;
       }
       lens[i] = L;
-      tiles = (L + p.tile - 1) / p.tile;
+      x[0] = (L + p.tile - 1) / p.tile;
+      x[1] = x[0] > 0 ? x[0] + p.seg_cost : 0;
+      first_r[i] = 0;
+      last_r[i] = -1;
     }
-    int x = tiles;  // inclusive warp scan
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
+    for (int k = 0; k < 2; ++k) {  // inclusive warp scans
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x[k], o);
+        if (lane >= o) x[k] += y;
+      }
+      if (lane == 31) warp_tot[k][wid] = x[k];
     }
-    if (lane == 31) warp_tot[wid] = x;
     __syncthreads();
-    if (wid == 0) {
-      int w = warp_tot[lane];
+    if (wid < 2) {
+      int w = warp_tot[wid][lane];
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, w, o);
         if (lane >= o) w += y;
       }
-      warp_tot[lane] = w;  // inclusive over warps
+      warp_tot[wid][lane] = w;  // inclusive over warps
     }
     __syncthreads();
-    const int incl = x + (wid > 0 ? warp_tot[wid - 1] : 0) + carry;
-    if (i < N) prefix[i + 1] = incl;
+    const int incl0 = x[0] + (wid > 0 ? warp_tot[0][wid - 1] : 0) + carry[0];
+    const int incl1 = x[1] + (wid > 0 ? warp_tot[1][wid - 1] : 0) + carry[1];
+    if (i < N) {
+      prefix[i + 1] = incl0;
+      vprefix[i + 1] = incl1;
+    }
     __syncthreads();
-    if (tid == 1023) carry = incl;
+    if (tid == 1023) {
+      carry[0] = incl0;
+      carry[1] = incl1;
+    }
     __syncthreads();
   }
-  // prefix and lens written above are visible to the whole block after the last __syncthreads
-  const int64_t total = prefix[N];
-  const int64_t R = effective_ranges(p.num_ranges, total);
+  // the arrays written above are visible to the whole block after the last __syncthreads
+  PlanView pv;
+  pv.prefix = prefix;
+  pv.vprefix = vprefix;
+  pv.n = N;
+  pv.total = prefix[N];
+  pv.vtotal = vprefix[N];
+  pv.R = effective_ranges(p.num_ranges, pv.total);
+  pv.cost = p.seg_cost;
   for (int r = tid; r < p.num_ranges; r += blockDim.x) {
     RangeInfo ri{0, 0};
-    if (r < R && total > 0) {
-      SegmentWalker walk(prefix, N, total, R, r);
+    if (r < pv.R && pv.total > 0) {
+      SegmentWalker walk(prefix, N, range_start(pv, r), range_start(pv, r + 1));
       Segment seg;
       ri.first = -1;
       while (walk.next(seg)) {
@@ -97,13 +125,17 @@ __global__ void __launch_bounds__(1024) mlra_prep_kernel(const PrepParams p) {
         d.len_whole = lens[seg.seq] | (seg.whole ? (int32_t)0x80000000u : 0);
         p.segs[ri.first + ri.count] = d;
         ++ri.count;
+        if (seg.tile0 == 0) first_r[seg.seq] = r;
+        if (seg.tile0 + seg.ntiles == prefix[seg.seq + 1] - prefix[seg.seq]) last_r[seg.seq] = r;
       }
     }
     p.ranges[r] = ri;
   }
+  __syncthreads();
   for (int sq = tid; sq < N; sq += blockDim.x) {
-    SeqInfo si{0, 0};
-    if (total > 0) seq_parts(prefix, sq, total, R, &si.r0, &si.nparts);
+    SeqInfo si;
+    si.r0 = first_r[sq];
+    si.r1 = last_r[sq];  // r0 - 1 for an empty sequence
     p.seqs[sq] = si;
   }
   for (int sq = wid; sq < N; sq += 32) {  // empty sequences (a warp each): out = 0, lse = -inf
@@ -113,13 +145,21 @@ __global__ void __launch_bounds__(1024) mlra_prep_kernel(const PrepParams p) {
     if (p.lse)
       for (int i = lane; i < p.H * p.B; i += 32) p.lse[(int64_t)sq * p.H * p.B + i] = -CUDART_INF_F;
   }
-  if (tid == 0) *p.status = flags;
+  if (tid == 0) *p.flags = flags;  // folded into the status word by the combine kernel
 }
 
 cudaError_t launch_prep(const PrepParams& p, cudaStream_t st) {
-  const size_t sh = p.N <= kPrepSmemSeqs ? (2 * (size_t)p.N + 1) * sizeof(int32_t) : 0;
-  mlra_prep_kernel<<<1, 1024, sh, st>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(1024);
+  cfg.dynamicSmemBytes = p.N <= kPrepSmemSeqs ? (5 * (size_t)p.N + 2) * sizeof(int32_t) : 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // hide the launch gap
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, mlra_prep_kernel, p);
 }
 
 // ----------------------------------------------------------------------------- K1
@@ -200,9 +240,19 @@ __global__ void __launch_bounds__(kCombineWarps * 32) mlra_combine_kernel(const 
   // padded column of this lane: branch mode over [0, dck), summed mode over [0, dblk_k)
   const int k = blockIdx.z * 128 + 4 * lane;
   const bool live = live_h && k < (p.summed ? p.dblk_k : p.dck);
+  // The next call's prep kernel may be scheduled now: it waits for this grid before it reads
+  // or writes anything.
+  pdl_launch_dependents();
   pdl_wait_prerequisites();  // the decode kernel's partials must be complete and visible
-  const int2 si = __ldcg(reinterpret_cast<const int2*>(p.seqs + s));  // (r0, nparts)
-  const int np = si.y;
+  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x < 32) {
+    // the call's status word: the bits every decode CTA (and the prep kernel) raised
+    uint32_t f = 0;
+    for (int i = threadIdx.x; i < p.n_flag_slots; i += 32) f |= __ldcg(p.cta_flags + i);
+    f = __reduce_or_sync(0xffffffffu, f);
+    if (threadIdx.x == 0) *p.status = f;
+  }
+  const int2 si = __ldcg(reinterpret_cast<const int2*>(p.seqs + s));  // (r0, r1)
+  const int np = si.y - si.x + 1;
   if (np == 0 || (np == 1 && p.final_written)) return;  // written by K0 / by the decode kernel
   const int width = p.summed ? p.d_blk_out : p.B * p.d_blk_out;
   float* out_row = p.out + ((int64_t)s * p.H + h) * width;

@@ -47,7 +47,7 @@ class PlanInfo(ctypes.Structure):
     _fields_ = [("repack", ctypes.c_int), ("launches", ctypes.c_int), ("num_ranges", ctypes.c_int),
                 ("ctas", ctypes.c_int), ("kernel_branch_width", ctypes.c_int),
                 ("branches_per_cta", ctypes.c_int), ("tile", ctypes.c_int),
-                ("partial_slots", ctypes.c_longlong),
+                ("partial_slots", ctypes.c_longlong), ("segment_cost_tiles", ctypes.c_int),
                 ("workspace_bytes", ctypes.c_size_t)]
 
 
@@ -78,9 +78,10 @@ def lib() -> ctypes.CDLL:
         L.mlra_decode_static_scratch.argtypes = L.mlra_decode.argtypes[:11] + [vp]
         L.mlra_read_status.argtypes = [vp, vp, u32p]
         L.mlra_debug_resolve_rows.argtypes = [vp, vp, ctypes.POINTER(Dims), vp, ctypes.c_int, vp]
-        L.mlra_plan_host.argtypes = [i32p, ctypes.c_int, ctypes.c_int, i32p, i32p]
-        L.mlra_plan_segments_host.argtypes = [i32p, ctypes.c_int, ctypes.c_int, i32p, i32p, i32p,
-                                              i32p, ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
+        L.mlra_plan_host.argtypes = [i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, i32p, i32p]
+        L.mlra_plan_segments_host.argtypes = [i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, i32p,
+                                              i32p, i32p, i32p, ctypes.c_int,
+                                              ctypes.POINTER(ctypes.c_int)]
         L.mlra_status_string.argtypes = [ctypes.c_int]
         L.mlra_status_string.restype = ctypes.c_char_p
         L.mlra_version.argtypes = []
@@ -273,26 +274,26 @@ def resolve_rows(seq_lens, page_table, dims: Dims, row_pitch: int, stream=None) 
     return rows
 
 
-def plan_host(tiles, num_ranges: int):
+def plan_host(tiles, num_ranges: int, seg_cost: int = 0):
     """Host replica of the split plan: (first range, number of parts) per sequence."""
     n = len(tiles)
     arr = (ctypes.c_int32 * n)(*[int(t) for t in tiles])
     first, parts = (ctypes.c_int32 * n)(), (ctypes.c_int32 * n)()
-    _check(lib().mlra_plan_host(arr, n, num_ranges, first, parts), "mlra_plan_host")
+    _check(lib().mlra_plan_host(arr, n, num_ranges, seg_cost, first, parts), "mlra_plan_host")
     return list(first), list(parts)
 
 
-def plan_segments_host(tiles, num_ranges: int):
+def plan_segments_host(tiles, num_ranges: int, seg_cost: int = 0):
     """Host replica of the kernel's per-CTA segment walk: list of (range, seq, tile0, ntiles)."""
     n = len(tiles)
     arr = (ctypes.c_int32 * n)(*[int(t) for t in tiles])
     count = ctypes.c_int(0)
-    _check(lib().mlra_plan_segments_host(arr, n, num_ranges, None, None, None, None, 0,
+    _check(lib().mlra_plan_segments_host(arr, n, num_ranges, seg_cost, None, None, None, None, 0,
                                          ctypes.byref(count)), "mlra_plan_segments_host")
     m = count.value
     bufs = [(ctypes.c_int32 * max(m, 1))() for _ in range(4)]
-    _check(lib().mlra_plan_segments_host(arr, n, num_ranges, *bufs, m, ctypes.byref(count)),
-           "mlra_plan_segments_host")
+    _check(lib().mlra_plan_segments_host(arr, n, num_ranges, seg_cost, *bufs, m,
+                                         ctypes.byref(count)), "mlra_plan_segments_host")
     return [tuple(b[i] for b in bufs) for i in range(m)]
 
 

@@ -245,6 +245,34 @@ def test_status_flags():
         assert torch.isfinite(cdec.out).all()
 
 
+@pytest.mark.parametrize("N,R", [(65, 0), (80, 7), (96, 300)])
+def test_more_sequences_than_the_in_kernel_plan(N, R):
+    """Batches above the in-kernel plan's limit take the prep-kernel path (one more launch);
+    results, empty sequences and the status word behave the same."""
+    rnd = np.random.default_rng(N)
+    lens = [int(x) for x in rnd.choice([0, 1, 17, 64, 128, 129, 300, 700], size=N)]
+    inp = small_inputs(lens=lens, heads=8, seed=N)
+    q, qr, c, kr, dlens, pt = to_dev(inp)
+    w = inp.workload
+    plan = mlra.query_plan(mlra.dims_for(q, qr, c, kr, dlens, pt, w.num_branches,
+                                         max_seq_len=inp.max_seq_len, num_ranges=R))
+    assert plan.launches == 3
+    out, lse = run_gpu(inp, num_ranges=R)
+    ref, ref_lse = run_oracle(inp)
+    assert_close(out, ref, f"N={N} R={R}")
+    assert_lse_close(lse, ref_lse, f"N={N} R={R}")
+    empty = [i for i, L in enumerate(lens) if L == 0]
+    assert (out[empty] == 0).all() and torch.isinf(lse[empty]).all()
+    bad = dlens.clone()
+    bad[3] = -5
+    dec = mlra.Decoder(q, qr, c, kr, dlens, pt, num_branches=w.num_branches, softmax_scale=w.sigma,
+                       max_seq_len=inp.max_seq_len, num_ranges=R)
+    dec(args=(q, qr, c, kr, bad, pt))
+    assert dec.status() == (mlra.MLRA_ERR_BAD_LENGTH, mlra.FLAG_BAD_LENGTH)
+    dec()
+    assert dec.status() == (mlra.MLRA_OK, 0)
+
+
 def test_repeat_calls_are_deterministic():
     inp = small_inputs()
     dev = to_dev(inp)

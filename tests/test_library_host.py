@@ -43,11 +43,12 @@ def dims(**kw):
 
 
 def test_workspace_size_layout():
-    # status 256 + lens + prefix + plan (a range record per range, a segment descriptor per
-    # slot, a sequence record per sequence) + (R + N - 1) slots of (m, l) and partial outputs
+    # status 256 + plan scratch (5 N + 2 ints) + plan (a range record per range, a segment
+    # descriptor per slot, a sequence record per sequence) + a status slot per CTA and one for
+    # the prep kernel + (R + N - 1) slots of (m, l) and partial outputs
     n = mlra.workspace_size(dims())
     slots, H, B, dck, R, N = 74 + 8 - 1, 64, 4, 512, 74, 8
-    plan = 8 * R + 16 * slots + 8 * N
+    plan = 4 * (5 * N + 2) + 8 * R + 16 * slots + 8 * N + 4 * (R * B + 1)
     expect_min = 256 + plan + slots * H * B * 2 * 4 + slots * H * dck * 4
     assert expect_min <= n <= expect_min + 8 * 256 + 64
     # fp32 input adds padded bf16 copies of queries and cache
@@ -117,6 +118,24 @@ def ranges_by_definition(tiles, R):
     return out
 
 
+def cost_boundaries(tiles, R, cost):
+    """Range starts of the cost-balanced plan, written from its definition: every non-empty
+    sequence is `cost` virtual tiles followed by its real tiles; range r starts at virtual
+    position floor(r V / R), mapped back to the real tile it falls on (a position among a
+    sequence's leading cost tiles maps to the sequence's first tile)."""
+    T = sum(tiles)
+    R = min(R, max(T, 1))
+    virtual = []  # real tile (or first tile of the sequence) of every virtual position
+    g = 0
+    for t in tiles:
+        if t == 0:
+            continue
+        virtual += [g] * cost + list(range(g, g + t))
+        g += t
+    V = len(virtual)
+    return [virtual[r * V // R] if r * V // R < V else T for r in range(R)] + [T]
+
+
 @pytest.mark.parametrize("seed", range(12))
 def test_plan_host_matches_definition(seed):
     rnd = random.Random(seed)
@@ -175,8 +194,63 @@ def test_segment_walk_covers_every_tile_once(seed):
             assert len(rs) == parts[s] and (not rs or rs[0] == first[s])
 
 
+@pytest.mark.parametrize("seed", range(16))
+def test_cost_balanced_plan_matches_definition(seed):
+    """The plan the kernels use (a cost of c tiles per sequence start) against its definition
+    written out position by position; every tile is covered once, the ranges of a sequence are
+    consecutive and non-empty, partial slots are unique."""
+    rnd = random.Random(500 + seed)
+    n = rnd.randint(1, 40)
+    tiles = [rnd.choice([0, 1, 2, 3, 5, 9, 40, 256, 300]) for _ in range(n)]
+    if sum(tiles) == 0:
+        tiles[-1] = 7
+    R = rnd.choice([1, 2, 3, 7, 37, 74, 148, 400])
+    cost = rnd.choice([0, 1, 3, 8])
+    bounds = cost_boundaries(tiles, R, cost)
+    segs = mlra.plan_segments_host(tiles, R, cost)
+    prefix = [0]
+    for t in tiles:
+        prefix.append(prefix[-1] + t)
+    # every segment is the overlap of its range with its sequence
+    expect = []
+    for r in range(len(bounds) - 1):
+        a, b = bounds[r], bounds[r + 1]
+        for s in range(n):
+            lo, hi = max(a, prefix[s]), min(b, prefix[s + 1])
+            if lo < hi:
+                expect.append((r, s, lo - prefix[s], hi - lo))
+    assert segs == expect
+    covered = sorted((s, t) for _, s, t0, nt in segs for t in range(t0, t0 + nt))
+    assert covered == [(s, t) for s in range(n) for t in range(tiles[s])]
+    first, parts = mlra.plan_host(tiles, R, cost)
+    for s in range(n):
+        rs = [r for r, ss, *_ in segs if ss == s]
+        assert len(rs) == parts[s] and rs == list(range(first[s], first[s] + parts[s])) if rs else parts[s] == 0
+    slots = [r + s for r, s, *_ in segs]
+    assert len(slots) == len(set(slots)) and max(slots) < R + n - 1
+    if cost == 0:
+        assert bounds == [r * sum(tiles) // min(R, sum(tiles)) for r in range(min(R, sum(tiles)))] + [sum(tiles)]
+
+
+def test_cost_balanced_plan_moves_work_off_sequence_starts():
+    # 8 sequences of 256 tiles over 37 ranges: a range in which a sequence starts gets fewer tiles
+    tiles, R, cost = [256] * 8, 37, 3
+    segs = mlra.plan_segments_host(tiles, R, cost)
+    per_range = {}
+    for r, s, t0, nt in segs:
+        per_range.setdefault(r, []).append((s, t0, nt))
+    sizes = {r: sum(nt for _, _, nt in v) for r, v in per_range.items()}
+    starts = {r: sum(1 for i, (s, t0, nt) in enumerate(v) if i > 0 and t0 == 0) for r, v in per_range.items()}
+    plain = [r for r in sizes if starts[r] == 0 and r > 0]
+    split = [r for r in sizes if starts[r] == 1]
+    assert split and plain
+    assert max(sizes[r] for r in split) <= min(sizes[r] for r in plain) - cost + 1
+
+
 def test_plan_host_rejects():
     with pytest.raises(mlra.MlraError):
         mlra.plan_host([1, -1], 4)
     with pytest.raises(mlra.MlraError):
         mlra.plan_host([1, 2], 0)
+    with pytest.raises(mlra.MlraError):
+        mlra.plan_host([1, 2], 4, -1)
