@@ -163,6 +163,19 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 store map over [dims[2]][dims[1]][dims[0]] (row pitches in elements), boxes of 32 x 16 x 1,
+// 128-byte swizzle: the attention kernel's epilogue stores through it.
+bool make_store_map(CUtensorMap* m, void* base, const uint64_t* dims, const uint64_t* pitches) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[3] = {dims[0], dims[1], dims[2]};
+  cuuint64_t gstride[2] = {pitches[0] * 4, pitches[1] * 4};
+  cuuint32_t box[3] = {32, 16, 1}, estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, gdim, gstride, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 // Scratch of mlra_decode_static_scratch.  In host code the name stands for the array only as a
@@ -319,6 +332,22 @@ mlra_status mlra_decode_profiled(const void* q_lat, const void* q_rope, const vo
   const bool summed = dims->out_mode == MLRA_OUT_SUMMED;
   const int out_width = summed ? dblk : dims->d_latent;  // floats per (sequence, head) row of out
   const int grid = pl.R * pl.n_groups;
+  // store maps of the attention kernel's epilogue: partial outputs always, final outputs when
+  // every branch block is whole 32-column boxes (else it stores them directly)
+  CUtensorMap tpart, tout;
+  const bool tma_out = !summed && dblk % 32 == 0 && out_width % 4 == 0;
+  {
+    const uint64_t dpart[3] = {(uint64_t)pl.dck, (uint64_t)H, (uint64_t)pl.slots};
+    const uint64_t ppart[2] = {(uint64_t)pl.dck, (uint64_t)pl.dck * H};
+    if (!make_store_map(&tpart, part_o, dpart, ppart)) return MLRA_ERR_CUDA;
+    if (tma_out) {
+      const uint64_t dout[3] = {(uint64_t)out_width, (uint64_t)H, (uint64_t)N};
+      const uint64_t pout[2] = {(uint64_t)out_width, (uint64_t)out_width * H};
+      if (!make_store_map(&tout, out, dout, pout)) return MLRA_ERR_CUDA;
+    } else {
+      tout = tpart;  // unused
+    }
+  }
   uint32_t* cta_flags = reinterpret_cast<uint32_t*>(ws + pl.off_flags);  // [grid] + prep's slot
   if (!pl.self_plan) {
     PrepParams pp;
@@ -347,10 +376,11 @@ mlra_status mlra_decode_profiled(const void* q_lat, const void* q_rope, const vo
   p.scale_log2 = scales->softmax_scale * 1.4426950408889634f;
   p.gamma = scales->branch_scale;
   p.write_final = summed ? 0 : 1;
+  p.tma_out = tma_out ? 1 : 0;
   p.timeout_ns = kTimeoutNs;
   if (k1_begin && cudaEventRecord(reinterpret_cast<cudaEvent_t>(k1_begin), s) != cudaSuccess)
     return MLRA_ERR_CUDA;
-  if (launch_decode(pl.variant, tq, tqr, tc, tkr, p, grid, s) != cudaSuccess)
+  if (launch_decode(pl.variant, tq, tqr, tc, tkr, tout, tpart, p, grid, s) != cudaSuccess)
     return MLRA_ERR_CUDA;
   if (k1_end && cudaEventRecord(reinterpret_cast<cudaEvent_t>(k1_end), s) != cudaSuccess)
     return MLRA_ERR_CUDA;

@@ -69,9 +69,12 @@ struct DecodeCfg {
   static constexpr int NBAR = 2 * NS + 2 + 2 * NSB + NPV + 2;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // TMEM address, abort flag, status bits
   static constexpr int OFF_PLAN = OFF_MISC + 16;       // in-kernel plan (self_plan)
-  static constexpr int PLAN_BYTES = 16 * (kSelfPlanMaxSeqs + 1) +            // segment list
-                                    4 * (3 * kSelfPlanMaxSeqs + 2) + 8;       // lens, prefixes, count
-  static constexpr int SMEM = OFF_PLAN + PLAN_BYTES;
+  static constexpr int PLAN_BYTES = 16 * kSelfPlanMaxSeqs +     // segment list
+                                    4 * kSelfPlanMaxSeqs + 16;    // lengths, count
+  // epilogue staging: one [16 rows x 32 fp32] box per softmax warp, 128-byte swizzled
+  static constexpr int OFF_STG = (OFF_PLAN + PLAN_BYTES + 1023) / 1024 * 1024;
+  static constexpr int STG_BYTES = 16 * 128;
+  static constexpr int SMEM = OFF_STG + 4 * STG_BYTES;
   static constexpr int SMEM_ALLOC = SMEM + 1024;    // slack to align the base to 1024 B
   static_assert(DBLK % 64 == 0 && DBLK <= 512, "branch width must be a multiple of 64, <= 512");
   static_assert(T == 64 || T == 128, "tile of 64 or 128 positions");
@@ -126,21 +129,21 @@ __device__ __forceinline__ int tile_row(const int32_t* page_table, int max_pages
 
 constexpr int kDecodeThreads = 224;
 
-// In-kernel plan for N <= kSelfPlanMaxSeqs (all threads call it): warp 0 clamps the lengths and
-// scans the real and virtual tile prefixes (mlra_plan.cuh) into shared memory; thread 0 lists the
-// segments of this CTA's range and, in the CTAs of branch 0, records for the combine kernel the
-// ranges holding each sequence's first and last tile; CTA 0 writes the empty sequences' records
-// and outputs.  Returns the segment count.
+// In-kernel plan for N <= kSelfPlanMaxSeqs = 64 (all threads call it).  Warp 0 holds sequences
+// lane and lane + 32: it clamps their lengths, scans the real and virtual tile prefixes
+// (mlra_plan.cuh) across the warp, finds the sequence holding each of the range's two virtual
+// boundaries with one ballot, and lets every sequence that overlaps the range write its own
+// segment at its rank in the warp.  The CTAs of branch 0 also record, for the combine kernel, the
+// ranges holding each sequence's first and last tile; CTA 0 writes the records and outputs of
+// empty sequences.  Returns the segment count.
 __device__ __noinline__ int plan_in_kernel(const DecodeParams& p, int range, int branch,
                                            uint8_t* plan, uint32_t* flags) {
-  int4* list = reinterpret_cast<int4*>(plan);                       // [kSelfPlanMaxSeqs + 1]
-  int32_t* lens = reinterpret_cast<int32_t*>(list + kSelfPlanMaxSeqs + 1);
-  int32_t* prefix = lens + kSelfPlanMaxSeqs;                          // [N + 1]
-  int32_t* vprefix = prefix + kSelfPlanMaxSeqs + 1;                   // [N + 1]
-  int32_t* count = vprefix + kSelfPlanMaxSeqs + 1;
+  int4* list = reinterpret_cast<int4*>(plan);                       // [kSelfPlanMaxSeqs]
+  int32_t* lens = reinterpret_cast<int32_t*>(list + kSelfPlanMaxSeqs);
+  int32_t* count = lens + kSelfPlanMaxSeqs;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, N = p.N;
   if (warp == 0) {
-    int L[2];
+    int L[2], t[2], lo[2], hi[2], vlo[2], vhi[2];
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const int i = 32 * c + lane;
@@ -150,67 +153,91 @@ __device__ __noinline__ int plan_in_kernel(const DecodeParams& p, int range, int
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const int i = 32 * c + lane;
-      int Lc = L[c];
-      if (i < N && (Lc < 0 || Lc > p.limit)) {
+      if (i < N && (L[c] < 0 || L[c] > p.limit)) {
         atomicOr(flags, kFlagBadLength);
-        Lc = Lc < 0 ? 0 : p.limit;
+        L[c] = L[c] < 0 ? 0 : p.limit;
       }
-      int t = i < N ? (Lc + p.tile - 1) / p.tile : 0;
-      int v = t > 0 ? t + p.seg_cost : 0;
+      t[c] = i < N ? (L[c] + p.tile - 1) / p.tile : 0;
+      int x = t[c], v = t[c] > 0 ? t[c] + p.seg_cost : 0;
+      const int vt = v;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int yt = __shfl_up_sync(kFull, t, o), yv = __shfl_up_sync(kFull, v, o);
+      for (int o = 1; o < 32; o <<= 1) {  // inclusive scans
+        const int yx = __shfl_up_sync(kFull, x, o), yv = __shfl_up_sync(kFull, v, o);
         if (lane >= o) {
-          t += yt;
+          x += yx;
           v += yv;
         }
       }
-      if (i < N) {
-        lens[i] = Lc;
-        prefix[i + 1] = t + carry_t;
-        vprefix[i + 1] = v + carry_v;
-      }
-      carry_t += __shfl_sync(kFull, t, 31);
+      hi[c] = x + carry_t;
+      lo[c] = hi[c] - t[c];
+      vhi[c] = v + carry_v;
+      vlo[c] = vhi[c] - vt;
+      carry_t += __shfl_sync(kFull, x, 31);
       carry_v += __shfl_sync(kFull, v, 31);
+      if (i < N) lens[i] = L[c];
     }
-    if (lane == 0) prefix[0] = vprefix[0] = 0;
+    const int64_t total = carry_t, vtotal = carry_v;
+    const int64_t R = effective_ranges(p.num_ranges, total);
+    int n = 0;
+    if (range < R && total > 0) {
+      // real tile of a virtual position: the sequence whose virtual interval holds it
+      auto tile_of = [&](int64_t v) -> int64_t {
+        int64_t g = 0;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const bool own = t[c] > 0 && vlo[c] <= v && v < vhi[c];
+          const uint32_t m = __ballot_sync(kFull, own);
+          if (m) {
+            const int src = __ffs(m) - 1;
+            const int64_t o = v - vlo[c] - p.seg_cost;
+            const int64_t mine = lo[c] + (o > 0 ? o : 0);
+            g = __shfl_sync(kFull, mine, src);
+          }
+        }
+        return g;
+      };
+      const int64_t g0 = tile_of((range * vtotal) / R);
+      const int64_t g1 = range + 1 < R ? tile_of(((range + 1) * vtotal) / R) : total;
+      int base = 0;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int i = 32 * c + lane;
+        const bool ov = t[c] > 0 && lo[c] < g1 && hi[c] > g0;
+        const uint32_t m = __ballot_sync(kFull, ov);
+        if (ov) {
+          const int64_t a = g0 > lo[c] ? g0 : lo[c], e = g1 < hi[c] ? g1 : hi[c];
+          const bool whole = a == lo[c] && e == hi[c];
+          list[base + __popc(m & ((1u << lane) - 1u))] =
+              make_int4(i, static_cast<int>(a - lo[c]), static_cast<int>(e - a),
+                        L[c] | (whole ? (int32_t)0x80000000u : 0));
+          if (branch == 0) {
+            if (a == lo[c]) p.seqs[i].r0 = range;  // the sequence's first tile is in this range
+            if (e == hi[c]) p.seqs[i].r1 = range;  // ... its last tile
+          }
+        }
+        base += __popc(m);
+      }
+      n = base;
+    }
+    if (blockIdx.x == 0) {
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int i = 32 * c + lane;
+        if (i < N && t[c] == 0) p.seqs[i] = SeqInfo{0, -1};
+      }
+    }
+    if (lane == 0) *count = n;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    PlanView pv;
-    pv.prefix = prefix;
-    pv.vprefix = vprefix;
-    pv.n = N;
-    pv.total = prefix[N];
-    pv.vtotal = vprefix[N];
-    pv.R = effective_ranges(p.num_ranges, pv.total);
-    pv.cost = p.seg_cost;
-    int n = 0;
-    if (range < pv.R && pv.total > 0) {
-      SegmentWalker walk(prefix, N, range_start(pv, range), range_start(pv, range + 1));
-      Segment seg;
-      while (walk.next(seg)) {
-        list[n++] = make_int4(seg.seq, seg.tile0, seg.ntiles,
-                              lens[seg.seq] | (seg.whole ? (int32_t)0x80000000u : 0));
-        if (branch == 0) {
-          if (seg.tile0 == 0) p.seqs[seg.seq].r0 = range;
-          if (seg.tile0 + seg.ntiles == prefix[seg.seq + 1] - prefix[seg.seq]) p.seqs[seg.seq].r1 = range;
-        }
-      }
-    }
-    *count = n;
-  }
   if (blockIdx.x == 0 && warp >= 1) {
     for (int sq = warp - 1; sq < N; sq += kDecodeThreads / 32 - 1) {  // empty: out = 0, lse = -inf
       if (lens[sq] != 0) continue;
-      if (lane == 0) p.seqs[sq] = SeqInfo{0, -1};
       float* row = p.out + (int64_t)sq * p.H * p.out_width;
       for (int i = lane; i < p.H * p.out_width; i += 32) row[i] = 0.f;
       if (p.lse)
         for (int i = lane; i < p.H * p.B; i += 32) p.lse[(int64_t)sq * p.H * p.B + i] = -CUDART_INF_F;
     }
   }
-  __syncthreads();
   return *count;
 }
 
@@ -245,6 +272,7 @@ template <int DBLK, int T, int NS>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
 mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
                    const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_kr,
+                   const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_part,
                    const __grid_constant__ DecodeParams p) {
   using C = DecodeCfg<DBLK, T, NS>;
   constexpr int NSB = C::NSB, NPV = C::NPV;
@@ -305,6 +333,8 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tma_prefetch_desc(&tm_qr);
     tma_prefetch_desc(&tm_c);
     tma_prefetch_desc(&tm_kr);
+    tma_prefetch_desc(&tm_part);
+    if (p.tma_out) tma_prefetch_desc(&tm_out);
   }
   tc_fence_before();
   __syncthreads();
@@ -472,6 +502,9 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int q = lane >> 4;                   // which half of the row's columns
     const int h = 16 * warp + (lane & 15);     // head
     const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    uint8_t* stg = smem + C::OFF_STG + warp * C::STG_BYTES;  // this warp's store staging box
+    const uint32_t stg_u = smem_u32(stg);
+    bool stg_pending = false;  // a bulk store may still be reading stg
     SegCursor walk(seg_list, list_global, seg_count);
     Segment seg;
     int L = 0;
@@ -581,39 +614,78 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       tc_fence_after();
       const bool to_final = seg.whole && p.write_final;
       const bool live = h < p.H;
-      float* dst;
       float scale;
       int ncols_out;
       if (to_final) {
-        dst = p.out + ((int64_t)seg.seq * p.H + h) * p.out_width + (int64_t)branch * p.d_blk_out;
         scale = p.gamma / l_sum;
         ncols_out = p.d_blk_out;
       } else {
-        const int64_t slot = (int64_t)range + seg.seq;
-        dst = p.part_o + (slot * p.H + h) * p.dck + (int64_t)branch * DBLK;
         scale = 1.f;
         ncols_out = DBLK;
       }
+      if (16 * warp >= p.H) {
+        // no head of this warp exists: nothing to store
+      } else if (!to_final || p.tma_out) {
+        // Through shared memory and the TMA: each [16 heads x 32 columns] box is staged in the
+        // 128-byte swizzled layout and stored by one bulk copy (rows past H are clipped by the
+        // tensor map).  Partials go to slot range + seq of part_o, finals to out.
+        const CUtensorMap* map = to_final ? &tm_out : &tm_part;
+        const int x0 = to_final ? branch * p.d_blk_out : branch * DBLK;
+        const int z = to_final ? seg.seq : range + seg.seq;
+        const int row = lane & 15;
 #pragma unroll 1
-      for (int ch = 0; ch < C::OCH; ++ch) {
+        for (int ch = 0; ch < C::OCH; ++ch) {
 #pragma unroll 1
-        for (int c0 = 0; c0 < C::OCW; c0 += 64) {
-          uint32_t r[32];
-          tmem_ld16x2_32(tmem + ((uint32_t)(32 * warp + 16 * (ch & 1)) << 16) + (ch >> 1) * C::OCW + c0, r);
-          tmem_wait_ld();
-          if (live) {
-            const int cbase = ch * C::OCW + c0 + 32 * q;
-            if (cbase + 32 <= ncols_out && ((reinterpret_cast<uintptr_t>(dst + cbase)) & 15) == 0) {
+          for (int c0 = 0; c0 < C::OCW; c0 += 64) {
+            uint32_t r[32];
+            tmem_ld16x2_32(tmem + ((uint32_t)(32 * warp + 16 * (ch & 1)) << 16) + (ch >> 1) * C::OCW + c0, r);
+            tmem_wait_ld();
 #pragma unroll
-              for (int k = 0; k < 32; k += 4) {
-                float4 o4 = make_float4(__uint_as_float(r[k]) * scale, __uint_as_float(r[k + 1]) * scale,
-                                        __uint_as_float(r[k + 2]) * scale, __uint_as_float(r[k + 3]) * scale);
-                *reinterpret_cast<float4*>(dst + cbase + k) = o4;
+            for (int half = 0; half < 2; ++half) {
+              const int col = ch * C::OCW + c0 + 32 * half;  // column inside the branch block
+              if (col >= ncols_out) continue;
+              if (lane == 0 && stg_pending) bulk_wait_read_all();
+              __syncwarp();
+              if (q == half) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                  *reinterpret_cast<float4*>(stg + row * 128 + ((k ^ (row & 7)) << 4)) =
+                      make_float4(__uint_as_float(r[4 * k]) * scale, __uint_as_float(r[4 * k + 1]) * scale,
+                                  __uint_as_float(r[4 * k + 2]) * scale, __uint_as_float(r[4 * k + 3]) * scale);
               }
-            } else {
+              fence_proxy_async_smem();  // the staged box is read by the bulk copy (async proxy)
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_3d(map, stg_u, x0 + col, 16 * warp, z);
+                bulk_commit();
+              }
+              stg_pending = true;
+            }
+          }
+        }
+      } else {
+        float* dst = p.out + ((int64_t)seg.seq * p.H + h) * p.out_width + (int64_t)branch * p.d_blk_out;
+#pragma unroll 1
+        for (int ch = 0; ch < C::OCH; ++ch) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < C::OCW; c0 += 64) {
+            uint32_t r[32];
+            tmem_ld16x2_32(tmem + ((uint32_t)(32 * warp + 16 * (ch & 1)) << 16) + (ch >> 1) * C::OCW + c0, r);
+            tmem_wait_ld();
+            if (live) {
+              const int cbase = ch * C::OCW + c0 + 32 * q;
+              if (cbase + 32 <= ncols_out && ((reinterpret_cast<uintptr_t>(dst + cbase)) & 15) == 0) {
 #pragma unroll
-              for (int k = 0; k < 32; ++k)
-                if (cbase + k < ncols_out) dst[cbase + k] = __uint_as_float(r[k]) * scale;
+                for (int k = 0; k < 32; k += 4) {
+                  float4 o4 = make_float4(__uint_as_float(r[k]) * scale, __uint_as_float(r[k + 1]) * scale,
+                                          __uint_as_float(r[k + 2]) * scale, __uint_as_float(r[k + 3]) * scale);
+                  *reinterpret_cast<float4*>(dst + cbase + k) = o4;
+                }
+              } else {
+#pragma unroll
+                for (int k = 0; k < 32; ++k)
+                  if (cbase + k < ncols_out) dst[cbase + k] = __uint_as_float(r[k]) * scale;
+              }
             }
           }
         }
@@ -629,6 +701,8 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
       }
     }
+    if (lane == 0 && stg_pending) bulk_wait_all();  // the bulk stores are performed before exit
+    __syncwarp();
   }
 
   __syncwarp();

@@ -65,6 +65,7 @@ struct DecodeParams {
   float scale_log2;           // softmax_scale * log2(e)
   float gamma;                // branch_scale
   int write_final;            // whole-sequence segments write `out` directly
+  int tma_out;                // ... through the out tensor map (d_blk_out % 32 == 0)
   uint64_t timeout_ns;        // bound on every wait inside the kernel
 };
 
@@ -100,9 +101,12 @@ enum Variant { kV64 = 0, kV128, kV256, kV512, kNumVariants };
 int variant_smem_bytes(Variant v);
 int variant_tile(Variant v);  // KV positions per tile (64 or 128)
 cudaError_t launch_prep(const PrepParams& p, cudaStream_t st);
+// tout / tpart: fp32 store maps of out [N, H, out_width] and part_o [slots, H, dck], boxes of
+// 16 heads x 32 columns, 128-byte swizzle
 cudaError_t launch_decode(Variant v, const CUtensorMap& tq, const CUtensorMap& tqr,
-                          const CUtensorMap& tc, const CUtensorMap& tkr, const DecodeParams& p,
-                          int grid, cudaStream_t st);
+                          const CUtensorMap& tc, const CUtensorMap& tkr, const CUtensorMap& tout,
+                          const CUtensorMap& tpart, const DecodeParams& p, int grid,
+                          cudaStream_t st);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t st);
 cudaError_t launch_repack(const RepackParams& p, cudaStream_t st);
 cudaError_t launch_resolve_rows(const int32_t* lens_or_null, const int32_t* seq_lens,

@@ -166,6 +166,7 @@ cudaError_t launch_prep(const PrepParams& p, cudaStream_t st) {
 template <int DBLK, int T, int NS>
 static cudaError_t launch_decode_t(const CUtensorMap& tq, const CUtensorMap& tqr,
                                    const CUtensorMap& tc, const CUtensorMap& tkr,
+                                   const CUtensorMap& tout, const CUtensorMap& tpart,
                                    const DecodeParams& p, int grid, cudaStream_t st) {
   using C = DecodeCfg<DBLK, T, NS>;
   auto kern = mlra_decode_kernel<DBLK, T, NS>;
@@ -181,7 +182,7 @@ static cudaError_t launch_decode_t(const CUtensorMap& tq, const CUtensorMap& tqr
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tq, tqr, tc, tkr, p);
+  return cudaLaunchKernelEx(&cfg, kern, tq, tqr, tc, tkr, tout, tpart, p);
 }
 
 // (padded branch width, positions per tile, cache-tile stages)
@@ -210,10 +211,12 @@ int variant_tile(Variant v) {
 }
 
 cudaError_t launch_decode(Variant v, const CUtensorMap& tq, const CUtensorMap& tqr,
-                          const CUtensorMap& tc, const CUtensorMap& tkr, const DecodeParams& p,
-                          int grid, cudaStream_t st) {
+                          const CUtensorMap& tc, const CUtensorMap& tkr, const CUtensorMap& tout,
+                          const CUtensorMap& tpart, const DecodeParams& p, int grid,
+                          cudaStream_t st) {
   switch (v) {
-#define X(id, D, T, NS) case id: return launch_decode_t<D, T, NS>(tq, tqr, tc, tkr, p, grid, st);
+#define X(id, D, T, NS) \
+  case id: return launch_decode_t<D, T, NS>(tq, tqr, tc, tkr, tout, tpart, p, grid, st);
     MLRA_VARIANTS(X)
 #undef X
     default: return cudaErrorInvalidValue;
