@@ -8,7 +8,7 @@ What it computes (sources: "Multi-Head Low-Rank Attention", yunpan.plus page):
   * section 1.3, steps 1-3 of MLA's efficient decode: the absorbed query
     ``q~`` is dotted with the cached latent vectors directly, as MQA-style
     attention with the latent as the shared key/value, and the value
-    up-projection comes afterwards (step 3, not computed here);
+    up-projection comes afterwards (step 3: ``project`` below);
   * section 2: the per-head NoPE key is a sum of B block projections of the
     latent, so splitting ``c_t`` into B column blocks ``c_{t,b}`` is exact;
   * section 3 / 3.1 (MLRA-4): the block sum moves behind the attention; each
@@ -154,3 +154,16 @@ def branch_probabilities(q_lat_s, q_rope_s, c_rows, kr_rows, num_branches, sigma
     _, _, probs = decode_heads(to_f64(q_lat_s), to_f64(q_rope_s), to_f64(c_rows), to_f64(kr_rows),
                                num_branches, sigma, 1.0, with_probs=True)
     return probs
+
+
+def project(out, w_uv):
+    """Step 3 of the absorbed decode (section 1.3; the branch sum of sections 3 and 3.3).
+
+    out [N, H, d_c]: the branch-mode output of ``decode`` (gamma * o_b, branch b in columns
+    b*d_blk .. (b+1)*d_blk).  w_uv [H, d_h, d_c]: head h's value up-projections side by side,
+    W^UV_{h,b} = w_uv[h, :, b*d_blk:(b+1)*d_blk].  The per-branch projections summed over the
+    branches are one product with the concatenation:
+
+        y[s, h] = sum_b W^UV_{h,b} out[s, h, b-block] = w_uv[h] @ out[s, h]      -> [N, H, d_h]
+    """
+    return np.einsum("hkd,shd->shk", to_f64(w_uv), to_f64(out))

@@ -61,7 +61,8 @@ def explicit_mlra(q_nope, q_rope, c, kr, W_uk, W_uv, sigma, gamma):
 
 
 def pin_absorbed_equals_explicit(orc, seed=0, H=6, B=4, d_blk=8, d_R=4, d_h=5, L=37):
-    """Step 1 absorption + step 2 + step 3 == explicit decompressed attention (section 1.3, 2, 3)."""
+    """Step 1 absorption + step 2 + step 3 (the oracle's ``project``) == explicit decompressed
+    attention (section 1.3, 2, 3)."""
     rng = np.random.default_rng(seed)
     W_uk, W_uv = _rand(rng, H, B, d_h, d_blk), _rand(rng, H, B, d_h, d_blk)
     q_nope, q_rope = _rand(rng, H, B, d_h), _rand(rng, H, d_R)
@@ -70,7 +71,8 @@ def pin_absorbed_equals_explicit(orc, seed=0, H=6, B=4, d_blk=8, d_R=4, d_h=5, L
     ref = explicit_mlra(q_nope, q_rope, c, kr, W_uk, W_uv, sigma, gamma)
     q_lat = np.concatenate([np.einsum("hkd,hk->hd", W_uk[:, b], q_nope[:, b]) for b in range(B)], 1)
     out, _ = _one_seq(orc, q_lat, q_rope, c, kr, B, sigma, gamma)
-    y = sum(np.einsum("hkd,hd->hk", W_uv[:, b], out[:, b * d_blk:(b + 1) * d_blk]) for b in range(B))
+    w_cat = np.concatenate([W_uv[:, b] for b in range(B)], axis=2)   # [H, d_h, d_c]
+    y = orc.project(out[None], w_cat)[0]                             # step 3
     err = np.abs(y - ref).max() / np.abs(ref).max()
     assert err <= 1e-12, f"absorbed vs explicit rel err {err:.3e}"
 
@@ -304,7 +306,28 @@ def pin_golden_rows(orc):
         assert cont == f["contiguous_rows"][s], f"contiguous rows of sequence {s}"
 
 
+def pin_project_brute_force(orc, seed=9, N=2, H=3, B=2, d_blk=4, d_h=3):
+    """Step 3 by plain loops: y[s,h,k] = sum_b sum_i W^UV_{h,b}[k,i] out[s,h,b*d_blk+i]; and with
+    identity blocks (d_h = d_blk) y is the plain sum of the branch outputs (section 3.3)."""
+    rng = np.random.default_rng(seed)
+    out = _rand(rng, N, H, B * d_blk)
+    w = _rand(rng, H, d_h, B * d_blk)
+    y = orc.project(out, w)
+    for s_ in range(N):
+        for h in range(H):
+            for k in range(d_h):
+                acc = 0.0
+                for b in range(B):
+                    for i in range(d_blk):
+                        acc += w[h, k, b * d_blk + i] * out[s_, h, b * d_blk + i]
+                assert abs(y[s_, h, k] - acc) <= 1e-12 * (1 + abs(acc)), "project vs loops"
+    eye = np.tile(np.eye(d_blk), (H, 1, B))                           # [H, d_blk, B*d_blk]
+    y_eye = orc.project(out, eye)
+    assert np.allclose(y_eye, out.reshape(N, H, B, d_blk).sum(axis=2), rtol=0, atol=1e-12), "identity"
+
+
 ALL_PINS = [
+    pin_project_brute_force,
     pin_absorbed_equals_explicit,
     pin_summed_equals_explicit_shared_wuv,
     pin_b1_equals_mqa,

@@ -33,6 +33,12 @@ MUTANTS = {
     "contiguous_pitch": ("return s * np.int64(max_seq_len) + j", "return s * np.int64(max_seq_len + 1) + j"),
     "empty_lse_zero": ("lse = np.full((hq, B), -np.inf)", "lse = np.zeros((hq, B))"),
     "probs_from_other_branch": ("probs.append(p)", "probs.append(p if b == 0 else probs[0])"),
+    "project_transposed_weight": ('np.einsum("hkd,shd->shk", to_f64(w_uv), to_f64(out))',
+                                  'np.einsum("hkd,shk->shd", to_f64(w_uv), to_f64(out)[..., :w_uv.shape[1]])'),
+    "project_first_branch_only": ('np.einsum("hkd,shd->shk", to_f64(w_uv), to_f64(out))',
+                                  'np.einsum("hkd,shd->shk", to_f64(w_uv)[..., :8], to_f64(out)[..., :8])'),
+    "project_head_shift": ('np.einsum("hkd,shd->shk", to_f64(w_uv), to_f64(out))',
+                           'np.einsum("hkd,shd->shk", np.roll(to_f64(w_uv), 1, axis=0), to_f64(out))'),
 }
 
 
