@@ -178,6 +178,23 @@ mlra_status mlra_decode_static_scratch(const void* q_lat, const void* q_rope, co
                                        float* out, float* lse, const mlra_dims* dims,
                                        mlra_stream_t stream);
 
+/* Step 3 of the absorbed decode: the value up-projection of every branch output, summed over the
+ * branches ("Multi-Head Low-Rank Attention", yunpan.plus page, section 1.3 step 3; the branch sum
+ * of sections 3 and 3.3).  Head h's projections sit side by side,
+ * W_h = [W^UV_{h,1} | ... | W^UV_{h,B}]:
+ *     y[s, h, :] = W_h o[s, h, :]
+ *   o     [N, H, d_latent] fp32 device: mlra_decode's output in MLRA_OUT_BRANCHES mode (gamma
+ *         already applied)
+ *   w_uv  [H, d_head, d_latent] bf16 device, row-major: W_h row k = w_uv[h, k, :]
+ *   y     [N, H, d_head] fp32 device (written)
+ *   status nullable device uint32: gets MLRA_FLAG_TIMEOUT if a bounded wait runs out
+ * Products in bf16 (o is rounded to bf16) with fp32 accumulation.  Asynchronous on `stream`.
+ * Errors: MLRA_ERR_INVALID_ARG for null pointers or sizes < 1; MLRA_ERR_UNSUPPORTED unless
+ * d_latent is a multiple of 64 up to 512, d_head a multiple of 64 and all three arrays 16-byte
+ * aligned; MLRA_ERR_CUDA when the launch fails.  The pages give no kernel for this step. */
+mlra_status mlra_project(const float* o, const void* w_uv, float* y, int N, int H, int d_latent,
+                         int d_head, uint32_t* status, mlra_stream_t stream);
+
 /* Reads the status word that the last mlra_decode on `workspace` left, after synchronising
  * `stream`.  *flags_host receives the MLRA_FLAG_* bits; the return value is MLRA_OK when no
  * bit is set, else the status of the most serious bit (timeout, bad page, bad length). */

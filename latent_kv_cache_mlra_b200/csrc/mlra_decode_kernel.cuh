@@ -628,38 +628,73 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       } else if (!to_final || p.tma_out) {
         // Through shared memory and the TMA: each [16 heads x 32 columns] box is staged in the
         // 128-byte swizzled layout and stored by one bulk copy (rows past H are clipped by the
-        // tensor map).  Partials go to slot range + seq of part_o, finals to out.
+        // tensor map).  Partials go to slot range + seq of part_o, finals to out.  In the
+        // range's last segment the stage ring is idle (every load landed, every product that
+        // read it completed), so each warp stages all its boxes there and issues them back to
+        // back; otherwise the boxes take turns in the warp's own 2 KB buffer.
+        const bool last_seg = walk.i == walk.count;
+        uint8_t* ring = smem + C::OFF_STAGE + warp * (16 * DBLK * 4);
         const CUtensorMap* map = to_final ? &tm_out : &tm_part;
         const int x0 = to_final ? branch * p.d_blk_out : branch * DBLK;
         const int z = to_final ? seg.seq : range + seg.seq;
         const int row = lane & 15;
+        if (last_seg) {
+          // both halves of every 64-column chunk at once (distinct boxes), one fence, then the
+          // whole warp's boxes are issued together
 #pragma unroll 1
-        for (int ch = 0; ch < C::OCH; ++ch) {
+          for (int ch = 0; ch < C::OCH; ++ch) {
 #pragma unroll 1
-          for (int c0 = 0; c0 < C::OCW; c0 += 64) {
-            uint32_t r[32];
-            tmem_ld16x2_32(tmem + ((uint32_t)(32 * warp + 16 * (ch & 1)) << 16) + (ch >> 1) * C::OCW + c0, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              const int col = ch * C::OCW + c0 + 32 * half;  // column inside the branch block
-              if (col >= ncols_out) continue;
-              if (lane == 0 && stg_pending) bulk_wait_read_all();
-              __syncwarp();
-              if (q == half) {
+            for (int c0 = 0; c0 < C::OCW; c0 += 64) {
+              uint32_t r[32];
+              tmem_ld16x2_32(tmem + ((uint32_t)(32 * warp + 16 * (ch & 1)) << 16) + (ch >> 1) * C::OCW + c0, r);
+              tmem_wait_ld();
+              const int col = ch * C::OCW + c0 + 32 * q;
+              if (col < ncols_out) {
+                uint8_t* buf = ring + (col / 32) * C::STG_BYTES;
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                  *reinterpret_cast<float4*>(stg + row * 128 + ((k ^ (row & 7)) << 4)) =
+                  *reinterpret_cast<float4*>(buf + row * 128 + ((k ^ (row & 7)) << 4)) =
                       make_float4(__uint_as_float(r[4 * k]) * scale, __uint_as_float(r[4 * k + 1]) * scale,
                                   __uint_as_float(r[4 * k + 2]) * scale, __uint_as_float(r[4 * k + 3]) * scale);
               }
-              fence_proxy_async_smem();  // the staged box is read by the bulk copy (async proxy)
-              __syncwarp();
-              if (lane == 0) {
-                tma_store_3d(map, stg_u, x0 + col, 16 * warp, z);
-                bulk_commit();
+            }
+          }
+          fence_proxy_async_smem();  // the staged boxes are read by the bulk copies (async proxy)
+          __syncwarp();
+          if (lane == 0) {
+            for (int col = 0; col < ncols_out && col < DBLK; col += 32)
+              tma_store_3d(map, smem_u32(ring + (col / 32) * C::STG_BYTES), x0 + col, 16 * warp, z);
+            bulk_commit();
+          }
+        } else {
+#pragma unroll 1
+          for (int ch = 0; ch < C::OCH; ++ch) {
+#pragma unroll 1
+            for (int c0 = 0; c0 < C::OCW; c0 += 64) {
+              uint32_t r[32];
+              tmem_ld16x2_32(tmem + ((uint32_t)(32 * warp + 16 * (ch & 1)) << 16) + (ch >> 1) * C::OCW + c0, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int half = 0; half < 2; ++half) {
+                const int col = ch * C::OCW + c0 + 32 * half;  // column inside the branch block
+                if (col >= ncols_out) continue;
+                if (lane == 0 && stg_pending) bulk_wait_read_all();
+                __syncwarp();
+                if (q == half) {
+#pragma unroll
+                  for (int k = 0; k < 8; ++k)
+                    *reinterpret_cast<float4*>(stg + row * 128 + ((k ^ (row & 7)) << 4)) =
+                        make_float4(__uint_as_float(r[4 * k]) * scale, __uint_as_float(r[4 * k + 1]) * scale,
+                                    __uint_as_float(r[4 * k + 2]) * scale, __uint_as_float(r[4 * k + 3]) * scale);
+                }
+                fence_proxy_async_smem();  // the staged box is read by the bulk copy (async proxy)
+                __syncwarp();
+                if (lane == 0) {
+                  tma_store_3d(map, stg_u, x0 + col, 16 * warp, z);
+                  bulk_commit();
+                }
+                stg_pending = true;
               }
-              stg_pending = true;
             }
           }
         }
@@ -701,7 +736,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
       }
     }
-    if (lane == 0 && stg_pending) bulk_wait_all();  // the bulk stores are performed before exit
+    if (lane == 0) bulk_wait_all();  // every bulk store of this warp is performed before exit
     __syncwarp();
   }
 

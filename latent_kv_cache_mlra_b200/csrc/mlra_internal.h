@@ -87,6 +87,15 @@ struct CombineParams {
   float gamma;
 };
 
+// Step 3 (K5): y[N, H, d_head] = per head, W_h [d_head, d_latent] times o[N, H, d_latent].
+struct ProjectParams {
+  const float* o;             // branch-mode output of the decode, fp32
+  float* y;
+  uint32_t* status;           // nullable: kFlagTimeout on a wait that ran out
+  int N, H, d_latent, d_head;
+  uint64_t timeout_ns;
+};
+
 struct RepackParams {
   const void* q_lat; const void* q_rope; const void* c_kv; const void* k_rope;
   uint16_t* q_out; uint16_t* qr_out; uint16_t* c_out; uint16_t* kr_out;
@@ -109,6 +118,8 @@ cudaError_t launch_decode(Variant v, const CUtensorMap& tq, const CUtensorMap& t
                           cudaStream_t st);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t st);
 cudaError_t launch_repack(const RepackParams& p, cudaStream_t st);
+// tw: bf16 map over W [H * d_head rows, d_latent columns], [64 x 64] boxes, 128-byte swizzle
+cudaError_t launch_project(const CUtensorMap& tw, const ProjectParams& p, cudaStream_t st);
 cudaError_t launch_resolve_rows(const int32_t* lens_or_null, const int32_t* seq_lens,
                                 const int32_t* page_table, int N, int max_pages, int page_size,
                                 int max_seq_len, int64_t n_pages, int oob_row, int64_t* rows_out,

@@ -6,12 +6,15 @@
 //   K2 mlra_combine_kernel   merges the partial softmax states of split sequences and writes
 //                            the call's status word
 //   K3 mlra_repack_kernel    fp32 / odd-width inputs -> padded bf16 copies in the workspace
+//   K5 mlra_project_kernel   step 3: per-head value up-projection summed over the branches
+//                            (mlra_project_kernel.cuh)
 //   mlra_resolve_rows_kernel test hook for the cache-row addressing of K1
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
 #include "mlra_decode_kernel.cuh"
 #include "mlra_merge.cuh"
+#include "mlra_project_kernel.cuh"
 #include "sm100_ptx.cuh"
 #include "mlra_internal.h"
 #include "mlra_plan.cuh"
@@ -358,6 +361,24 @@ cudaError_t launch_repack(const RepackParams& p, cudaStream_t st) {
   if (p.src_f32) mlra_repack_kernel<float><<<grid, 256, 0, st>>>(p);
   else mlra_repack_kernel<uint16_t><<<grid, 256, 0, st>>>(p);
   return cudaGetLastError();
+}
+
+// ----------------------------------------------------------------------------- K5
+cudaError_t launch_project(const CUtensorMap& tw, const ProjectParams& p, cudaStream_t st) {
+  const int smem = project_smem_bytes(p.d_latent / 64);
+  cudaError_t e = cudaFuncSetAttribute(mlra_project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.H * (p.d_head / kProjM), (p.N + kProjN - 1) / kProjN);
+  cfg.blockDim = dim3(kProjThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, mlra_project_kernel, tw, p);
 }
 
 // ----------------------------------------------------------------------------- test hook

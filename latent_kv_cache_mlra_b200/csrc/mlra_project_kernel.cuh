@@ -1,0 +1,145 @@
+// mlra_project_kernel.cuh -- K5: step 3 of the absorbed decode on sm_100a.
+//
+// "Multi-Head Low-Rank Attention" (yunpan.plus page), section 1.3 step 3 with the branch sum of
+// sections 3 and 3.3: the value up-projection of every branch output, summed over the branches.
+// With head h's projections side by side, W_h = [W^UV_{h,1} | ... | W^UV_{h,B}] (d_head x d_latent),
+// and o[s, h] the concatenated branch outputs of step 2 (gamma already applied):
+//     y[s, h, :] = W_h o[s, h, :]
+// One CTA per (head, 64 rows of d_head, 64 sequences): a tcgen05 product with M = 64 rows of W_h,
+// N = the sequences (padded to a multiple of 8), K = d_latent, accumulated in TMEM.
+//   * W_h's rows arrive by TMA as [64 x 64] bf16 boxes (128-byte swizzle, K-major);
+//   * o (fp32) is rounded to bf16 by all threads into the same swizzled K-major layout;
+//   * one thread issues the d_latent / 16 MMAs; the epilogue reads D with tcgen05.ld and
+//     writes y (a warp's 16 rows of one sequence are 64 contiguous bytes).
+// The work is bound by streaming W (H d_head d_latent bf16) from HBM.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+
+#include "mlra_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace mlra {
+
+constexpr int kProjThreads = 128;
+constexpr int kProjM = 64;     // rows of W_h per CTA
+constexpr int kProjN = 64;     // sequences per CTA
+constexpr int kProjBox = 8192; // one [64 x 64] bf16 box
+
+// shared memory: W boxes, o boxes, two mbarriers, the TMEM address
+inline int project_smem_bytes(int kb) { return 2 * kb * kProjBox + 32 + 1024; }
+
+__device__ __forceinline__ bool project_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns,
+                                             uint32_t* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > timeout_ns) {
+      if (status) atomicOr(status, kFlagTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+__global__ void __launch_bounds__(kProjThreads, 1)
+mlra_project_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ ProjectParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int KB = p.d_latent / 64;
+  uint8_t* sW = smem;
+  uint8_t* sX = smem + KB * kProjBox;
+  const uint32_t bar_full = smem_u32(sX + KB * kProjBox);
+  const uint32_t bar_done = bar_full + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sX + KB * kProjBox + 16);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mtiles = p.d_head / kProjM;
+  const int h = blockIdx.x / mtiles, m0 = (blockIdx.x % mtiles) * kProjM;
+  const int n0 = blockIdx.y * kProjN;
+  const int rows_n = min(kProjN, p.N - n0);
+  const int npad = (rows_n + 7) / 8 * 8;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_full, 1);
+    mbar_init(bar_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 64);
+    tmem_relinquish();
+  }
+  if (warp == 1 && lane == 0) tma_prefetch_desc(&tm_w);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // o comes from the previous kernel on the stream (programmatic serialization)
+  pdl_wait_prerequisites();
+
+  if (warp == 1 && lane == 0) {
+    mbar_arrive_expect_tx(bar_full, KB * kProjBox);
+    for (int kb = 0; kb < KB; ++kb)
+      tma_load_2d(smem_u32(sW + kb * kProjBox), &tm_w, bar_full, 64 * kb, h * p.d_head + m0);
+  }
+  // o[n0 + r, h, :] -> bf16, box kb holds columns 64 kb .. 64 kb + 63 of row r at 128 r, its
+  // 16-byte chunk j at position j ^ (r & 7)
+  for (int idx = threadIdx.x; idx < kProjN * KB * 8; idx += kProjThreads) {
+    const int r = idx / (KB * 8), cidx = idx - r * (KB * 8);
+    const int kb = cidx >> 3, j = cidx & 7;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (r < rows_n) {
+      const float4* src = reinterpret_cast<const float4*>(
+          p.o + ((int64_t)(n0 + r) * p.H + h) * p.d_latent + kb * 64 + j * 8);
+      const float4 a = __ldcg(src), b = __ldcg(src + 1);
+      v = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
+                     pack_bf16x2(b.z, b.w));
+    }
+    *reinterpret_cast<uint4*>(sX + kb * kProjBox + r * 128 + ((j ^ (r & 7)) << 4)) = v;
+  }
+  fence_proxy_async_smem();  // read by the MMA (async proxy)
+  __syncthreads();
+
+  bool ok = true;
+  if (threadIdx.x == 0) {
+    ok = project_wait(bar_full, 0, p.timeout_ns, p.status);
+    if (ok) {
+      tc_fence_after();
+      const uint32_t idesc = idesc_bf16_f32(kProjM, npad, false, false);
+      for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_bf16(tmem, sw128_desc(smem_u32(sW + kb * kProjBox) + kk * 32, 16, 1024),
+                    sw128_desc(smem_u32(sX + kb * kProjBox) + kk * 32, 16, 1024), idesc,
+                    (kb | kk) ? 1u : 0u);
+      umma_commit(bar_done);
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;  // warp 0 knows; others just wait below
+  if (warp != 0 || ok) {
+    // every thread waits for the products (bounded); warp 0 skips when nothing was issued
+    const bool done = __all_sync(0xffffffffu,
+                                 project_wait(bar_done, 0, p.timeout_ns, warp == 0 ? p.status : nullptr));
+    if (done) {  // warp-uniform: tcgen05.ld is a warp-wide instruction
+      tc_fence_after();
+      // D rows 16 w .. 16 w + 15 live in lanes 32 w + [0, 16); lane half q holds columns
+      // 32 q .. 32 q + 31 (the sequences n0 + column)
+      uint32_t r[32];
+      tmem_ld16x2_32(tmem + ((uint32_t)(32 * warp) << 16), r);
+      tmem_wait_ld();
+      const int row = m0 + 16 * warp + (lane & 15), q = lane >> 4;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const int col = 32 * q + k;
+        if (col < rows_n)
+          p.y[((int64_t)(n0 + col) * p.H + h) * p.d_head + row] = __uint_as_float(r[k]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 64);
+}
+
+}  // namespace mlra

@@ -27,7 +27,7 @@ FLAG_TIMEOUT, FLAG_BAD_PAGE, FLAG_BAD_LENGTH = 0x1, 0x2, 0x4
 EXPORTS = ("mlra_workspace_size", "mlra_decode", "mlra_decode_profiled", "mlra_query_plan",
            "mlra_decode_static_scratch",
            "mlra_read_status", "mlra_debug_resolve_rows", "mlra_plan_host",
-           "mlra_plan_segments_host", "mlra_status_string", "mlra_version")
+           "mlra_plan_segments_host", "mlra_project", "mlra_status_string", "mlra_version")
 
 
 class Dims(ctypes.Structure):
@@ -82,13 +82,15 @@ def lib() -> ctypes.CDLL:
         L.mlra_plan_segments_host.argtypes = [i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, i32p,
                                               i32p, i32p, i32p, ctypes.c_int,
                                               ctypes.POINTER(ctypes.c_int)]
+        L.mlra_project.argtypes = [vp, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                   vp, vp]
         L.mlra_status_string.argtypes = [ctypes.c_int]
         L.mlra_status_string.restype = ctypes.c_char_p
         L.mlra_version.argtypes = []
         for f in ("mlra_workspace_size", "mlra_decode", "mlra_decode_profiled", "mlra_query_plan",
                   "mlra_decode_static_scratch",
                   "mlra_read_status", "mlra_debug_resolve_rows", "mlra_plan_host",
-                  "mlra_plan_segments_host"):
+                  "mlra_plan_segments_host", "mlra_project"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -151,6 +153,24 @@ def dims_for(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table, num_branches, *,
                      kr_row_stride=k_rope.stride(0), page_size=page_size,
                      max_pages_per_seq=max_pages, dtype=dtype, out_mode=out_mode,
                      num_ranges=num_ranges)
+
+
+def project(o: torch.Tensor, w_uv: torch.Tensor, y: Optional[torch.Tensor] = None, status=None,
+            stream=None) -> torch.Tensor:
+    """Step 3 through ``mlra_project``: y[s, h] = w_uv[h] @ o[s, h] (o fp32 [N, H, d_latent] from
+    ``decode`` in branch mode, w_uv bf16 [H, d_head, d_latent]); returns y fp32 [N, H, d_head]."""
+    N, H, d_latent = o.shape
+    d_head = w_uv.shape[1]
+    if o.dtype != torch.float32 or w_uv.dtype != torch.bfloat16 or w_uv.shape != (H, d_head, d_latent):
+        raise ValueError("project: o fp32 [N, H, d_latent], w_uv bf16 [H, d_head, d_latent]")
+    if not (o.is_contiguous() and w_uv.is_contiguous()):
+        raise ValueError("project: contiguous tensors expected")
+    if y is None:
+        y = torch.empty(N, H, d_head, dtype=torch.float32, device=o.device)
+    st = stream if stream is not None else torch.cuda.current_stream(o.device).cuda_stream
+    _check(lib().mlra_project(_ptr(o), _ptr(w_uv), _ptr(y), N, H, d_latent, d_head, _ptr(status),
+                              ctypes.c_void_p(st)), "mlra_project")
+    return y
 
 
 def decode(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table=None, *, num_branches: int,

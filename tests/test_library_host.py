@@ -254,3 +254,17 @@ def test_plan_host_rejects():
         mlra.plan_host([1, 2], 0)
     with pytest.raises(mlra.MlraError):
         mlra.plan_host([1, 2], 4, -1)
+
+
+def test_project_argument_errors_without_a_gpu():
+    """mlra_project checks its sizes and alignment before touching the device."""
+    lib = mlra.lib()
+    fake = ctypes.c_void_p(4096)
+    ok = [fake, fake, fake, 8, 64, 512, 128, None, None]
+    for i, v, want in [(0, None, mlra.MLRA_ERR_INVALID_ARG), (3, 0, mlra.MLRA_ERR_INVALID_ARG),
+                       (4, 0, mlra.MLRA_ERR_INVALID_ARG), (5, 96, mlra.MLRA_ERR_UNSUPPORTED),
+                       (5, 576, mlra.MLRA_ERR_UNSUPPORTED), (6, 100, mlra.MLRA_ERR_UNSUPPORTED),
+                       (2, ctypes.c_void_p(4100), mlra.MLRA_ERR_UNSUPPORTED)]:
+        args = list(ok)
+        args[i] = v
+        assert lib.mlra_project(*args) == want, (i, v)
