@@ -297,11 +297,14 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
     launches_per_step = dec.plan.launches
     nbytes, nflops = cache_bytes(inp), algorithmic_flops(inp)
-    flush = None if nbytes > L2_BYTES else torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    # inputs smaller than L2 are evicted before each step by reading a buffer twice the L2 size
+    # (a read leaves clean lines: the timed kernels pay no write-back of the flush)
+    flush = None if nbytes > L2_BYTES else torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
 
     def step(ev=None):
         if flush is not None:
-            flush.zero_()
+            torch.sum(flush, out=sink)
         dec(k1_events=ev)
 
     for _ in range(args.warmup):
@@ -408,6 +411,62 @@ def run_ours(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- step 3
+def run_project(args):
+    """Times step 3 (mlra_project) alone on the workload's shapes: o = one decode's output,
+    W^UV [H, d_head = 128, d_latent] bf16 drawn N(0, 1/d_latent).  Bound by streaming W."""
+    from latent_kv_cache_mlra_b200 import mlra
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = workloads.get(args.workload)
+    inp = workloads.make_inputs(w)
+    pt = None if inp.page_table is None else inp.page_table.to(dev)
+    dec = mlra.Decoder(inp.q_lat.to(dev), inp.q_rope.to(dev), inp.c_kv.to(dev), inp.k_rope.to(dev),
+                       inp.seq_lens.to(dev), pt, num_branches=w.num_branches, softmax_scale=w.sigma,
+                       branch_scale=w.gamma, max_seq_len=inp.max_seq_len, page_size=w.page_size)
+    o = dec().contiguous()
+    d_head = 128
+    g = torch.Generator().manual_seed(w.seed + 77)
+    w_uv = (torch.randn(w.heads, d_head, w.d_latent, generator=g) / w.d_latent ** 0.5).to(
+        torch.bfloat16).to(dev)
+    y = torch.empty(w.batch, w.heads, d_head, dtype=torch.float32, device=dev)
+    # W fits in L2: evict it before each launch by reading a buffer twice the L2 size (a read
+    # leaves clean lines, so the timed kernel pays no write-back of the flush)
+    flush = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        torch.sum(flush, out=sink)
+        mlra.project(o, w_uv, y)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    with ClockSampler(0) as clk:
+        for a, b in evs:
+            torch.sum(flush, out=sink)
+            a.record()
+            mlra.project(o, w_uv, y)
+            b.record()
+        torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+    nbytes = w_uv.numel() * 2 + o.numel() * 4 + y.numel() * 4
+    flops = 2 * w.batch * w.heads * d_head * w.d_latent
+    peaks = measured_peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    print(json.dumps({
+        "metric": "step-3 projection (W^UV, branch sum) time per decode step", "value": ms * 1e3,
+        "unit": "us", "higher_is_better": False, "steps": args.steps, "warmup": args.warmup,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "d_latent": w.d_latent,
+                   "d_head": d_head, "l2": "L2 flushed (read of 2x L2) before each launch"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "kernel": "mlra_project_kernel",
+                     "algorithmic_bytes_per_launch": nbytes,
+                     "tensor_tflops": flops / (ms * 1e-3) / 1e12},
+        "clocks": clk.summary()}))
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -416,11 +475,15 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stage", choices=["decode", "project"], default="decode",
+                    help="decode: the attention path (default line); project: step 3 alone")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.stage == "project":
+        return run_project(args)
     return run_ours(args)
 
 
