@@ -26,8 +26,9 @@ constexpr int kProjM = 64;     // rows of W_h per CTA
 constexpr int kProjN = 64;     // sequences per CTA
 constexpr int kProjBox = 8192; // one [64 x 64] bf16 box
 
-// shared memory: W boxes, o boxes, two mbarriers, the TMEM address
-inline int project_smem_bytes(int kb) { return 2 * kb * kProjBox + 32 + 1024; }
+// shared memory: W boxes, o boxes, an mbarrier per W box and one for the products, the TMEM
+// address
+inline int project_smem_bytes(int kb) { return 2 * kb * kProjBox + 8 * (kb + 1) + 16 + 1024; }
 
 __device__ __forceinline__ bool project_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns,
                                              uint32_t* status) {
@@ -50,9 +51,10 @@ mlra_project_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
   const int KB = p.d_latent / 64;
   uint8_t* sW = smem;
   uint8_t* sX = smem + KB * kProjBox;
-  const uint32_t bar_full = smem_u32(sX + KB * kProjBox);
-  const uint32_t bar_done = bar_full + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sX + KB * kProjBox + 16);
+  const uint32_t bar_full = smem_u32(sX + KB * kProjBox);  // [KB]: W box kb landed
+  const uint32_t bar_done = bar_full + 8 * KB;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sX + KB * kProjBox + 8 * (KB + 1));
+  volatile uint32_t* issued_all = tmem_slot + 1;  // every product was issued (no time-out)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int mtiles = p.d_head / kProjM;
   const int h = blockIdx.x / mtiles, m0 = (blockIdx.x % mtiles) * kProjM;
@@ -61,7 +63,7 @@ mlra_project_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
   const int npad = (rows_n + 7) / 8 * 8;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_full, 1);
+    for (int kb = 0; kb < KB; ++kb) mbar_init(bar_full + 8 * kb, 1);
     mbar_init(bar_done, 1);
     fence_barrier_init();
   }
@@ -78,49 +80,67 @@ mlra_project_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
   pdl_wait_prerequisites();
 
   if (warp == 1 && lane == 0) {
-    mbar_arrive_expect_tx(bar_full, KB * kProjBox);
-    for (int kb = 0; kb < KB; ++kb)
-      tma_load_2d(smem_u32(sW + kb * kProjBox), &tm_w, bar_full, 64 * kb, h * p.d_head + m0);
+    for (int kb = 0; kb < KB; ++kb) {
+      mbar_arrive_expect_tx(bar_full + 8 * kb, kProjBox);
+      tma_load_2d(smem_u32(sW + kb * kProjBox), &tm_w, bar_full + 8 * kb, 64 * kb, h * p.d_head + m0);
+    }
   }
   // o[n0 + r, h, :] -> bf16, box kb holds columns 64 kb .. 64 kb + 63 of row r at 128 r, its
-  // 16-byte chunk j at position j ^ (r & 7)
-  for (int idx = threadIdx.x; idx < kProjN * KB * 8; idx += kProjThreads) {
-    const int r = idx / (KB * 8), cidx = idx - r * (KB * 8);
-    const int kb = cidx >> 3, j = cidx & 7;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (r < rows_n) {
-      const float4* src = reinterpret_cast<const float4*>(
-          p.o + ((int64_t)(n0 + r) * p.H + h) * p.d_latent + kb * 64 + j * 8);
-      const float4 a = __ldcg(src), b = __ldcg(src + 1);
-      v = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
-                     pack_bf16x2(b.z, b.w));
+  // 16-byte chunk j at position j ^ (r & 7).  Only the npad rows the products read are staged
+  // (rows past the batch as zeros); the loads of 8 chunks are issued before any is converted.
+  constexpr int kU = 8;
+  const int chunks = npad * KB * 8;
+  for (int base = threadIdx.x; base < chunks; base += kProjThreads * kU) {
+    float4 va[kU], vb[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int idx = base + u * kProjThreads;
+      const int r = idx / (KB * 8), cidx = idx - r * (KB * 8);
+      va[u] = vb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (idx < chunks && r < rows_n) {
+        const float4* src = reinterpret_cast<const float4*>(
+            p.o + ((int64_t)(n0 + r) * p.H + h) * p.d_latent + cidx * 8);
+        va[u] = __ldcg(src);
+        vb[u] = __ldcg(src + 1);
+      }
     }
-    *reinterpret_cast<uint4*>(sX + kb * kProjBox + r * 128 + ((j ^ (r & 7)) << 4)) = v;
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int idx = base + u * kProjThreads;
+      if (idx >= chunks) break;
+      const int r = idx / (KB * 8), cidx = idx - r * (KB * 8);
+      const int kb = cidx >> 3, j = cidx & 7;
+      *reinterpret_cast<uint4*>(sX + kb * kProjBox + r * 128 + ((j ^ (r & 7)) << 4)) =
+          make_uint4(pack_bf16x2(va[u].x, va[u].y), pack_bf16x2(va[u].z, va[u].w),
+                     pack_bf16x2(vb[u].x, vb[u].y), pack_bf16x2(vb[u].z, vb[u].w));
+    }
   }
   fence_proxy_async_smem();  // read by the MMA (async proxy)
   __syncthreads();
 
   bool ok = true;
   if (threadIdx.x == 0) {
-    ok = project_wait(bar_full, 0, p.timeout_ns, p.status);
-    if (ok) {
+    // the products of box kb start as soon as it lands
+    const uint32_t idesc = idesc_bf16_f32(kProjM, npad, false, false);
+    for (int kb = 0; ok && kb < KB; ++kb) {
+      ok = project_wait(bar_full + 8 * kb, 0, p.timeout_ns, p.status);
+      if (!ok) break;
       tc_fence_after();
-      const uint32_t idesc = idesc_bf16_f32(kProjM, npad, false, false);
-      for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_bf16(tmem, sw128_desc(smem_u32(sW + kb * kProjBox) + kk * 32, 16, 1024),
-                    sw128_desc(smem_u32(sX + kb * kProjBox) + kk * 32, 16, 1024), idesc,
-                    (kb | kk) ? 1u : 0u);
-      umma_commit(bar_done);
+      for (int kk = 0; kk < 4; ++kk)
+        umma_bf16(tmem, sw128_desc(smem_u32(sW + kb * kProjBox) + kk * 32, 16, 1024),
+                  sw128_desc(smem_u32(sX + kb * kProjBox) + kk * 32, 16, 1024), idesc,
+                  (kb | kk) ? 1u : 0u);
     }
+    *issued_all = ok ? 1u : 0u;
+    umma_commit(bar_done);  // also after a time-out: it tracks whatever was issued
   }
-  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;  // warp 0 knows; others just wait below
-  if (warp != 0 || ok) {
-    // every thread waits for the products (bounded); warp 0 skips when nothing was issued
-    const bool done = __all_sync(0xffffffffu,
-                                 project_wait(bar_done, 0, p.timeout_ns, warp == 0 ? p.status : nullptr));
-    if (done) {  // warp-uniform: tcgen05.ld is a warp-wide instruction
+  __syncthreads();
+  {
+    // every thread waits for the products (bounded)
+    const bool done = __all_sync(0xffffffffu, project_wait(bar_done, 0, p.timeout_ns,
+                                                           threadIdx.x == 0 ? p.status : nullptr));
+    if (done && *issued_all) {  // warp-uniform: tcgen05.ld is a warp-wide instruction
       tc_fence_after();
       // D rows 16 w .. 16 w + 15 live in lanes 32 w + [0, 16); lane half q holds columns
       // 32 q .. 32 q + 31 (the sequences n0 + column)
