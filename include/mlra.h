@@ -183,17 +183,25 @@ mlra_status mlra_decode_static_scratch(const void* q_lat, const void* q_rope, co
  * of sections 3 and 3.3).  Head h's projections sit side by side,
  * W_h = [W^UV_{h,1} | ... | W^UV_{h,B}]:
  *     y[s, h, :] = W_h o[s, h, :]
- *   o     [N, H, d_latent] fp32 device: mlra_decode's output in MLRA_OUT_BRANCHES mode (gamma
- *         already applied)
- *   w_uv  [H, d_head, d_latent] bf16 device, row-major: W_h row k = w_uv[h, k, :]
- *   y     [N, H, d_head] fp32 device (written)
+ *   o        [N, H, d_latent] fp32 device: mlra_decode's output in MLRA_OUT_BRANCHES mode (gamma
+ *            already applied)
+ *   w_packed H * d_head * d_latent bf16 device: the weights W^UV as mlra_pack_wuv wrote them
+ *   y        [N, H, d_head] fp32 device (written)
  *   status nullable device uint32: gets MLRA_FLAG_TIMEOUT if a bounded wait runs out
  * Products in bf16 (o is rounded to bf16) with fp32 accumulation.  Asynchronous on `stream`.
  * Errors: MLRA_ERR_INVALID_ARG for null pointers or sizes < 1; MLRA_ERR_UNSUPPORTED unless
  * d_latent is a multiple of 64 up to 512, d_head a multiple of 64 and all three arrays 16-byte
  * aligned; MLRA_ERR_CUDA when the launch fails.  The pages give no kernel for this step. */
-mlra_status mlra_project(const float* o, const void* w_uv, float* y, int N, int H, int d_latent,
+mlra_status mlra_project(const float* o, const void* w_packed, float* y, int N, int H, int d_latent,
                          int d_head, uint32_t* status, mlra_stream_t stream);
+
+/* Packs the step-3 weights once for mlra_project (they are model weights: pack at load time).
+ *   w_uv     [H, d_head, d_latent] bf16 device, row-major: W_h row k = w_uv[h, k, :]
+ *   w_packed H * d_head * d_latent bf16 device (written; same size, caller-owned): per head and
+ *            64-row tile, the d_latent / 64 blocks of 64 columns in the tensor-core image
+ * Asynchronous on `stream`.  Errors as mlra_project (sizes, 16-byte alignment). */
+mlra_status mlra_pack_wuv(const void* w_uv, void* w_packed, int H, int d_latent, int d_head,
+                          mlra_stream_t stream);
 
 /* Reads the status word that the last mlra_decode on `workspace` left, after synchronising
  * `stream`.  *flags_host receives the MLRA_FLAG_* bits; the return value is MLRA_OK when no

@@ -451,21 +451,30 @@ mlra_status mlra_read_status(const void* workspace, mlra_stream_t stream, uint32
   return MLRA_OK;
 }
 
-mlra_status mlra_project(const float* o, const void* w_uv, float* y, int N, int H, int d_latent,
+mlra_status mlra_pack_wuv(const void* w_uv, void* w_packed, int H, int d_latent, int d_head,
+                          mlra_stream_t stream) {
+  if (!w_uv || !w_packed || H < 1 || d_latent < 1 || d_head < 1) return MLRA_ERR_INVALID_ARG;
+  if (d_latent % 64 != 0 || d_latent > 512 || d_head % 64 != 0) return MLRA_ERR_UNSUPPORTED;
+  if ((int64_t)H * d_head > INT_MAX) return MLRA_ERR_UNSUPPORTED;
+  if (!aligned16(w_uv) || !aligned16(w_packed)) return MLRA_ERR_UNSUPPORTED;
+  if (launch_pack_wuv(w_uv, w_packed, H, d_latent, d_head, reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return MLRA_ERR_CUDA;
+  return MLRA_OK;
+}
+
+mlra_status mlra_project(const float* o, const void* w_packed, float* y, int N, int H, int d_latent,
                          int d_head, uint32_t* status, mlra_stream_t stream) {
-  if (!o || !w_uv || !y || N < 1 || H < 1 || d_latent < 1 || d_head < 1) return MLRA_ERR_INVALID_ARG;
+  if (!o || !w_packed || !y || N < 1 || H < 1 || d_latent < 1 || d_head < 1) return MLRA_ERR_INVALID_ARG;
   if (d_latent % 64 != 0 || d_latent > 512 || d_head % 64 != 0) return MLRA_ERR_UNSUPPORTED;
   if ((int64_t)H * d_head > INT_MAX || (int64_t)N > 65535 * 64) return MLRA_ERR_UNSUPPORTED;
-  if (!aligned16(o) || !aligned16(w_uv) || !aligned16(y)) return MLRA_ERR_UNSUPPORTED;
-  CUtensorMap tw;
-  const uint64_t dw[2] = {(uint64_t)d_latent, (uint64_t)H * d_head};
-  const uint64_t sw[1] = {(uint64_t)d_latent};
-  if (!make_map(&tw, w_uv, 2, dw, sw)) return MLRA_ERR_CUDA;
+  if (!aligned16(o) || !aligned16(w_packed) || !aligned16(y)) return MLRA_ERR_UNSUPPORTED;
   ProjectParams p;
+  p.w_packed = w_packed;
   p.o = o; p.y = y; p.status = status;
   p.N = N; p.H = H; p.d_latent = d_latent; p.d_head = d_head;
   p.timeout_ns = kTimeoutNs;
-  if (launch_project(tw, p, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MLRA_ERR_CUDA;
+  if (launch_project(p, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MLRA_ERR_CUDA;
   return MLRA_OK;
 }
 

@@ -89,6 +89,7 @@ struct CombineParams {
 
 // Step 3 (K5): y[N, H, d_head] = per head, W_h [d_head, d_latent] times o[N, H, d_latent].
 struct ProjectParams {
+  const void* w_packed;       // W^UV in the packed image of mlra_pack_wuv_kernel
   const float* o;             // branch-mode output of the decode, fp32
   float* y;
   uint32_t* status;           // nullable: kFlagTimeout on a wait that ran out
@@ -118,8 +119,9 @@ cudaError_t launch_decode(Variant v, const CUtensorMap& tq, const CUtensorMap& t
                           cudaStream_t st);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t st);
 cudaError_t launch_repack(const RepackParams& p, cudaStream_t st);
-// tw: bf16 map over W [H * d_head rows, d_latent columns], [64 x 64] boxes, 128-byte swizzle
-cudaError_t launch_project(const CUtensorMap& tw, const ProjectParams& p, cudaStream_t st);
+cudaError_t launch_project(const ProjectParams& p, cudaStream_t st);
+cudaError_t launch_pack_wuv(const void* w, void* packed, int H, int d_latent, int d_head,
+                            cudaStream_t st);
 cudaError_t launch_resolve_rows(const int32_t* lens_or_null, const int32_t* seq_lens,
                                 const int32_t* page_table, int N, int max_pages, int page_size,
                                 int max_seq_len, int64_t n_pages, int oob_row, int64_t* rows_out,

@@ -7,7 +7,7 @@
 //                            the call's status word
 //   K3 mlra_repack_kernel    fp32 / odd-width inputs -> padded bf16 copies in the workspace
 //   K5 mlra_project_kernel   step 3: per-head value up-projection summed over the branches
-//                            (mlra_project_kernel.cuh)
+//                            (mlra_project_kernel.cuh); mlra_pack_wuv_kernel packs its weights
 //   mlra_resolve_rows_kernel test hook for the cache-row addressing of K1
 #include <cuda_bf16.h>
 #include <math_constants.h>
@@ -364,7 +364,14 @@ cudaError_t launch_repack(const RepackParams& p, cudaStream_t st) {
 }
 
 // ----------------------------------------------------------------------------- K5
-cudaError_t launch_project(const CUtensorMap& tw, const ProjectParams& p, cudaStream_t st) {
+cudaError_t launch_pack_wuv(const void* w, void* packed, int H, int d_latent, int d_head,
+                            cudaStream_t st) {
+  mlra_pack_wuv_kernel<<<592, 256, 0, st>>>(static_cast<const uint16_t*>(w),
+                                            static_cast<uint16_t*>(packed), H, d_latent, d_head);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_project(const ProjectParams& p, cudaStream_t st) {
   const int smem = project_smem_bytes(p.d_latent / 64);
   cudaError_t e = cudaFuncSetAttribute(mlra_project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -378,7 +385,7 @@ cudaError_t launch_project(const CUtensorMap& tw, const ProjectParams& p, cudaSt
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, mlra_project_kernel, tw, p);
+  return cudaLaunchKernelEx(&cfg, mlra_project_kernel, p);
 }
 
 // ----------------------------------------------------------------------------- test hook

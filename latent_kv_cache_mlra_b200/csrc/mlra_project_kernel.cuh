@@ -7,7 +7,9 @@
 //     y[s, h, :] = W_h o[s, h, :]
 // One CTA per (head, 64 rows of d_head, 64 sequences): a tcgen05 product with M = 64 rows of W_h,
 // N = the sequences (padded to a multiple of 8), K = d_latent, accumulated in TMEM.
-//   * W_h's rows arrive by TMA as [64 x 64] bf16 boxes (128-byte swizzle, K-major);
+//   * W is packed once (mlra_pack_wuv_kernel) into the product's shared-memory image: per
+//     (head, 64-row tile) d_latent / 64 boxes of [64 rows x 64 columns] bf16 in the 128-byte
+//     swizzled K-major layout, contiguous, so each box arrives with one contiguous bulk copy;
 //   * o (fp32) is rounded to bf16 by all threads into the same swizzled K-major layout;
 //   * one thread issues the d_latent / 16 MMAs; the epilogue reads D with tcgen05.ld and
 //     writes y (a warp's 16 rows of one sequence are 64 contiguous bytes).
@@ -25,6 +27,25 @@ constexpr int kProjThreads = 128;
 constexpr int kProjM = 64;     // rows of W_h per CTA
 constexpr int kProjN = 64;     // sequences per CTA
 constexpr int kProjBox = 8192; // one [64 x 64] bf16 box
+
+// W [H, d_head, d_latent] (row-major) -> the packed image: tile t = h * (d_head / 64) + m, box
+// kb, row r: 16-byte chunk j of columns kb * 64 + 8 j .. + 7 at byte r * 128 + 16 (j ^ (r & 7)).
+__global__ void __launch_bounds__(256) mlra_pack_wuv_kernel(const uint16_t* w, uint16_t* packed,
+                                                            int H, int d_latent, int d_head) {
+  const int KB = d_latent / 64;
+  const int64_t chunks = (int64_t)H * d_head * d_latent / 8;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < chunks;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t box = i >> 9;            // 512 chunks of 16 bytes per 8 KB box
+    const int within = static_cast<int>(i & 511);
+    const int r = within >> 3, jpos = within & 7, j = jpos ^ (r & 7);
+    const int64_t t = box / KB;
+    const int kb = static_cast<int>(box - t * KB);
+    const int64_t row = t * kProjM + r;    // = h * d_head + m * 64 + r
+    const uint4 v = *reinterpret_cast<const uint4*>(w + row * d_latent + kb * 64 + j * 8);
+    *reinterpret_cast<uint4*>(packed + i * 8) = v;
+  }
+}
 
 // shared memory: W boxes, o boxes, an mbarrier per W box and one for the products, the TMEM
 // address
@@ -44,7 +65,7 @@ __device__ __forceinline__ bool project_wait(uint32_t bar, uint32_t parity, uint
 }
 
 __global__ void __launch_bounds__(kProjThreads, 1)
-mlra_project_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ ProjectParams p) {
+mlra_project_kernel(const __grid_constant__ ProjectParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -71,7 +92,6 @@ mlra_project_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
     tmem_alloc(smem_u32(tmem_slot), 64);
     tmem_relinquish();
   }
-  if (warp == 1 && lane == 0) tma_prefetch_desc(&tm_w);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -80,9 +100,11 @@ mlra_project_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
   pdl_wait_prerequisites();
 
   if (warp == 1 && lane == 0) {
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(p.w_packed) +
+                         ((int64_t)h * mtiles + m0 / kProjM) * KB * kProjBox;
     for (int kb = 0; kb < KB; ++kb) {
       mbar_arrive_expect_tx(bar_full + 8 * kb, kProjBox);
-      tma_load_2d(smem_u32(sW + kb * kProjBox), &tm_w, bar_full + 8 * kb, 64 * kb, h * p.d_head + m0);
+      bulk_load(smem_u32(sW + kb * kProjBox), src + kb * kProjBox, kProjBox, bar_full + 8 * kb);
     }
   }
   // o[n0 + r, h, :] -> bf16, box kb holds columns 64 kb .. 64 kb + 63 of row r at 128 r, its

@@ -27,7 +27,8 @@ FLAG_TIMEOUT, FLAG_BAD_PAGE, FLAG_BAD_LENGTH = 0x1, 0x2, 0x4
 EXPORTS = ("mlra_workspace_size", "mlra_decode", "mlra_decode_profiled", "mlra_query_plan",
            "mlra_decode_static_scratch",
            "mlra_read_status", "mlra_debug_resolve_rows", "mlra_plan_host",
-           "mlra_plan_segments_host", "mlra_project", "mlra_status_string", "mlra_version")
+           "mlra_plan_segments_host", "mlra_project", "mlra_pack_wuv", "mlra_status_string",
+           "mlra_version")
 
 
 class Dims(ctypes.Structure):
@@ -84,13 +85,14 @@ def lib() -> ctypes.CDLL:
                                               ctypes.POINTER(ctypes.c_int)]
         L.mlra_project.argtypes = [vp, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                    vp, vp]
+        L.mlra_pack_wuv.argtypes = [vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp]
         L.mlra_status_string.argtypes = [ctypes.c_int]
         L.mlra_status_string.restype = ctypes.c_char_p
         L.mlra_version.argtypes = []
         for f in ("mlra_workspace_size", "mlra_decode", "mlra_decode_profiled", "mlra_query_plan",
                   "mlra_decode_static_scratch",
                   "mlra_read_status", "mlra_debug_resolve_rows", "mlra_plan_host",
-                  "mlra_plan_segments_host", "mlra_project"):
+                  "mlra_plan_segments_host", "mlra_project", "mlra_pack_wuv"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -155,21 +157,36 @@ def dims_for(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table, num_branches, *,
                      num_ranges=num_ranges)
 
 
-def project(o: torch.Tensor, w_uv: torch.Tensor, y: Optional[torch.Tensor] = None, status=None,
+def pack_wuv(w_uv: torch.Tensor, stream=None) -> torch.Tensor:
+    """Packs the step-3 weights (bf16 [H, d_head, d_latent]) for ``project`` through
+    ``mlra_pack_wuv``; the result has the same shape and dtype, packed content."""
+    if w_uv.dtype != torch.bfloat16 or w_uv.dim() != 3 or not w_uv.is_contiguous():
+        raise ValueError("pack_wuv: contiguous bf16 [H, d_head, d_latent] expected")
+    H, d_head, d_latent = w_uv.shape
+    packed = torch.empty_like(w_uv)
+    st = stream if stream is not None else torch.cuda.current_stream(w_uv.device).cuda_stream
+    _check(lib().mlra_pack_wuv(_ptr(w_uv), _ptr(packed), H, d_latent, d_head, ctypes.c_void_p(st)),
+           "mlra_pack_wuv")
+    return packed
+
+
+def project(o: torch.Tensor, w_packed: torch.Tensor, y: Optional[torch.Tensor] = None, status=None,
             stream=None) -> torch.Tensor:
-    """Step 3 through ``mlra_project``: y[s, h] = w_uv[h] @ o[s, h] (o fp32 [N, H, d_latent] from
-    ``decode`` in branch mode, w_uv bf16 [H, d_head, d_latent]); returns y fp32 [N, H, d_head]."""
+    """Step 3 through ``mlra_project``: y[s, h] = W_h @ o[s, h] with o fp32 [N, H, d_latent] from
+    ``decode`` in branch mode and ``w_packed`` from ``pack_wuv`` (shape [H, d_head, d_latent]);
+    returns y fp32 [N, H, d_head]."""
     N, H, d_latent = o.shape
-    d_head = w_uv.shape[1]
-    if o.dtype != torch.float32 or w_uv.dtype != torch.bfloat16 or w_uv.shape != (H, d_head, d_latent):
-        raise ValueError("project: o fp32 [N, H, d_latent], w_uv bf16 [H, d_head, d_latent]")
-    if not (o.is_contiguous() and w_uv.is_contiguous()):
+    d_head = w_packed.shape[1]
+    if (o.dtype != torch.float32 or w_packed.dtype != torch.bfloat16
+            or w_packed.shape != (H, d_head, d_latent)):
+        raise ValueError("project: o fp32 [N, H, d_latent], w_packed bf16 [H, d_head, d_latent]")
+    if not (o.is_contiguous() and w_packed.is_contiguous()):
         raise ValueError("project: contiguous tensors expected")
     if y is None:
         y = torch.empty(N, H, d_head, dtype=torch.float32, device=o.device)
     st = stream if stream is not None else torch.cuda.current_stream(o.device).cuda_stream
-    _check(lib().mlra_project(_ptr(o), _ptr(w_uv), _ptr(y), N, H, d_latent, d_head, _ptr(status),
-                              ctypes.c_void_p(st)), "mlra_project")
+    _check(lib().mlra_project(_ptr(o), _ptr(w_packed), _ptr(y), N, H, d_latent, d_head,
+                              _ptr(status), ctypes.c_void_p(st)), "mlra_project")
     return y
 
 

@@ -31,7 +31,7 @@ def rand_project(N, H, d_latent, d_head, seed):
 ])
 def test_project_matches_oracle(N, H, d_latent, d_head):
     o, w = rand_project(N, H, d_latent, d_head, seed=N + H)
-    y = mlra.project(o.cuda(), w.cuda())
+    y = mlra.project(o.cuda(), mlra.pack_wuv(w.cuda()))
     torch.cuda.synchronize()
     ref_rounded = oracle.project(o.to(torch.bfloat16).float(), w.float())
     yd = y.cpu().double().numpy()
@@ -47,7 +47,7 @@ def test_project_after_decode_matches_oracle():
     w = inp.workload
     g = torch.Generator().manual_seed(5)
     w_uv = (torch.randn(8, 128, w.d_latent, generator=g) / w.d_latent ** 0.5).to(torch.bfloat16)
-    y = mlra.project(out.contiguous(), w_uv.cuda())
+    y = mlra.project(out.contiguous(), mlra.pack_wuv(w_uv.cuda()))
     ref_out, _ = oracle.decode(inp.q_lat, inp.q_rope, inp.c_kv, inp.k_rope, inp.seq_lens, None,
                                w.num_branches, w.sigma, w.gamma, max_seq_len=inp.max_seq_len)
     assert_close(y, oracle.project(ref_out, w_uv.float()), "decode + project")
@@ -67,3 +67,20 @@ def test_project_rejects():
     assert lib.mlra_project(*args) == mlra.MLRA_ERR_UNSUPPORTED        # d_head not a multiple of 64
     args[3] = 0
     assert lib.mlra_project(*args) == mlra.MLRA_ERR_INVALID_ARG
+
+
+def test_pack_wuv_layout():
+    """The packed image puts W[h, m*64 + r, kb*64 + 8j .. +7] at box (h*(d_head/64) + m)*KB + kb,
+    row r, 16-byte chunk j ^ (r % 8) (the 128-byte swizzled K-major tensor-core layout)."""
+    H, d_head, d_latent = 3, 128, 192
+    w = torch.arange(H * d_head * d_latent, dtype=torch.float32).remainder(251).to(torch.bfloat16)
+    w = w.view(H, d_head, d_latent).cuda()
+    packed = mlra.pack_wuv(w).view(-1).cpu()
+    wc = w.cpu()
+    KB, mt = d_latent // 64, d_head // 64
+    for (h, m, kb, r, j) in [(0, 0, 0, 0, 0), (2, 1, 2, 63, 7), (1, 0, 1, 5, 3), (1, 1, 0, 9, 6)]:
+        box = (h * mt + m) * KB + kb
+        pos = j ^ (r % 8)
+        got = packed[box * 4096 + r * 64 + pos * 8: box * 4096 + r * 64 + pos * 8 + 8]
+        want = wc[h, m * 64 + r, kb * 64 + 8 * j: kb * 64 + 8 * j + 8]
+        assert torch.equal(got, want), (h, m, kb, r, j)

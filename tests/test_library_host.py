@@ -268,3 +268,12 @@ def test_project_argument_errors_without_a_gpu():
         args = list(ok)
         args[i] = v
         assert lib.mlra_project(*args) == want, (i, v)
+
+
+def test_pack_wuv_argument_errors_without_a_gpu():
+    lib = mlra.lib()
+    fake = ctypes.c_void_p(4096)
+    assert lib.mlra_pack_wuv(None, fake, 2, 512, 128, None) == mlra.MLRA_ERR_INVALID_ARG
+    assert lib.mlra_pack_wuv(fake, fake, 2, 96, 128, None) == mlra.MLRA_ERR_UNSUPPORTED
+    assert lib.mlra_pack_wuv(fake, fake, 2, 512, 100, None) == mlra.MLRA_ERR_UNSUPPORTED
+    assert lib.mlra_pack_wuv(ctypes.c_void_p(4100), fake, 2, 512, 128, None) == mlra.MLRA_ERR_UNSUPPORTED
