@@ -8,7 +8,9 @@ What it computes (sources: "Multi-Head Low-Rank Attention", yunpan.plus page):
   * section 1.3, steps 1-3 of MLA's efficient decode: the absorbed query
     ``q~`` is dotted with the cached latent vectors directly, as MQA-style
     attention with the latent as the shared key/value, and the value
-    up-projection comes afterwards (step 3: ``project`` below);
+    up-projection comes afterwards (step 3: ``project`` below; step 1, the
+    absorption, and the decoupled RoPE with the cache append: ``absorb``,
+    ``rope`` and ``append_token`` below);
   * section 2: the per-head NoPE key is a sum of B block projections of the
     latent, so splitting ``c_t`` into B column blocks ``c_{t,b}`` is exact;
   * section 3 / 3.1 (MLRA-4): the block sum moves behind the attention; each
@@ -167,3 +169,55 @@ def project(out, w_uv):
         y[s, h] = sum_b W^UV_{h,b} out[s, h, b-block] = w_uv[h] @ out[s, h]      -> [N, H, d_h]
     """
     return np.einsum("hkd,shd->shk", to_f64(w_uv), to_f64(out))
+
+
+def absorb(q_nope, w_uk):
+    """Step 1 of the absorbed decode (section 1.3): the query absorbs the key up-projections.
+
+    q_nope [N, H, d_head]: each head's query before the keys' up-projection.  w_uk
+    [H, d_head, d_c]: head h's key up-projections side by side, W^UK_{h,b} = w_uk[h, :, b-block],
+    so that head h's key for branch b is W^UK_{h,b} c_b (section 2).  Then
+        q_lat[s, h, b-block] = (W^UK_{h,b})^T q_nope[s, h]      -> [N, H, d_c]
+    and q_lat[s, h, b-block] . c_b equals the head's query dotted with its branch-b key.
+    """
+    return np.einsum("hkd,shk->shd", to_f64(w_uk), to_f64(q_nope))
+
+
+def rope(x, positions, base=10000.0):
+    """Rotary position embedding of the decoupled RoPE vectors (the page's section on DeepSeek's
+    decoupled RoPE; the rotation itself is the standard one, the pages give no variant).
+
+    x [..., d] with d even; positions broadcast against x[..., 0].  Pair (2i, 2i+1) of a vector at
+    position p is rotated by the angle p * base^(-2i/d):
+        y[2i]   = x[2i] cos(a) - x[2i+1] sin(a)
+        y[2i+1] = x[2i] sin(a) + x[2i+1] cos(a)
+    """
+    x = to_f64(x)
+    d = x.shape[-1]
+    i = np.arange(d // 2, dtype=np.float64)
+    theta = base ** (-2.0 * i / d)
+    a = np.asarray(positions, dtype=np.float64)[..., None] * theta
+    c, s_ = np.cos(a), np.sin(a)
+    x0, x1 = x[..., 0::2], x[..., 1::2]
+    y = np.empty_like(x)
+    y[..., 0::2] = x0 * c - x1 * s_
+    y[..., 1::2] = x0 * s_ + x1 * c
+    return y
+
+
+def append_token(c_kv, k_rope, seq_lens, page_table, page_size, max_seq_len, c_new, kr_new):
+    """The new token of every sequence goes into the cache at position p = seq_lens[s] (its
+    row by the same addressing as the decode: page table or contiguous), latent c_new[s] and
+    RoPE key kr_new[s] (already rotated).  Returns updated copies of (c_kv, k_rope) and the new
+    lengths."""
+    c_kv, k_rope = to_f64(c_kv).copy(), to_f64(k_rope).copy()
+    lens = np.asarray(seq_lens.tolist() if hasattr(seq_lens, "tolist") else seq_lens, dtype=np.int64)
+    pt = None if page_table is None else np.asarray(
+        page_table.tolist() if hasattr(page_table, "tolist") else page_table, dtype=np.int64)
+    c_new, kr_new = to_f64(c_new), to_f64(kr_new)
+    for s in range(len(lens)):
+        p = int(lens[s])
+        row = int(resolve_rows(p + 1, s, pt, page_size, max_seq_len)[p])
+        c_kv[row, :c_new.shape[1]] = c_new[s]
+        k_rope[row, :kr_new.shape[1]] = kr_new[s]
+    return c_kv, k_rope, lens + 1

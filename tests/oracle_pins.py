@@ -326,7 +326,77 @@ def pin_project_brute_force(orc, seed=9, N=2, H=3, B=2, d_blk=4, d_h=3):
     assert np.allclose(y_eye, out.reshape(N, H, B, d_blk).sum(axis=2), rtol=0, atol=1e-12), "identity"
 
 
+def pin_absorb_equals_explicit(orc, seed=10, H=4, B=4, d_blk=8, d_R=4, d_h=6, L=23):
+    """Step 1 (``absorb``: one query per head, W^UK of every branch side by side) -> step 2 ->
+    step 3 == explicit attention whose branch-b keys are W^UK_{h,b} c_b (sections 1.3, 2, 3)."""
+    rng = np.random.default_rng(seed)
+    W_uk, W_uv = _rand(rng, H, B, d_h, d_blk), _rand(rng, H, B, d_h, d_blk)
+    q_head, q_rope = _rand(rng, H, d_h), _rand(rng, H, d_R)
+    c, kr = _rand(rng, L, B * d_blk), _rand(rng, L, d_R)
+    sigma, gamma = 0.29, 1.0 / B
+    ref = explicit_mlra(np.repeat(q_head[:, None], B, axis=1), q_rope, c, kr, W_uk, W_uv, sigma, gamma)
+    w_uk = np.concatenate([W_uk[:, b] for b in range(B)], axis=2)    # [H, d_h, d_c]
+    q_lat = orc.absorb(q_head[None], w_uk)[0]                         # step 1
+    out, _ = _one_seq(orc, q_lat, q_rope, c, kr, B, sigma, gamma)
+    y = orc.project(out[None], np.concatenate([W_uv[:, b] for b in range(B)], axis=2))[0]
+    err = np.abs(y - ref).max() / np.abs(ref).max()
+    assert err <= 1e-12, f"absorb -> decode -> project vs explicit rel err {err:.3e}"
+
+
+def pin_rope(orc, seed=11):
+    """RoPE: the identity at position 0, a rotation (norms kept), scores that depend on the
+    relative position only, the closed forms of the first two pairs, and 2x2 rotations by loops."""
+    rng = np.random.default_rng(seed)
+    d, base = 8, 10000.0
+    x = _rand(rng, 5, d)
+    assert np.allclose(orc.rope(x, np.zeros(5), base), x, rtol=0, atol=1e-15), "position 0"
+    pos = rng.integers(0, 100000, size=5).astype(np.float64)
+    y = orc.rope(x, pos, base)
+    assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-12), "norm"
+    q, k = _rand(rng, d), _rand(rng, d)
+    for m, n in [(7, 3), (1000, 12), (54321, 54300)]:
+        lhs = orc.rope(q[None], [m], base)[0] @ orc.rope(k[None], [n], base)[0]
+        rhs = orc.rope(q[None], [m - n], base)[0] @ k
+        assert abs(lhs - rhs) <= 1e-9 * (1 + abs(rhs)), "relative position"
+    for p_ in (0.5, 2.0, 31.0):
+        e0 = orc.rope(np.array([[1.0, 0.0, 0.0, 1.0]]), [p_], base)[0]
+        a1 = p_ * base ** -0.5
+        want = [math.cos(p_), math.sin(p_), -math.sin(a1), math.cos(a1)]
+        assert np.allclose(e0, want, rtol=0, atol=1e-13), "closed form"
+    for r in range(5):
+        for i in range(d // 2):
+            a = pos[r] * base ** (-2.0 * i / d)
+            rot = [x[r, 2 * i] * math.cos(a) - x[r, 2 * i + 1] * math.sin(a),
+                   x[r, 2 * i] * math.sin(a) + x[r, 2 * i + 1] * math.cos(a)]
+            assert abs(y[r, 2 * i] - rot[0]) + abs(y[r, 2 * i + 1] - rot[1]) <= 1e-9, "loops"
+
+
+def pin_append_token(orc, seed=12):
+    """The new token lands at position seq_lens[s] (the decode's row addressing), nothing else
+    changes, and the decode then sees exactly one more position."""
+    rng = np.random.default_rng(seed)
+    N, d_c, d_R, P = 3, 8, 4, 64
+    lens = np.array([5, 64, 0])
+    pt = np.array([[3, 1], [0, 2], [4, 5]])                # pages of 64 rows
+    rows = 6 * P
+    c_kv, k_rope = _rand(rng, rows, d_c), _rand(rng, rows, d_R)
+    c_new, kr_new = _rand(rng, N, d_c), _rand(rng, N, d_R)
+    c2, k2, lens2 = orc.append_token(c_kv, k_rope, lens, pt, P, 0, c_new, kr_new)
+    assert list(lens2) == [6, 65, 1]
+    want_rows = [3 * P + 5, 2 * P + 0, 4 * P + 0]
+    changed = sorted(set(np.nonzero((c2 != c_kv).any(1))[0]) | set(np.nonzero((k2 != k_rope).any(1))[0]))
+    assert changed == sorted(want_rows), (changed, want_rows)
+    for s_, r in enumerate(want_rows):
+        assert np.array_equal(c2[r], c_new[s_]) and np.array_equal(k2[r], kr_new[s_])
+    # contiguous layout: row s * max_seq_len + L
+    c3, _, _ = orc.append_token(c_kv, k_rope, [2, 0, 7], None, 0, 10, c_new, kr_new)
+    assert [r for r in range(rows) if (c3[r] != c_kv[r]).any()] == [2, 10, 27]
+
+
 ALL_PINS = [
+    pin_absorb_equals_explicit,
+    pin_rope,
+    pin_append_token,
     pin_project_brute_force,
     pin_absorbed_equals_explicit,
     pin_summed_equals_explicit_shared_wuv,

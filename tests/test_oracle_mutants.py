@@ -37,6 +37,12 @@ MUTANTS = {
                                   'np.einsum("hkd,shk->shd", to_f64(w_uv), to_f64(out)[..., :w_uv.shape[1]])'),
     "project_first_branch_only": ('np.einsum("hkd,shd->shk", to_f64(w_uv), to_f64(out))',
                                   'np.einsum("hkd,shd->shk", to_f64(w_uv)[..., :8], to_f64(out)[..., :8])'),
+    "absorb_transposed": ('np.einsum("hkd,shk->shd", to_f64(w_uk), to_f64(q_nope))',
+                          'np.einsum("hkd,shd->shk", to_f64(w_uk), to_f64(q_nope)[..., :w_uk.shape[2]])'),
+    "rope_sin_sign": ("y[..., 0::2] = x0 * c - x1 * s_", "y[..., 0::2] = x0 * c + x1 * s_"),
+    "rope_pairs_halves": ("x0, x1 = x[..., 0::2], x[..., 1::2]", "x0, x1 = x[..., : d // 2], x[..., d // 2:]"),
+    "rope_frequency_exponent": ("theta = base ** (-2.0 * i / d)", "theta = base ** (-1.0 * i / d)"),
+    "append_off_by_one": ("        p = int(lens[s])\n", "        p = max(int(lens[s]) - 1, 0)\n"),
     "project_head_shift": ('np.einsum("hkd,shd->shk", to_f64(w_uv), to_f64(out))',
                            'np.einsum("hkd,shd->shk", np.roll(to_f64(w_uv), 1, axis=0), to_f64(out))'),
 }
