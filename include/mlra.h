@@ -203,6 +203,49 @@ mlra_status mlra_project(const float* o, const void* w_packed, float* y, int N, 
 mlra_status mlra_pack_wuv(const void* w_uv, void* w_packed, int H, int d_latent, int d_head,
                           mlra_stream_t stream);
 
+/* Step 1 of the absorbed decode: each head's query absorbs the key up-projections of the B
+ * branches ("Multi-Head Low-Rank Attention", yunpan.plus page, section 1.3 step 1; the block form
+ * of section 2): q_lat[s, h, b-block] = (W^UK_{h,b})^T q_nope[s, h].
+ *   q_nope   [N, H, d_head] fp32 device
+ *   w_packed H * d_head * d_latent bf16 device, written by mlra_pack_wuk
+ *   q_lat    [N, H, d_latent] bf16 device (written): mlra_decode's q_lat
+ *   status   nullable device uint32: MLRA_FLAG_TIMEOUT if a bounded wait runs out
+ * Products in bf16 (q_nope rounded) with fp32 accumulation, the result rounded to bf16.
+ * Errors: MLRA_ERR_INVALID_ARG for null pointers or sizes < 1; MLRA_ERR_UNSUPPORTED unless d_head
+ * is a multiple of 64 up to 512, d_latent a multiple of 64 and the arrays 16-byte aligned. */
+mlra_status mlra_absorb(const float* q_nope, const void* w_packed, void* q_lat, int N, int H,
+                        int d_head, int d_latent, uint32_t* status, mlra_stream_t stream);
+
+/* Packs the step-1 weights once for mlra_absorb (model weights: pack at load time).
+ *   w_uk     [H, d_head, d_latent] bf16 device, row-major: head h's key up-projections side by
+ *            side, W^UK_{h,b} = w_uk[h, :, b*d_blk : (b+1)*d_blk]
+ *   w_packed H * d_head * d_latent bf16 device (written): the transposes, in the tensor-core image
+ * Errors as mlra_absorb. */
+mlra_status mlra_pack_wuk(const void* w_uk, void* w_packed, int H, int d_head, int d_latent,
+                          mlra_stream_t stream);
+
+/* The new token of every sequence, before step 2: rotary position embedding of its RoPE query
+ * (one per head) and of its RoPE key (shared by all heads and branches), and the append of its
+ * latent and key to the cache.  The pages describe DeepSeek's decoupled RoPE without the rotation's
+ * details; the rotation is the standard one: pair (2i, 2i+1) of a vector at position p turns by
+ * p * rope_base^(-2i / d_rope).  The token's position is p = seq_lens[s] and its cache row follows
+ * mlra_decode's addressing (page table, or s * max_seq_len + p); the caller then passes
+ * seq_lens + 1 to mlra_decode.
+ *   q_rope_in  [N, H, d_rope] fp32 device     kr_new [N, d_rope] fp32     c_new [N, d_latent] fp32
+ *   seq_lens   [N] int32 device; page_table as for mlra_decode (NULL: contiguous)
+ *   dims       the cache geometry as for mlra_decode (bf16 cache; batch, heads, d_latent, d_rope,
+ *              page_size / max_pages_per_seq or max_seq_len, cache_rows, row strides)
+ *   c_kv, k_rope  the bf16 caches (row `row` written)
+ *   q_rope_out [N, H, d_rope] bf16 device (written): mlra_decode's q_rope
+ *   status     nullable device uint32: MLRA_FLAG_BAD_LENGTH (position outside the sequence's
+ *              cache space) or MLRA_FLAG_BAD_PAGE (invalid page id); that append is skipped
+ * Errors: MLRA_ERR_INVALID_ARG for null pointers, a non-positive base or invalid dims;
+ * MLRA_ERR_UNSUPPORTED for an fp32 cache or an odd d_rope. */
+mlra_status mlra_rope_append(const float* q_rope_in, const float* kr_new, const float* c_new,
+                             const int32_t* seq_lens, const int32_t* page_table,
+                             const mlra_dims* dims, void* c_kv, void* k_rope, void* q_rope_out,
+                             double rope_base, uint32_t* status, mlra_stream_t stream);
+
 /* Reads the status word that the last mlra_decode on `workspace` left, after synchronising
  * `stream`.  *flags_host receives the MLRA_FLAG_* bits; the return value is MLRA_OK when no
  * bit is set, else the status of the most serious bit (timeout, bad page, bad length). */

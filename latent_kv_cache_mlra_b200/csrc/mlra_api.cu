@@ -451,30 +451,91 @@ mlra_status mlra_read_status(const void* workspace, mlra_stream_t stream, uint32
   return MLRA_OK;
 }
 
-mlra_status mlra_pack_wuv(const void* w_uv, void* w_packed, int H, int d_latent, int d_head,
-                          mlra_stream_t stream) {
-  if (!w_uv || !w_packed || H < 1 || d_latent < 1 || d_head < 1) return MLRA_ERR_INVALID_ARG;
-  if (d_latent % 64 != 0 || d_latent > 512 || d_head % 64 != 0) return MLRA_ERR_UNSUPPORTED;
-  if ((int64_t)H * d_head > INT_MAX) return MLRA_ERR_UNSUPPORTED;
-  if (!aligned16(w_uv) || !aligned16(w_packed)) return MLRA_ERR_UNSUPPORTED;
-  if (launch_pack_wuv(w_uv, w_packed, H, d_latent, d_head, reinterpret_cast<cudaStream_t>(stream)) !=
+namespace {
+// Shared checks of the per-head products: widths in 64-column boxes, at most 512 input columns,
+// 16-byte aligned arrays.
+mlra_status check_product(const void* a, const void* b, const void* c, int N, int H, int d_in,
+                          int d_out) {
+  if (!a || !b || !c || N < 1 || H < 1 || d_in < 1 || d_out < 1) return MLRA_ERR_INVALID_ARG;
+  if (d_in % 64 != 0 || d_in > 512 || d_out % 64 != 0) return MLRA_ERR_UNSUPPORTED;
+  if ((int64_t)H * d_out > INT_MAX || (int64_t)N > 65535 * 64) return MLRA_ERR_UNSUPPORTED;
+  if (!aligned16(a) || !aligned16(b) || !aligned16(c)) return MLRA_ERR_UNSUPPORTED;
+  return MLRA_OK;
+}
+
+mlra_status run_product(const float* x, const void* w_packed, void* y, int N, int H, int d_in,
+                        int d_out, bool out_bf16, uint32_t* status, mlra_stream_t stream) {
+  const mlra_status st = check_product(x, w_packed, y, N, H, d_in, d_out);
+  if (st != MLRA_OK) return st;
+  ProjectParams p;
+  p.w_packed = w_packed;
+  p.x = x; p.y = y; p.status = status;
+  p.N = N; p.H = H; p.d_in = d_in; p.d_out = d_out;
+  p.out_bf16 = out_bf16 ? 1 : 0;
+  p.timeout_ns = kTimeoutNs;
+  if (launch_project(p, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MLRA_ERR_CUDA;
+  return MLRA_OK;
+}
+
+mlra_status run_pack(const void* w, void* packed, int H, int d_in, int d_out, bool transpose,
+                     mlra_stream_t stream) {
+  const mlra_status st = check_product(w, packed, packed, 1, H, d_in, d_out);
+  if (st != MLRA_OK) return st;
+  if (launch_pack(w, packed, H, d_in, d_out, transpose, reinterpret_cast<cudaStream_t>(stream)) !=
       cudaSuccess)
     return MLRA_ERR_CUDA;
   return MLRA_OK;
 }
+}  // namespace
+
+mlra_status mlra_pack_wuv(const void* w_uv, void* w_packed, int H, int d_latent, int d_head,
+                          mlra_stream_t stream) {
+  return run_pack(w_uv, w_packed, H, d_latent, d_head, false, stream);
+}
 
 mlra_status mlra_project(const float* o, const void* w_packed, float* y, int N, int H, int d_latent,
                          int d_head, uint32_t* status, mlra_stream_t stream) {
-  if (!o || !w_packed || !y || N < 1 || H < 1 || d_latent < 1 || d_head < 1) return MLRA_ERR_INVALID_ARG;
-  if (d_latent % 64 != 0 || d_latent > 512 || d_head % 64 != 0) return MLRA_ERR_UNSUPPORTED;
-  if ((int64_t)H * d_head > INT_MAX || (int64_t)N > 65535 * 64) return MLRA_ERR_UNSUPPORTED;
-  if (!aligned16(o) || !aligned16(w_packed) || !aligned16(y)) return MLRA_ERR_UNSUPPORTED;
-  ProjectParams p;
-  p.w_packed = w_packed;
-  p.o = o; p.y = y; p.status = status;
-  p.N = N; p.H = H; p.d_latent = d_latent; p.d_head = d_head;
-  p.timeout_ns = kTimeoutNs;
-  if (launch_project(p, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MLRA_ERR_CUDA;
+  return run_product(o, w_packed, y, N, H, d_latent, d_head, false, status, stream);
+}
+
+mlra_status mlra_pack_wuk(const void* w_uk, void* w_packed, int H, int d_head, int d_latent,
+                          mlra_stream_t stream) {
+  return run_pack(w_uk, w_packed, H, d_head, d_latent, true, stream);
+}
+
+mlra_status mlra_absorb(const float* q_nope, const void* w_packed, void* q_lat, int N, int H,
+                        int d_head, int d_latent, uint32_t* status, mlra_stream_t stream) {
+  return run_product(q_nope, w_packed, q_lat, N, H, d_head, d_latent, true, status, stream);
+}
+
+mlra_status mlra_rope_append(const float* q_rope_in, const float* kr_new, const float* c_new,
+                             const int32_t* seq_lens, const int32_t* page_table,
+                             const mlra_dims* dims, void* c_kv, void* k_rope, void* q_rope_out,
+                             double rope_base, uint32_t* status, mlra_stream_t stream) {
+  if (!q_rope_in || !kr_new || !c_new || !seq_lens || !dims || !c_kv || !k_rope || !q_rope_out)
+    return MLRA_ERR_INVALID_ARG;
+  if (!(rope_base > 0.0) || !std::isfinite(rope_base)) return MLRA_ERR_INVALID_ARG;
+  const bool paged = page_table != nullptr;
+  const mlra_status st = check_dims(dims, paged);
+  if (st != MLRA_OK) return st;
+  if (dims->dtype != MLRA_BF16 || dims->d_rope % 2 != 0) return MLRA_ERR_UNSUPPORTED;
+  RopeAppendParams p;
+  p.q_rope_in = q_rope_in; p.kr_new = kr_new; p.c_new = c_new;
+  p.seq_lens = seq_lens; p.page_table = page_table;
+  p.max_pages = paged ? dims->max_pages_per_seq : 0;
+  p.page_size = paged ? dims->page_size : 0;
+  p.max_seq_len = dims->max_seq_len;
+  p.n_pages = paged ? dims->cache_rows / dims->page_size : 0;
+  p.c_kv = static_cast<uint16_t*>(c_kv);
+  p.k_rope = static_cast<uint16_t*>(k_rope);
+  p.c_row_stride = dims->c_row_stride;
+  p.kr_row_stride = dims->kr_row_stride;
+  p.q_rope_out = static_cast<uint16_t*>(q_rope_out);
+  p.N = dims->batch; p.H = dims->heads; p.d_rope = dims->d_rope; p.d_latent = dims->d_latent;
+  p.base = rope_base;
+  p.status = status;
+  if (launch_rope_append(p, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MLRA_ERR_CUDA;
   return MLRA_OK;
 }
 

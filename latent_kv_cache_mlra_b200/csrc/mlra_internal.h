@@ -87,14 +87,33 @@ struct CombineParams {
   float gamma;
 };
 
-// Step 3 (K5): y[N, H, d_head] = per head, W_h [d_head, d_latent] times o[N, H, d_latent].
+// Per-head products (K5), steps 1 and 3: out[N, H, d_out] = A_h x[N, H, d_in] per head h.
 struct ProjectParams {
-  const void* w_packed;       // W^UV in the packed image of mlra_pack_wuv_kernel
-  const float* o;             // branch-mode output of the decode, fp32
-  float* y;
+  const void* w_packed;       // A in the packed image of mlra_pack_kernel
+  const float* x;             // [N, H, d_in] fp32
+  void* y;                    // [N, H, d_out], fp32 or bf16
   uint32_t* status;           // nullable: kFlagTimeout on a wait that ran out
-  int N, H, d_latent, d_head;
+  int N, H, d_in, d_out;
+  int out_bf16;
   uint64_t timeout_ns;
+};
+
+// RoPE of the new token's query and key, and its append to the cache (K7).
+struct RopeAppendParams {
+  const float* q_rope_in;     // [N, H, d_rope] before rotation
+  const float* kr_new;        // [N, d_rope] before rotation
+  const float* c_new;         // [N, d_latent]
+  const int32_t* seq_lens;    // [N]: the new token's position
+  const int32_t* page_table;  // [N, max_pages] or nullptr (contiguous)
+  int max_pages, page_size, max_seq_len;
+  int64_t n_pages;
+  uint16_t* c_kv;             // bf16 cache rows, pitch c_row_stride
+  uint16_t* k_rope;           // bf16 cache rows, pitch kr_row_stride
+  int64_t c_row_stride, kr_row_stride;
+  uint16_t* q_rope_out;       // [N, H, d_rope] bf16
+  int N, H, d_rope, d_latent;
+  double base;                // RoPE base
+  uint32_t* status;           // nullable: kFlagBadPage / kFlagBadLength for a skipped append
 };
 
 struct RepackParams {
@@ -120,8 +139,9 @@ cudaError_t launch_decode(Variant v, const CUtensorMap& tq, const CUtensorMap& t
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t st);
 cudaError_t launch_repack(const RepackParams& p, cudaStream_t st);
 cudaError_t launch_project(const ProjectParams& p, cudaStream_t st);
-cudaError_t launch_pack_wuv(const void* w, void* packed, int H, int d_latent, int d_head,
-                            cudaStream_t st);
+cudaError_t launch_pack(const void* w, void* packed, int H, int d_in, int d_out, bool transpose,
+                        cudaStream_t st);
+cudaError_t launch_rope_append(const RopeAppendParams& p, cudaStream_t st);
 cudaError_t launch_resolve_rows(const int32_t* lens_or_null, const int32_t* seq_lens,
                                 const int32_t* page_table, int N, int max_pages, int page_size,
                                 int max_seq_len, int64_t n_pages, int oob_row, int64_t* rows_out,

@@ -6,8 +6,10 @@
 //   K2 mlra_combine_kernel   merges the partial softmax states of split sequences and writes
 //                            the call's status word
 //   K3 mlra_repack_kernel    fp32 / odd-width inputs -> padded bf16 copies in the workspace
-//   K5 mlra_project_kernel   step 3: per-head value up-projection summed over the branches
-//                            (mlra_project_kernel.cuh); mlra_pack_wuv_kernel packs its weights
+//   K5 mlra_project_kernel   per-head products: step 1 (query absorption) and step 3 (value
+//                            up-projection summed over the branches); mlra_pack_kernel packs
+//                            their weights (mlra_project_kernel.cuh)
+//   K7 mlra_rope_append_kernel  RoPE of the new token's query and key, cache append
 //   mlra_resolve_rows_kernel test hook for the cache-row addressing of K1
 #include <cuda_bf16.h>
 #include <math_constants.h>
@@ -364,19 +366,20 @@ cudaError_t launch_repack(const RepackParams& p, cudaStream_t st) {
 }
 
 // ----------------------------------------------------------------------------- K5
-cudaError_t launch_pack_wuv(const void* w, void* packed, int H, int d_latent, int d_head,
-                            cudaStream_t st) {
-  mlra_pack_wuv_kernel<<<592, 256, 0, st>>>(static_cast<const uint16_t*>(w),
-                                            static_cast<uint16_t*>(packed), H, d_latent, d_head);
+cudaError_t launch_pack(const void* w, void* packed, int H, int d_in, int d_out, bool transpose,
+                        cudaStream_t st) {
+  mlra_pack_kernel<<<592, 256, 0, st>>>(static_cast<const uint16_t*>(w),
+                                        static_cast<uint16_t*>(packed), H, d_in, d_out,
+                                        transpose ? 1 : 0);
   return cudaGetLastError();
 }
 
 cudaError_t launch_project(const ProjectParams& p, cudaStream_t st) {
-  const int smem = project_smem_bytes(p.d_latent / 64);
+  const int smem = project_smem_bytes(p.d_in / 64);
   cudaError_t e = cudaFuncSetAttribute(mlra_project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.H * (p.d_head / kProjM), (p.N + kProjN - 1) / kProjN);
+  cfg.gridDim = dim3(p.H * (p.d_out / kProjM), (p.N + kProjN - 1) / kProjN);
   cfg.blockDim = dim3(kProjThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -386,6 +389,74 @@ cudaError_t launch_project(const ProjectParams& p, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, mlra_project_kernel, p);
+}
+
+// ----------------------------------------------------------------------------- K7
+// One block per sequence.  The new token sits at position p = seq_lens[s]: its row follows the
+// decode's addressing (page table, or s * max_seq_len + p).  Pair (2i, 2i+1) of the head queries
+// and of the key is rotated by the angle p * base^(-2i/d_rope) (angle in double precision: p
+// reaches 10^5 and more), the rotated query is written in bf16 for the decode, and the rotated
+// key and the latent c_new are written in bf16 to the cache row.  A position past the cache or an
+// invalid page id flags the status word and skips the append (the query is still rotated).
+__global__ void __launch_bounds__(256) mlra_rope_append_kernel(const RopeAppendParams p) {
+  const int s = blockIdx.x;
+  pdl_wait_prerequisites();  // the inputs come from the previous kernels on the stream
+  const int pos = p.seq_lens[s];
+  int64_t row = -1;
+  uint32_t bad = 0;
+  if (pos < 0) {
+    bad = kFlagBadLength;
+  } else if (p.page_table != nullptr) {
+    const int page = pos / p.page_size;
+    if (page >= p.max_pages) {
+      bad = kFlagBadLength;
+    } else {
+      const int pid = p.page_table[(int64_t)s * p.max_pages + page];
+      if (pid < 0 || pid >= p.n_pages) bad = kFlagBadPage;
+      else row = (int64_t)pid * p.page_size + pos % p.page_size;
+    }
+  } else {
+    if (pos >= p.max_seq_len) bad = kFlagBadLength;
+    else row = (int64_t)s * p.max_seq_len + pos;
+  }
+  if (bad && threadIdx.x == 0 && p.status) atomicOr(p.status, bad);
+  const double pd = pos > 0 ? (double)pos : 0.0;
+  const int half = p.d_rope / 2;
+  for (int t = threadIdx.x; t < (p.H + 1) * half; t += blockDim.x) {
+    const int v = t / half, i = t - v * half;
+    double sn, cs;
+    sincos(pd * pow(p.base, -2.0 * i / p.d_rope), &sn, &cs);
+    const float c = static_cast<float>(cs), sf = static_cast<float>(sn);
+    const float* src = v < p.H ? p.q_rope_in + ((int64_t)s * p.H + v) * p.d_rope
+                               : p.kr_new + (int64_t)s * p.d_rope;
+    const float x0 = src[2 * i], x1 = src[2 * i + 1];
+    const uint16_t y0 = __bfloat16_as_ushort(__float2bfloat16_rn(x0 * c - x1 * sf));
+    const uint16_t y1 = __bfloat16_as_ushort(__float2bfloat16_rn(x0 * sf + x1 * c));
+    uint16_t* dst = nullptr;
+    if (v < p.H) dst = p.q_rope_out + ((int64_t)s * p.H + v) * p.d_rope + 2 * i;
+    else if (row >= 0) dst = p.k_rope + row * p.kr_row_stride + 2 * i;
+    if (dst) {
+      dst[0] = y0;
+      dst[1] = y1;
+    }
+  }
+  if (row >= 0)
+    for (int j = threadIdx.x; j < p.d_latent; j += blockDim.x)
+      p.c_kv[row * p.c_row_stride + j] =
+          __bfloat16_as_ushort(__float2bfloat16_rn(p.c_new[(int64_t)s * p.d_latent + j]));
+}
+
+cudaError_t launch_rope_append(const RopeAppendParams& p, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.N);
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, mlra_rope_append_kernel, p);
 }
 
 // ----------------------------------------------------------------------------- test hook

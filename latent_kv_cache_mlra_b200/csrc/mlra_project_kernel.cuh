@@ -1,22 +1,27 @@
-// mlra_project_kernel.cuh -- K5: step 3 of the absorbed decode on sm_100a.
+// mlra_project_kernel.cuh -- K5: the per-head products of steps 1 and 3 of the absorbed decode.
 //
-// "Multi-Head Low-Rank Attention" (yunpan.plus page), section 1.3 step 3 with the branch sum of
-// sections 3 and 3.3: the value up-projection of every branch output, summed over the branches.
-// With head h's projections side by side, W_h = [W^UV_{h,1} | ... | W^UV_{h,B}] (d_head x d_latent),
-// and o[s, h] the concatenated branch outputs of step 2 (gamma already applied):
-//     y[s, h, :] = W_h o[s, h, :]
-// One CTA per (head, 64 rows of d_head, 64 sequences): a tcgen05 product with M = 64 rows of W_h,
-// N = the sequences (padded to a multiple of 8), K = d_latent, accumulated in TMEM.
-//   * W is packed once (mlra_pack_wuv_kernel) into the product's shared-memory image: per
-//     (head, 64-row tile) d_latent / 64 boxes of [64 rows x 64 columns] bf16 in the 128-byte
+// "Multi-Head Low-Rank Attention" (yunpan.plus page), section 1.3:
+//   step 3 with the branch sum of sections 3 and 3.3 -- the value up-projection of every branch
+//     output, summed over the branches.  With head h's projections side by side,
+//     W_h = [W^UV_{h,1} | ... | W^UV_{h,B}] (d_head x d_latent), and o[s, h] the concatenated branch
+//     outputs of step 2 (gamma applied):  y[s, h, :] = W_h o[s, h, :];
+//   step 1 -- the absorbed query q~[s, h, b-block] = (W^UK_{h,b})^T q[s, h], i.e. the product with
+//     the transpose of [W^UK_{h,1} | ... | W^UK_{h,B}] (d_head x d_latent).
+// Both are x_out[s, h, :] = A_h x_in[s, h, :] with A_h of d_out x d_in.
+// One CTA per (head, 64 rows of A_h, 64 sequences): a tcgen05 product with M = 64 rows of A_h,
+// N = the sequences (padded to a multiple of 8), K = d_in, accumulated in TMEM.
+//   * A is packed once (mlra_pack_kernel, at model load) into the product's shared-memory image:
+//     per (head, 64-row tile) d_in / 64 boxes of [64 rows x 64 columns] bf16 in the 128-byte
 //     swizzled K-major layout, contiguous, so each box arrives with one contiguous bulk copy;
-//   * o (fp32) is rounded to bf16 by all threads into the same swizzled K-major layout;
-//   * one thread issues the d_latent / 16 MMAs; the epilogue reads D with tcgen05.ld and
-//     writes y (a warp's 16 rows of one sequence are 64 contiguous bytes).
-// The work is bound by streaming W (H d_head d_latent bf16) from HBM.
+//   * x_in (fp32) is rounded to bf16 by all threads into the same swizzled K-major layout;
+//   * one thread issues the d_in / 16 MMAs; the epilogue reads D with tcgen05.ld and writes
+//     x_out in fp32 or bf16 (a warp's 16 rows of one sequence are contiguous).
+// The work is bound by streaming A (H d_out d_in bf16) from HBM.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
+
+#include <cuda_bf16.h>
 
 #include "mlra_internal.h"
 #include "sm100_ptx.cuh"
@@ -24,16 +29,18 @@
 namespace mlra {
 
 constexpr int kProjThreads = 128;
-constexpr int kProjM = 64;     // rows of W_h per CTA
+constexpr int kProjM = 64;     // rows of A_h per CTA
 constexpr int kProjN = 64;     // sequences per CTA
 constexpr int kProjBox = 8192; // one [64 x 64] bf16 box
 
-// W [H, d_head, d_latent] (row-major) -> the packed image: tile t = h * (d_head / 64) + m, box
-// kb, row r: 16-byte chunk j of columns kb * 64 + 8 j .. + 7 at byte r * 128 + 16 (j ^ (r & 7)).
-__global__ void __launch_bounds__(256) mlra_pack_wuv_kernel(const uint16_t* w, uint16_t* packed,
-                                                            int H, int d_latent, int d_head) {
-  const int KB = d_latent / 64;
-  const int64_t chunks = (int64_t)H * d_head * d_latent / 8;
+// A_h (d_out x d_in) -> the packed image: tile t = h * (d_out / 64) + m, box kb, row r: the
+// 16-byte chunk j of columns kb * 64 + 8 j .. + 7 at byte r * 128 + 16 (j ^ (r & 7)).  The
+// source w is [H, d_out, d_in] row-major (A_h = w[h]), or with `transpose` [H, d_in, d_out]
+// (A_h = w[h]^T).
+__global__ void __launch_bounds__(256) mlra_pack_kernel(const uint16_t* w, uint16_t* packed, int H,
+                                                        int d_in, int d_out, int transpose) {
+  const int KB = d_in / 64;
+  const int64_t chunks = (int64_t)H * d_out * d_in / 8;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < chunks;
        i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t box = i >> 9;            // 512 chunks of 16 bytes per 8 KB box
@@ -41,14 +48,25 @@ __global__ void __launch_bounds__(256) mlra_pack_wuv_kernel(const uint16_t* w, u
     const int r = within >> 3, jpos = within & 7, j = jpos ^ (r & 7);
     const int64_t t = box / KB;
     const int kb = static_cast<int>(box - t * KB);
-    const int64_t row = t * kProjM + r;    // = h * d_head + m * 64 + r
-    const uint4 v = *reinterpret_cast<const uint4*>(w + row * d_latent + kb * 64 + j * 8);
+    const int64_t row = t * kProjM + r;    // = h * d_out + m * 64 + r
+    const int col = kb * 64 + j * 8;
+    uint4 v;
+    if (!transpose) {
+      v = *reinterpret_cast<const uint4*>(w + row * d_in + col);
+    } else {
+      const int64_t h = row / d_out, o = row - h * d_out;
+      uint16_t e[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) e[u] = w[(h * d_in + col + u) * d_out + o];
+      v = make_uint4(e[0] | ((uint32_t)e[1] << 16), e[2] | ((uint32_t)e[3] << 16),
+                     e[4] | ((uint32_t)e[5] << 16), e[6] | ((uint32_t)e[7] << 16));
+    }
     *reinterpret_cast<uint4*>(packed + i * 8) = v;
   }
 }
 
-// shared memory: W boxes, o boxes, an mbarrier per W box and one for the products, the TMEM
-// address
+// shared memory: A boxes, x boxes, an mbarrier per A box and one for the products, the TMEM
+// address and a flag
 inline int project_smem_bytes(int kb) { return 2 * kb * kProjBox + 8 * (kb + 1) + 16 + 1024; }
 
 __device__ __forceinline__ bool project_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns,
@@ -69,7 +87,7 @@ mlra_project_kernel(const __grid_constant__ ProjectParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const int KB = p.d_latent / 64;
+  const int KB = p.d_in / 64;
   uint8_t* sW = smem;
   uint8_t* sX = smem + KB * kProjBox;
   const uint32_t bar_full = smem_u32(sX + KB * kProjBox);  // [KB]: W box kb landed
@@ -77,7 +95,7 @@ mlra_project_kernel(const __grid_constant__ ProjectParams p) {
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sX + KB * kProjBox + 8 * (KB + 1));
   volatile uint32_t* issued_all = tmem_slot + 1;  // every product was issued (no time-out)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mtiles = p.d_head / kProjM;
+  const int mtiles = p.d_out / kProjM;
   const int h = blockIdx.x / mtiles, m0 = (blockIdx.x % mtiles) * kProjM;
   const int n0 = blockIdx.y * kProjN;
   const int rows_n = min(kProjN, p.N - n0);
@@ -121,7 +139,7 @@ mlra_project_kernel(const __grid_constant__ ProjectParams p) {
       va[u] = vb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (idx < chunks && r < rows_n) {
         const float4* src = reinterpret_cast<const float4*>(
-            p.o + ((int64_t)(n0 + r) * p.H + h) * p.d_latent + cidx * 8);
+            p.x + ((int64_t)(n0 + r) * p.H + h) * p.d_in + cidx * 8);
         va[u] = __ldcg(src);
         vb[u] = __ldcg(src + 1);
       }
@@ -173,8 +191,13 @@ mlra_project_kernel(const __grid_constant__ ProjectParams p) {
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
         const int col = 32 * q + k;
-        if (col < rows_n)
-          p.y[((int64_t)(n0 + col) * p.H + h) * p.d_head + row] = __uint_as_float(r[k]);
+        if (col < rows_n) {
+          const int64_t at = ((int64_t)(n0 + col) * p.H + h) * p.d_out + row;
+          if (p.out_bf16)
+            static_cast<__nv_bfloat16*>(p.y)[at] = __float2bfloat16_rn(__uint_as_float(r[k]));
+          else
+            static_cast<float*>(p.y)[at] = __uint_as_float(r[k]);
+        }
       }
     }
   }

@@ -27,8 +27,8 @@ FLAG_TIMEOUT, FLAG_BAD_PAGE, FLAG_BAD_LENGTH = 0x1, 0x2, 0x4
 EXPORTS = ("mlra_workspace_size", "mlra_decode", "mlra_decode_profiled", "mlra_query_plan",
            "mlra_decode_static_scratch",
            "mlra_read_status", "mlra_debug_resolve_rows", "mlra_plan_host",
-           "mlra_plan_segments_host", "mlra_project", "mlra_pack_wuv", "mlra_status_string",
-           "mlra_version")
+           "mlra_plan_segments_host", "mlra_project", "mlra_pack_wuv", "mlra_absorb",
+           "mlra_pack_wuk", "mlra_rope_append", "mlra_status_string", "mlra_version")
 
 
 class Dims(ctypes.Structure):
@@ -86,13 +86,18 @@ def lib() -> ctypes.CDLL:
         L.mlra_project.argtypes = [vp, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                    vp, vp]
         L.mlra_pack_wuv.argtypes = [vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp]
+        L.mlra_absorb.argtypes = L.mlra_project.argtypes
+        L.mlra_pack_wuk.argtypes = L.mlra_pack_wuv.argtypes
+        L.mlra_rope_append.argtypes = [vp, vp, vp, vp, vp, ctypes.POINTER(Dims), vp, vp, vp,
+                                       ctypes.c_double, vp, vp]
         L.mlra_status_string.argtypes = [ctypes.c_int]
         L.mlra_status_string.restype = ctypes.c_char_p
         L.mlra_version.argtypes = []
         for f in ("mlra_workspace_size", "mlra_decode", "mlra_decode_profiled", "mlra_query_plan",
                   "mlra_decode_static_scratch",
                   "mlra_read_status", "mlra_debug_resolve_rows", "mlra_plan_host",
-                  "mlra_plan_segments_host", "mlra_project", "mlra_pack_wuv"):
+                  "mlra_plan_segments_host", "mlra_project", "mlra_pack_wuv", "mlra_absorb",
+                  "mlra_pack_wuk", "mlra_rope_append"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -188,6 +193,56 @@ def project(o: torch.Tensor, w_packed: torch.Tensor, y: Optional[torch.Tensor] =
     _check(lib().mlra_project(_ptr(o), _ptr(w_packed), _ptr(y), N, H, d_latent, d_head,
                               _ptr(status), ctypes.c_void_p(st)), "mlra_project")
     return y
+
+
+def pack_wuk(w_uk: torch.Tensor, stream=None) -> torch.Tensor:
+    """Packs the step-1 weights (bf16 [H, d_head, d_latent], head h's W^UK_{h,b} side by side)
+    for ``absorb`` through ``mlra_pack_wuk``; the result has the same shape, packed content."""
+    if w_uk.dtype != torch.bfloat16 or w_uk.dim() != 3 or not w_uk.is_contiguous():
+        raise ValueError("pack_wuk: contiguous bf16 [H, d_head, d_latent] expected")
+    H, d_head, d_latent = w_uk.shape
+    packed = torch.empty_like(w_uk)
+    st = stream if stream is not None else torch.cuda.current_stream(w_uk.device).cuda_stream
+    _check(lib().mlra_pack_wuk(_ptr(w_uk), _ptr(packed), H, d_head, d_latent, ctypes.c_void_p(st)),
+           "mlra_pack_wuk")
+    return packed
+
+
+def absorb(q_nope: torch.Tensor, w_packed: torch.Tensor, q_lat: Optional[torch.Tensor] = None,
+           status=None, stream=None) -> torch.Tensor:
+    """Step 1 through ``mlra_absorb``: q_lat[s, h, b-block] = W^UK_{h,b}^T q_nope[s, h] with
+    q_nope fp32 [N, H, d_head] and ``w_packed`` from ``pack_wuk``; returns bf16 [N, H, d_latent]."""
+    N, H, d_head = q_nope.shape
+    d_latent = w_packed.shape[2]
+    if (q_nope.dtype != torch.float32 or w_packed.dtype != torch.bfloat16
+            or w_packed.shape != (H, d_head, d_latent) or not q_nope.is_contiguous()):
+        raise ValueError("absorb: q_nope fp32 [N, H, d_head], w_packed bf16 [H, d_head, d_latent]")
+    if q_lat is None:
+        q_lat = torch.empty(N, H, d_latent, dtype=torch.bfloat16, device=q_nope.device)
+    st = stream if stream is not None else torch.cuda.current_stream(q_nope.device).cuda_stream
+    _check(lib().mlra_absorb(_ptr(q_nope), _ptr(w_packed), _ptr(q_lat), N, H, d_head, d_latent,
+                             _ptr(status), ctypes.c_void_p(st)), "mlra_absorb")
+    return q_lat
+
+
+def rope_append(q_rope_in, kr_new, c_new, seq_lens, page_table, c_kv, k_rope, *, max_seq_len=None,
+                page_size=0, rope_base=10000.0, q_rope_out=None, status=None, stream=None):
+    """RoPE of the new token's query and key and its append to the (bf16) cache at position
+    seq_lens[s], through ``mlra_rope_append``; returns the rotated query bf16 [N, H, d_rope]."""
+    N, H, d_rope = q_rope_in.shape
+    d_latent = c_new.shape[1]
+    q_lat_like = torch.empty(N, H, d_latent, dtype=torch.bfloat16, device=c_kv.device)
+    q_rope_like = torch.empty(N, H, d_rope, dtype=torch.bfloat16, device=c_kv.device)
+    dims = dims_for(q_lat_like, q_rope_like, c_kv, k_rope, seq_lens, page_table, 1,
+                    max_seq_len=max_seq_len, page_size=page_size)
+    if q_rope_out is None:
+        q_rope_out = q_rope_like
+    st = stream if stream is not None else torch.cuda.current_stream(c_kv.device).cuda_stream
+    _check(lib().mlra_rope_append(_ptr(q_rope_in), _ptr(kr_new), _ptr(c_new), _ptr(seq_lens),
+                                  _ptr(page_table), ctypes.byref(dims), _ptr(c_kv), _ptr(k_rope),
+                                  _ptr(q_rope_out), float(rope_base), _ptr(status),
+                                  ctypes.c_void_p(st)), "mlra_rope_append")
+    return q_rope_out
 
 
 def decode(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table=None, *, num_branches: int,
