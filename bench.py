@@ -480,67 +480,114 @@ def run_ours(args):
     return 0
 
 
-# ----------------------------------------------------------------------------- step 3
-def run_project(args):
-    """Times step 3 (mlra_project) alone on the workload's shapes: o = one decode's output,
-    W^UV [H, d_head = 128, d_latent] bf16 drawn N(0, 1/d_latent).  Bound by streaming W."""
+# ----------------------------------------------------------------------------- steps 1 and 3
+def graph_time(body, steps, pre=None):
+    """Mean device time (ms) of body() over `steps` calls replayed from one CUDA graph (no host
+    launch work between an event and its kernels); pre() runs before each call, untimed."""
+    evs = [(torch.cuda.Event(enable_timing=True, external=True),
+            torch.cuda.Event(enable_timing=True, external=True)) for _ in range(steps)]
+    dev = torch.cuda.current_device()
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side), torch.cuda.graph(graph, stream=side):
+        for a, b in evs:
+            if pre is not None:
+                pre()
+            a.record()
+            body()
+            b.record()
+    torch.cuda.synchronize()
+    graph.replay()
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+
+
+def run_stage(args):
+    """Times the steps around the attention path on the workload's shapes (d_head = 128 per head):
+      project: step 3 (value up-projection + branch sum) alone, W^UV evicted from L2 each call;
+      absorb:  step 1 (query absorption of W^UK) alone, W^UK evicted from L2 each call;
+      layer:   one attention layer's whole decode step -- step 1, the new token's RoPE and cache
+               append, step 2 (the path's two kernels) and step 3 -- back to back.
+    Weights are N(0, 1/fan-in) bf16 draws, packed once.  Prints one JSON line."""
     from latent_kv_cache_mlra_b200 import mlra
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     w = workloads.get(args.workload)
     inp = workloads.make_inputs(w)
-    pt = None if inp.page_table is None else inp.page_table.to(dev)
-    dec = mlra.Decoder(inp.q_lat.to(dev), inp.q_rope.to(dev), inp.c_kv.to(dev), inp.k_rope.to(dev),
-                       inp.seq_lens.to(dev), pt, num_branches=w.num_branches, softmax_scale=w.sigma,
-                       branch_scale=w.gamma, max_seq_len=inp.max_seq_len, page_size=w.page_size)
-    o = dec().contiguous()
-    d_head = 128
+    d_head, N, H, d_c, d_R = 128, w.batch, w.heads, w.d_latent, w.d_rope
     g = torch.Generator().manual_seed(w.seed + 77)
-    w_uv = (torch.randn(w.heads, d_head, w.d_latent, generator=g) / w.d_latent ** 0.5).to(
-        torch.bfloat16).to(dev)
-    w_uv = mlra.pack_wuv(w_uv)  # model weights are packed once, at load time
-    y = torch.empty(w.batch, w.heads, d_head, dtype=torch.float32, device=dev)
-    # W fits in L2: evict it before each launch by reading a buffer twice the L2 size (a read
-    # leaves clean lines, so the timed kernel pays no write-back of the flush)
+    w_uv = mlra.pack_wuv((torch.randn(H, d_head, d_c, generator=g) / d_c ** 0.5).to(torch.bfloat16).to(dev))
+    w_uk = mlra.pack_wuk((torch.randn(H, d_head, d_c, generator=g) / d_head ** 0.5).to(torch.bfloat16).to(dev))
+    pt = None if inp.page_table is None else inp.page_table.to(dev)
+    c, kr, lens = inp.c_kv.to(dev), inp.k_rope.to(dev), inp.seq_lens.to(dev)
+    q_lat, q_rope = inp.q_lat.to(dev), inp.q_rope.to(dev)
     flush = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
     sink = torch.empty((), dtype=torch.float32, device=dev)
-    for _ in range(args.warmup):
-        torch.sum(flush, dim=0, out=sink)
-        mlra.project(o, w_uv, y)
-    torch.cuda.synchronize()
-    # replayed from a CUDA graph so that no host launch work sits between an event and its kernel
-    evs = [(torch.cuda.Event(enable_timing=True, external=True),
-            torch.cuda.Event(enable_timing=True, external=True)) for _ in range(args.steps)]
-    side = torch.cuda.Stream(dev)
-    side.wait_stream(torch.cuda.current_stream(dev))
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(side), torch.cuda.graph(graph, stream=side):
-        for a, b in evs:
-            torch.sum(flush, dim=0, out=sink)
-            a.record()
-            mlra.project(o, w_uv, y)
-            b.record()
-    torch.cuda.synchronize()
-    with ClockSampler(0) as clk:
-        graph.replay()
-        torch.cuda.synchronize()
-    ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
-    nbytes = w_uv.numel() * 2 + o.numel() * 4 + y.numel() * 4
-    flops = 2 * w.batch * w.heads * d_head * w.d_latent
+    evict = lambda: torch.sum(flush, dim=0, out=sink)  # noqa: E731  (a read: clean lines)
+    q_nope = torch.randn(N, H, d_head, generator=g).to(dev)
     peaks = measured_peaks()
-    gbs = nbytes / (ms * 1e-3) / 1e9
-    print(json.dumps({
-        "metric": "step-3 projection (W^UV, branch sum) time per decode step", "value": ms * 1e3,
-        "unit": "us", "higher_is_better": False, "steps": args.steps, "warmup": args.warmup,
-        "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "d_latent": w.d_latent,
-                   "d_head": d_head, "l2": "L2 flushed (read of 2x L2) before each launch"},
-        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": gbs / peaks["hbm_gbs"], "kernel": "mlra_project_kernel",
-                     "algorithmic_bytes_per_launch": nbytes,
-                     "tensor_tflops": flops / (ms * 1e-3) / 1e12},
-        "clocks": clk.summary()}))
+    if args.stage in ("project", "absorb"):
+        if args.stage == "project":
+            dec = mlra.Decoder(q_lat, q_rope, c, kr, lens, pt, num_branches=w.num_branches,
+                               softmax_scale=w.sigma, branch_scale=w.gamma,
+                               max_seq_len=inp.max_seq_len, page_size=w.page_size)
+            x, wt = dec().contiguous(), w_uv
+            y = torch.empty(N, H, d_head, dtype=torch.float32, device=dev)
+            body = lambda: mlra.project(x, wt, y)  # noqa: E731
+            kernel, what = "mlra_project_kernel", "step-3 projection (W^UV, branch sum)"
+        else:
+            x, wt = q_nope, w_uk
+            y = torch.empty(N, H, d_c, dtype=torch.bfloat16, device=dev)
+            body = lambda: mlra.absorb(x, wt, y)  # noqa: E731
+            kernel, what = "mlra_project_kernel", "step-1 absorption (W^UK)"
+        for _ in range(args.warmup):
+            evict()
+            body()
+        with ClockSampler(0) as clk:
+            ms = graph_time(body, args.steps, pre=evict)
+        nbytes = wt.numel() * 2 + x.numel() * x.element_size() + y.numel() * y.element_size()
+        flops = 2 * N * H * d_head * d_c
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        line = {"metric": f"{what} time per decode step", "value": ms * 1e3, "unit": "us",
+                "higher_is_better": False,
+                "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                             "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "kernel": kernel,
+                             "algorithmic_bytes_per_launch": nbytes,
+                             "tensor_tflops": flops / (ms * 1e-3) / 1e12},
+                "l2": "L2 flushed (read of 2x L2) before each launch"}
+    else:  # layer
+        q_rope_in = torch.randn(N, H, d_R, generator=g).to(dev)
+        k_new, c_new = torch.randn(N, d_R, generator=g).to(dev), torch.randn(N, d_c, generator=g).to(dev)
+        q_lat2 = torch.empty(N, H, d_c, dtype=torch.bfloat16, device=dev)
+        q_rope2 = torch.empty(N, H, d_R, dtype=torch.bfloat16, device=dev)
+        lens_in = (lens - 1).clamp(min=0).to(torch.int32)   # the new token is the last position
+        dec = mlra.Decoder(q_lat2, q_rope2, c, kr, lens, pt, num_branches=w.num_branches,
+                           softmax_scale=w.sigma, branch_scale=w.gamma,
+                           max_seq_len=inp.max_seq_len, page_size=w.page_size)
+        y = torch.empty(N, H, d_head, dtype=torch.float32, device=dev)
+
+        def body():
+            mlra.absorb(q_nope, w_uk, q_lat2)
+            mlra.rope_append(q_rope_in, k_new, c_new, lens_in, pt, c, kr,
+                             max_seq_len=inp.max_seq_len if pt is None else None,
+                             page_size=w.page_size, q_rope_out=q_rope2)
+            mlra.project(dec(), w_uv, y)
+
+        for _ in range(args.warmup):
+            body()
+        with ClockSampler(0) as clk:
+            ms = graph_time(body, args.steps)
+        line = {"metric": "attention layer decode step (steps 1-3, RoPE and cache append)",
+                "value": N / (ms * 1e-3), "unit": "tokens/s", "higher_is_better": True,
+                "ms_per_step": ms, "kernels_per_step": 5 + (0 if dec.plan.launches == 2 else 1),
+                "l2": "inputs larger than L2" if cache_bytes(inp) > L2_BYTES else "L2 not flushed"}
+    line.update({"steps": args.steps, "warmup": args.warmup, "dtype": "bf16", "data": "synthetic",
+                 "config": {"workload": w.name, "batch": N, "heads": H, "d_latent": d_c,
+                            "d_rope": d_R, "d_head": d_head},
+                 "clocks": clk.summary()})
+    print(json.dumps(line))
     return 0
 
 
@@ -552,15 +599,16 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--stage", choices=["decode", "project"], default="decode",
-                    help="decode: the attention path (default line); project: step 3 alone")
+    ap.add_argument("--stage", choices=["decode", "project", "absorb", "layer"], default="decode",
+                    help="decode: the attention path (the default line); project / absorb: step 3 "
+                         "/ step 1 alone; layer: steps 1-3 with RoPE and the cache append")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
-    if args.stage == "project":
-        return run_project(args)
+    if args.stage != "decode":
+        return run_stage(args)
     return run_ours(args)
 
 

@@ -188,7 +188,10 @@ mlra_status mlra_decode_static_scratch(const void* q_lat, const void* q_rope, co
  *   w_packed H * d_head * d_latent bf16 device: the weights W^UV as mlra_pack_wuv wrote them
  *   y        [N, H, d_head] fp32 device (written)
  *   status nullable device uint32: gets MLRA_FLAG_TIMEOUT if a bounded wait runs out
- * Products in bf16 (o is rounded to bf16) with fp32 accumulation.  Asynchronous on `stream`.
+ * Products in bf16 (o is rounded to bf16) with fp32 accumulation.  Asynchronous on `stream`; the
+ * kernel starts reading w_packed before it waits for the previous kernel on the stream
+ * (programmatic serialization), so w_packed must not be written by a kernel that lets its
+ * dependents start early (mlra_pack_wuv does not).
  * Errors: MLRA_ERR_INVALID_ARG for null pointers or sizes < 1; MLRA_ERR_UNSUPPORTED unless
  * d_latent is a multiple of 64 up to 512, d_head a multiple of 64 and all three arrays 16-byte
  * aligned; MLRA_ERR_CUDA when the launch fails.  The pages give no kernel for this step. */
@@ -211,6 +214,7 @@ mlra_status mlra_pack_wuv(const void* w_uv, void* w_packed, int H, int d_latent,
  *   q_lat    [N, H, d_latent] bf16 device (written): mlra_decode's q_lat
  *   status   nullable device uint32: MLRA_FLAG_TIMEOUT if a bounded wait runs out
  * Products in bf16 (q_nope rounded) with fp32 accumulation, the result rounded to bf16.
+ * Asynchronous on `stream`; w_packed is read early as in mlra_project.
  * Errors: MLRA_ERR_INVALID_ARG for null pointers or sizes < 1; MLRA_ERR_UNSUPPORTED unless d_head
  * is a multiple of 64 up to 512, d_latent a multiple of 64 and the arrays 16-byte aligned. */
 mlra_status mlra_absorb(const float* q_nope, const void* w_packed, void* q_lat, int N, int H,
@@ -240,7 +244,8 @@ mlra_status mlra_pack_wuk(const void* w_uk, void* w_packed, int H, int d_head, i
  *   status     nullable device uint32: MLRA_FLAG_BAD_LENGTH (position outside the sequence's
  *              cache space) or MLRA_FLAG_BAD_PAGE (invalid page id); that append is skipped
  * Errors: MLRA_ERR_INVALID_ARG for null pointers, a non-positive base or invalid dims;
- * MLRA_ERR_UNSUPPORTED for an fp32 cache or an odd d_rope. */
+ * MLRA_ERR_UNSUPPORTED for an fp32 cache, an odd d_rope, d_latent, kr_row_stride or c_row_stride,
+ * or an array that is not 16-byte aligned. */
 mlra_status mlra_rope_append(const float* q_rope_in, const float* kr_new, const float* c_new,
                              const int32_t* seq_lens, const int32_t* page_table,
                              const mlra_dims* dims, void* c_kv, void* k_rope, void* q_rope_out,

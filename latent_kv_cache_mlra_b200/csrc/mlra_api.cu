@@ -519,6 +519,11 @@ mlra_status mlra_rope_append(const float* q_rope_in, const float* kr_new, const 
   const mlra_status st = check_dims(dims, paged);
   if (st != MLRA_OK) return st;
   if (dims->dtype != MLRA_BF16 || dims->d_rope % 2 != 0) return MLRA_ERR_UNSUPPORTED;
+  // pairs are moved as 8-byte (fp32) and 4-byte (bf16) words
+  if (!(aligned16(q_rope_in) && aligned16(kr_new) && aligned16(c_new) && aligned16(q_rope_out) &&
+        aligned16(k_rope) && aligned16(c_kv)) ||
+      dims->kr_row_stride % 2 != 0 || dims->d_latent % 2 != 0 || dims->c_row_stride % 2 != 0)
+    return MLRA_ERR_UNSUPPORTED;
   RopeAppendParams p;
   p.q_rope_in = q_rope_in; p.kr_new = kr_new; p.c_new = c_new;
   p.seq_lens = seq_lens; p.page_table = page_table;

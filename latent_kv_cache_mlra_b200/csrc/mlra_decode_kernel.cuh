@@ -394,11 +394,15 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           const uint32_t full = bar_stage_full + 8 * st;
           const uint32_t dst = sStage + st * C::STAGE;
           mbar_arrive_expect_tx(full, C::STAGE);
+          // the latent rows are read once per call (by this CTA alone): first out of L2, so the
+          // queries, RoPE rows (shared by the branch CTAs) and partial results stay
+          const uint64_t once = l2_policy_evict_first();
 #pragma unroll
           for (int l = 0; l < C::TB; ++l) {
 #pragma unroll
             for (int k = 0; k < C::NCB; ++k)
-              tma_load_2d(dst + k * C::CBLK + l * C::BOX, &tm_c, full, col0 + 64 * k, rows[l]);
+              tma_load_2d_hint(dst + k * C::CBLK + l * C::BOX, &tm_c, full, col0 + 64 * k, rows[l],
+                               once);
             tma_load_2d(dst + C::NCB * C::CBLK + l * C::BOX, &tm_kr, full, 0, rows[l]);
           }
         }

@@ -12,6 +12,7 @@ constexpr uint32_t kFlagBadPage = 0x2u;
 constexpr uint32_t kFlagBadLength = 0x4u;
 // Up to this many sequences the decode kernel plans its work range itself (no prep kernel).
 constexpr int kSelfPlanMaxSeqs = 64;
+constexpr int kMaxRopePairs = 32;     // d_rope <= 64
 
 // The split plan as the prep kernel writes it for the decode and combine kernels.
 //   RangeInfo[r]  : descriptors segs[first, first + count) of work range r, in tile order

@@ -392,16 +392,39 @@ cudaError_t launch_project(const ProjectParams& p, cudaStream_t st) {
 }
 
 // ----------------------------------------------------------------------------- K7
-// One block per sequence.  The new token sits at position p = seq_lens[s]: its row follows the
-// decode's addressing (page table, or s * max_seq_len + p).  Pair (2i, 2i+1) of the head queries
-// and of the key is rotated by the angle p * base^(-2i/d_rope) (angle in double precision: p
-// reaches 10^5 and more), the rotated query is written in bf16 for the decode, and the rotated
-// key and the latent c_new are written in bf16 to the cache row.  A position past the cache or an
-// invalid page id flags the status word and skips the append (the query is still rotated).
-__global__ void __launch_bounds__(256) mlra_rope_append_kernel(const RopeAppendParams p) {
+// Block (s, y) handles 256 of sequence s's items: the H * d_rope / 2 query pairs, then the
+// d_rope / 2 key pairs, then the d_latent / 2 pairs of c_new (copied, not rotated).  The new token
+// sits at position p = seq_lens[s]: its row follows the decode's addressing (page table, or
+// s * max_seq_len + p).  Pair (2i, 2i+1) of the head queries and of the key is rotated by the
+// angle p * base^(-2i/d_rope) (angle in double precision: p reaches 10^5 and more); the rotated
+// query is written in bf16 for the decode, the rotated key and the latent in bf16 to the cache row.
+// A position past the cache or an invalid page id flags the status word (block y = 0) and skips
+// the append (the query is still rotated).  Each thread's input pair is loaded before the angles
+// are computed, so the loads and the double-precision angle overlap.
+constexpr int kRopeThreads = 256;
+
+__global__ void __launch_bounds__(kRopeThreads) mlra_rope_append_kernel(const RopeAppendParams p) {
+  __shared__ float2 rot[kMaxRopePairs];  // (cos, sin) of the d_rope / 2 angles of this position
   const int s = blockIdx.x;
+  const int half = p.d_rope / 2;
+  const int nq = p.H * half, nk = nq + half, items = nk + p.d_latent / 2;
+  const int t = blockIdx.y * kRopeThreads + threadIdx.x;
   pdl_wait_prerequisites();  // the inputs come from the previous kernels on the stream
+  pdl_launch_dependents();   // the decode kernel may start its prologue
+  float2 x = make_float2(0.f, 0.f);
+  if (t < nq)
+    x = *reinterpret_cast<const float2*>(p.q_rope_in + (int64_t)s * p.H * p.d_rope + 2 * t);
+  else if (t < nk)
+    x = *reinterpret_cast<const float2*>(p.kr_new + (int64_t)s * p.d_rope + 2 * (t - nq));
+  else if (t < items)
+    x = *reinterpret_cast<const float2*>(p.c_new + (int64_t)s * p.d_latent + 2 * (t - nk));
   const int pos = p.seq_lens[s];
+  if (threadIdx.x < half) {
+    const double pd = pos > 0 ? (double)pos : 0.0;
+    double sn, cs;
+    sincos(pd * pow(p.base, -2.0 * threadIdx.x / p.d_rope), &sn, &cs);
+    rot[threadIdx.x] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+  }
   int64_t row = -1;
   uint32_t bad = 0;
   if (pos < 0) {
@@ -419,37 +442,29 @@ __global__ void __launch_bounds__(256) mlra_rope_append_kernel(const RopeAppendP
     if (pos >= p.max_seq_len) bad = kFlagBadLength;
     else row = (int64_t)s * p.max_seq_len + pos;
   }
-  if (bad && threadIdx.x == 0 && p.status) atomicOr(p.status, bad);
-  const double pd = pos > 0 ? (double)pos : 0.0;
-  const int half = p.d_rope / 2;
-  for (int t = threadIdx.x; t < (p.H + 1) * half; t += blockDim.x) {
-    const int v = t / half, i = t - v * half;
-    double sn, cs;
-    sincos(pd * pow(p.base, -2.0 * i / p.d_rope), &sn, &cs);
-    const float c = static_cast<float>(cs), sf = static_cast<float>(sn);
-    const float* src = v < p.H ? p.q_rope_in + ((int64_t)s * p.H + v) * p.d_rope
-                               : p.kr_new + (int64_t)s * p.d_rope;
-    const float x0 = src[2 * i], x1 = src[2 * i + 1];
-    const uint16_t y0 = __bfloat16_as_ushort(__float2bfloat16_rn(x0 * c - x1 * sf));
-    const uint16_t y1 = __bfloat16_as_ushort(__float2bfloat16_rn(x0 * sf + x1 * c));
-    uint16_t* dst = nullptr;
-    if (v < p.H) dst = p.q_rope_out + ((int64_t)s * p.H + v) * p.d_rope + 2 * i;
-    else if (row >= 0) dst = p.k_rope + row * p.kr_row_stride + 2 * i;
-    if (dst) {
-      dst[0] = y0;
-      dst[1] = y1;
-    }
+  if (bad && blockIdx.y == 0 && threadIdx.x == 0 && p.status) atomicOr(p.status, bad);
+  __syncthreads();
+  if (t >= items) return;
+  float2 y = x;
+  if (t < nk) {
+    const float2 r = rot[t < nq ? t % half : t - nq];
+    y = make_float2(x.x * r.x - x.y * r.y, x.x * r.y + x.y * r.x);
   }
-  if (row >= 0)
-    for (int j = threadIdx.x; j < p.d_latent; j += blockDim.x)
-      p.c_kv[row * p.c_row_stride + j] =
-          __bfloat16_as_ushort(__float2bfloat16_rn(p.c_new[(int64_t)s * p.d_latent + j]));
+  const uint32_t w = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y.x)) |
+                     ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y.y)) << 16);
+  uint16_t* dst = nullptr;
+  if (t < nq) dst = p.q_rope_out + (int64_t)s * p.H * p.d_rope + 2 * t;
+  else if (row < 0) dst = nullptr;
+  else if (t < nk) dst = p.k_rope + row * p.kr_row_stride + 2 * (t - nq);
+  else dst = p.c_kv + row * p.c_row_stride + 2 * (t - nk);
+  if (dst) *reinterpret_cast<uint32_t*>(dst) = w;
 }
 
 cudaError_t launch_rope_append(const RopeAppendParams& p, cudaStream_t st) {
+  const int items = p.H * (p.d_rope / 2) + p.d_rope / 2 + p.d_latent / 2;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.N);
-  cfg.blockDim = dim3(256);
+  cfg.gridDim = dim3(p.N, (items + kRopeThreads - 1) / kRopeThreads);
+  cfg.blockDim = dim3(kRopeThreads);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

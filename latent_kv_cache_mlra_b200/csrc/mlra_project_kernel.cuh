@@ -12,7 +12,9 @@
 // N = the sequences (padded to a multiple of 8), K = d_in, accumulated in TMEM.
 //   * A is packed once (mlra_pack_kernel, at model load) into the product's shared-memory image:
 //     per (head, 64-row tile) d_in / 64 boxes of [64 rows x 64 columns] bf16 in the 128-byte
-//     swizzled K-major layout, contiguous, so each box arrives with one contiguous bulk copy;
+//     swizzled K-major layout, contiguous, so each box arrives with one contiguous bulk copy.
+//     The copies are issued first thing, before the wait on the previous kernel (A is never
+//     written by it), so under programmatic serialization the weight stream overlaps its tail;
 //   * x_in (fp32) is rounded to bf16 by all threads into the same swizzled K-major layout;
 //   * one thread issues the d_in / 16 MMAs; the epilogue reads D with tcgen05.ld and writes
 //     x_out in fp32 or bf16 (a warp's 16 rows of one sequence are contiguous).
@@ -105,6 +107,14 @@ mlra_project_kernel(const __grid_constant__ ProjectParams p) {
     for (int kb = 0; kb < KB; ++kb) mbar_init(bar_full + 8 * kb, 1);
     mbar_init(bar_done, 1);
     fence_barrier_init();
+    // The packed weights are constant (packed at load), never the output of the previous kernel
+    // on the stream: their stream starts before the wait below, under that kernel's tail.
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(p.w_packed) +
+                         ((int64_t)h * mtiles + m0 / kProjM) * KB * kProjBox;
+    for (int kb = 0; kb < KB; ++kb) {
+      mbar_arrive_expect_tx(bar_full + 8 * kb, kProjBox);
+      bulk_load(smem_u32(sW + kb * kProjBox), src + kb * kProjBox, kProjBox, bar_full + 8 * kb);
+    }
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), 64);
@@ -114,17 +124,10 @@ mlra_project_kernel(const __grid_constant__ ProjectParams p) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // o comes from the previous kernel on the stream (programmatic serialization)
+  // x comes from the previous kernel on the stream (programmatic serialization); the next kernel
+  // may start its own prologue now (it waits for this grid before reading what it writes)
   pdl_wait_prerequisites();
-
-  if (warp == 1 && lane == 0) {
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(p.w_packed) +
-                         ((int64_t)h * mtiles + m0 / kProjM) * KB * kProjBox;
-    for (int kb = 0; kb < KB; ++kb) {
-      mbar_arrive_expect_tx(bar_full + 8 * kb, kProjBox);
-      bulk_load(smem_u32(sW + kb * kProjBox), src + kb * kProjBox, kProjBox, bar_full + 8 * kb);
-    }
-  }
+  pdl_launch_dependents();
   // o[n0 + r, h, :] -> bf16, box kb holds columns 64 kb .. 64 kb + 63 of row r at 128 r, its
   // 16-byte chunk j at position j ^ (r & 7).  Only the npad rows the products read are staged
   // (rows past the batch as zeros); the loads of 8 chunks are issued before any is converted.

@@ -277,3 +277,29 @@ def test_pack_wuv_argument_errors_without_a_gpu():
     assert lib.mlra_pack_wuv(fake, fake, 2, 96, 128, None) == mlra.MLRA_ERR_UNSUPPORTED
     assert lib.mlra_pack_wuv(fake, fake, 2, 512, 100, None) == mlra.MLRA_ERR_UNSUPPORTED
     assert lib.mlra_pack_wuv(ctypes.c_void_p(4100), fake, 2, 512, 128, None) == mlra.MLRA_ERR_UNSUPPORTED
+
+
+def test_rope_append_argument_errors_without_a_gpu():
+    """mlra_rope_append checks its arguments (base, dims, dtype, alignment) before any launch."""
+    lib = mlra.lib()
+    fake = ctypes.c_void_p(4096)
+
+    def call(dims, base=10000.0, **ptrs):
+        a = dict(q_in=fake, kr=fake, c=fake, lens=fake, pt=None, ckv=fake, krc=fake, q_out=fake)
+        a.update(ptrs)
+        return lib.mlra_rope_append(a["q_in"], a["kr"], a["c"], a["lens"], a["pt"], ctypes.byref(dims),
+                                    a["ckv"], a["krc"], a["q_out"], ctypes.c_double(base), None, None)
+
+    good = dict(batch=2, heads=4, num_branches=1, d_latent=128, d_rope=64, max_seq_len=64,
+                cache_rows=128)
+    assert call(mlra.make_dims(**good), base=0.0) == mlra.MLRA_ERR_INVALID_ARG
+    assert call(mlra.make_dims(**good), base=float("nan")) == mlra.MLRA_ERR_INVALID_ARG
+    assert call(mlra.make_dims(**good), q_in=None) == mlra.MLRA_ERR_INVALID_ARG
+    assert call(mlra.make_dims(**dict(good, d_rope=63))) == mlra.MLRA_ERR_UNSUPPORTED
+    assert call(mlra.make_dims(**dict(good, dtype="f32"))) == mlra.MLRA_ERR_UNSUPPORTED
+    assert call(mlra.make_dims(**dict(good, kr_row_stride=65))) == mlra.MLRA_ERR_UNSUPPORTED
+    assert call(mlra.make_dims(**dict(good, d_latent=127))) == mlra.MLRA_ERR_UNSUPPORTED
+    assert call(mlra.make_dims(**dict(good, c_row_stride=129))) == mlra.MLRA_ERR_UNSUPPORTED
+    for name in ("q_in", "kr", "c", "q_out", "krc", "ckv"):
+        assert call(mlra.make_dims(**good), **{name: ctypes.c_void_p(4104)}) == mlra.MLRA_ERR_UNSUPPORTED, name
+    assert call(mlra.make_dims(**dict(good, cache_rows=100))) == mlra.MLRA_ERR_INVALID_ARG  # 2 x 64 rows
