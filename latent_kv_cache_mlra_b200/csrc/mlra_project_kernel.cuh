@@ -16,8 +16,9 @@
 //     The copies are issued first thing, before the wait on the previous kernel (A is never
 //     written by it), so under programmatic serialization the weight stream overlaps its tail;
 //   * x_in (fp32) is rounded to bf16 by all threads into the same swizzled K-major layout;
-//   * one thread issues the d_in / 16 MMAs; the epilogue reads D with tcgen05.ld and writes
-//     x_out in fp32 or bf16 (a warp's 16 rows of one sequence are contiguous).
+//   * one thread issues the d_in / 16 MMAs, a group of four boxes (one copy, one mbarrier) at a
+//     time; the epilogue reads D with tcgen05.ld, transposes it through shared memory and writes
+//     x_out in fp32 or bf16 with 16-byte stores (64 consecutive rows of one sequence).
 // The work is bound by streaming A (H d_out d_in bf16) from HBM.
 #pragma once
 #include <cstdint>
@@ -34,6 +35,7 @@ constexpr int kProjThreads = 128;
 constexpr int kProjM = 64;     // rows of A_h per CTA
 constexpr int kProjN = 64;     // sequences per CTA
 constexpr int kProjBox = 8192; // one [64 x 64] bf16 box
+constexpr int kProjGroup = 4;  // boxes per weight copy and per mbarrier (32 KB)
 
 // A_h (d_out x d_in) -> the packed image: tile t = h * (d_out / 64) + m, box kb, row r: the
 // 16-byte chunk j of columns kb * 64 + 8 j .. + 7 at byte r * 128 + 16 (j ^ (r & 7)).  The
@@ -67,8 +69,8 @@ __global__ void __launch_bounds__(256) mlra_pack_kernel(const uint16_t* w, uint1
   }
 }
 
-// shared memory: A boxes, x boxes, an mbarrier per A box and one for the products, the TMEM
-// address and a flag
+// shared memory: A boxes, x boxes, an mbarrier per group of A boxes (at most one per box) and
+// one for the products, the TMEM address and a flag
 inline int project_smem_bytes(int kb) { return 2 * kb * kProjBox + 8 * (kb + 1) + 16 + 1024; }
 
 __device__ __forceinline__ bool project_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns,
@@ -92,7 +94,7 @@ mlra_project_kernel(const __grid_constant__ ProjectParams p) {
   const int KB = p.d_in / 64;
   uint8_t* sW = smem;
   uint8_t* sX = smem + KB * kProjBox;
-  const uint32_t bar_full = smem_u32(sX + KB * kProjBox);  // [KB]: W box kb landed
+  const uint32_t bar_full = smem_u32(sX + KB * kProjBox);  // [groups]: W boxes of group g landed
   const uint32_t bar_done = bar_full + 8 * KB;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sX + KB * kProjBox + 8 * (KB + 1));
   volatile uint32_t* issued_all = tmem_slot + 1;  // every product was issued (no time-out)
@@ -103,17 +105,21 @@ mlra_project_kernel(const __grid_constant__ ProjectParams p) {
   const int rows_n = min(kProjN, p.N - n0);
   const int npad = (rows_n + 7) / 8 * 8;
 
+  const int ngroups = (KB + kProjGroup - 1) / kProjGroup;
   if (threadIdx.x == 0) {
-    for (int kb = 0; kb < KB; ++kb) mbar_init(bar_full + 8 * kb, 1);
+    for (int g = 0; g < ngroups; ++g) mbar_init(bar_full + 8 * g, 1);
     mbar_init(bar_done, 1);
     fence_barrier_init();
     // The packed weights are constant (packed at load), never the output of the previous kernel
-    // on the stream: their stream starts before the wait below, under that kernel's tail.
+    // on the stream: their stream starts before the wait below, under that kernel's tail.  The
+    // boxes of a group are contiguous in the packed image: one copy (and one mbarrier) each.
     const uint8_t* src = reinterpret_cast<const uint8_t*>(p.w_packed) +
                          ((int64_t)h * mtiles + m0 / kProjM) * KB * kProjBox;
-    for (int kb = 0; kb < KB; ++kb) {
-      mbar_arrive_expect_tx(bar_full + 8 * kb, kProjBox);
-      bulk_load(smem_u32(sW + kb * kProjBox), src + kb * kProjBox, kProjBox, bar_full + 8 * kb);
+    for (int g = 0; g < ngroups; ++g) {
+      const int kb0 = g * kProjGroup;
+      const uint32_t bytes = (uint32_t)(min(KB - kb0, kProjGroup) * kProjBox);
+      mbar_arrive_expect_tx(bar_full + 8 * g, bytes);
+      bulk_load(smem_u32(sW + kb0 * kProjBox), src + kb0 * kProjBox, bytes, bar_full + 8 * g);
     }
   }
   if (warp == 0) {
@@ -163,44 +169,61 @@ mlra_project_kernel(const __grid_constant__ ProjectParams p) {
 
   bool ok = true;
   if (threadIdx.x == 0) {
-    // the products of box kb start as soon as it lands
+    // the products of a group start as soon as it lands; within a group they are issued back to
+    // back (a wait between two products costs more than the product)
     const uint32_t idesc = idesc_bf16_f32(kProjM, npad, false, false);
-    for (int kb = 0; ok && kb < KB; ++kb) {
-      ok = project_wait(bar_full + 8 * kb, 0, p.timeout_ns, p.status);
+    for (int g = 0; ok && g < ngroups; ++g) {
+      ok = project_wait(bar_full + 8 * g, 0, p.timeout_ns, p.status);
       if (!ok) break;
       tc_fence_after();
+      for (int kb = g * kProjGroup; kb < min(KB, (g + 1) * kProjGroup); ++kb) {
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        umma_bf16(tmem, sw128_desc(smem_u32(sW + kb * kProjBox) + kk * 32, 16, 1024),
-                  sw128_desc(smem_u32(sX + kb * kProjBox) + kk * 32, 16, 1024), idesc,
-                  (kb | kk) ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk)
+          umma_bf16(tmem, sw128_desc(smem_u32(sW + kb * kProjBox) + kk * 32, 16, 1024),
+                    sw128_desc(smem_u32(sX + kb * kProjBox) + kk * 32, 16, 1024), idesc,
+                    (kb | kk) ? 1u : 0u);
+      }
     }
     *issued_all = ok ? 1u : 0u;
     umma_commit(bar_done);  // also after a time-out: it tracks whatever was issued
   }
   __syncthreads();
-  {
-    // every thread waits for the products (bounded)
-    const bool done = __all_sync(0xffffffffu, project_wait(bar_done, 0, p.timeout_ns,
-                                                           threadIdx.x == 0 ? p.status : nullptr));
-    if (done && *issued_all) {  // warp-uniform: tcgen05.ld is a warp-wide instruction
-      tc_fence_after();
-      // D rows 16 w .. 16 w + 15 live in lanes 32 w + [0, 16); lane half q holds columns
-      // 32 q .. 32 q + 31 (the sequences n0 + column)
-      uint32_t r[32];
-      tmem_ld16x2_32(tmem + ((uint32_t)(32 * warp) << 16), r);
-      tmem_wait_ld();
-      const int row = m0 + 16 * warp + (lane & 15), q = lane >> 4;
+  // every thread waits for the products (bounded); the epilogue runs only if the whole block saw
+  // them complete (it has block-wide barriers)
+  const bool done = __syncthreads_and(project_wait(bar_done, 0, p.timeout_ns,
+                                                   threadIdx.x == 0 ? p.status : nullptr)) != 0;
+  if (done && *issued_all) {
+    tc_fence_after();
+    // D rows 16 w .. 16 w + 15 live in lanes 32 w + [0, 16); lane half q holds columns
+    // 32 q .. 32 q + 31 (the sequences n0 + column).  They go through shared memory (the A boxes
+    // are free now) as sT[column][row], so that each output row segment of 64 values leaves as
+    // 16-byte stores: one scattered 4-byte store per value costs several times more.
+    uint32_t r[32];
+    tmem_ld16x2_32(tmem + ((uint32_t)(32 * warp) << 16), r);
+    tmem_wait_ld();
+    float* sT = reinterpret_cast<float*>(sW);  // [64][64] fp32 = 16 KB <= 2 * KB * 8 KB
+    const int q = lane >> 4, rr = 16 * warp + (lane & 15);
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const int col = 32 * q + k;
-        if (col < rows_n) {
-          const int64_t at = ((int64_t)(n0 + col) * p.H + h) * p.d_out + row;
-          if (p.out_bf16)
-            static_cast<__nv_bfloat16*>(p.y)[at] = __float2bfloat16_rn(__uint_as_float(r[k]));
-          else
-            static_cast<float*>(p.y)[at] = __uint_as_float(r[k]);
-        }
+    for (int k = 0; k < 32; ++k) sT[(32 * q + k) * kProjM + rr] = __uint_as_float(r[k]);
+    __syncthreads();
+    if (p.out_bf16) {
+      // 8 rows (16 bytes) per store
+      for (int it = threadIdx.x; it < rows_n * (kProjM / 8); it += kProjThreads) {
+        const int col = it / (kProjM / 8), c8 = it % (kProjM / 8);
+        const float4 a = *reinterpret_cast<const float4*>(sT + col * kProjM + 8 * c8);
+        const float4 b = *reinterpret_cast<const float4*>(sT + col * kProjM + 8 * c8 + 4);
+        const int64_t at = ((int64_t)(n0 + col) * p.H + h) * p.d_out + m0 + 8 * c8;
+        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.y) + at) =
+            make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
+                       pack_bf16x2(b.z, b.w));
+      }
+    } else {
+      // 4 rows (16 bytes) per store
+      for (int it = threadIdx.x; it < rows_n * (kProjM / 4); it += kProjThreads) {
+        const int col = it / (kProjM / 4), c4 = it % (kProjM / 4);
+        const int64_t at = ((int64_t)(n0 + col) * p.H + h) * p.d_out + m0 + 4 * c4;
+        *reinterpret_cast<float4*>(static_cast<float*>(p.y) + at) =
+            *reinterpret_cast<const float4*>(sT + col * kProjM + 4 * c4);
       }
     }
   }
