@@ -62,17 +62,20 @@ def measured_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
-def kernel_hash() -> str:
+PROJECT_SOURCES = ["mlra_project_kernel.cuh", "sm100_ptx.cuh", "mlra_internal.h"]
+
+
+def kernel_hash(sources=None) -> str:
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in sources or KERNEL_SOURCES:
         h.update((ROOT / "latent_kv_cache_mlra_b200" / "csrc" / name).read_bytes())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
-    """DRAM bytes per attention launch from the committed ncu summary, if it matches the
-    current kernel source; else None."""
-    f = PROFILE_DIR / f"decode_kernel_{workload}.md"
+def recorded_traffic(workload: str, kind: str = "decode_kernel", sources=None):
+    """DRAM bytes per launch of a kernel from the committed ncu summary
+    profiles/<kind>_<workload>.md, if it matches the current kernel source; else None."""
+    f = PROFILE_DIR / f"{kind}_{workload}.md"
     if not f.exists():
         return None
     vals = {}
@@ -80,7 +83,7 @@ def recorded_traffic(workload: str):
         if line.startswith("- ") and ":" in line:
             k, v = line[2:].split(":", 1)
             vals[k.strip()] = v.strip()
-    if vals.get("kernel_source_hash") != kernel_hash():
+    if vals.get("kernel_source_hash") != kernel_hash(sources):
         return None
     try:
         return int(float(vals["dram_bytes_per_launch"]))
@@ -555,6 +558,8 @@ def run_stage(args):
                 "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
                              "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "kernel": kernel,
                              "algorithmic_bytes_per_launch": nbytes,
+                             "traffic": recorded_traffic(w.name, f"{args.stage}_kernel",
+                                                         PROJECT_SOURCES),
                              "tensor_tflops": flops / (ms * 1e-3) / 1e12},
                 "l2": "L2 flushed (read of 2x L2) before each launch"}
     else:  # layer
