@@ -511,7 +511,8 @@ def run_stage(args):
       project: step 3 (value up-projection + branch sum) alone, W^UV evicted from L2 each call;
       absorb:  step 1 (query absorption of W^UK) alone, W^UK evicted from L2 each call;
       layer:   one attention layer's whole decode step -- step 1, the new token's RoPE and cache
-               append, step 2 (the path's two kernels) and step 3 -- back to back.
+               append, step 2 (the path's two kernels) and step 3 -- with L2 evicted before each
+               step (and, for reference, back to back).
     Weights are N(0, 1/fan-in) bf16 draws, packed once.  Prints one JSON line."""
     from latent_kv_cache_mlra_b200 import mlra
 
@@ -583,11 +584,17 @@ def run_stage(args):
         for _ in range(args.warmup):
             body()
         with ClockSampler(0) as clk:
-            ms = graph_time(body, args.steps)
+            # L2 evicted before every step, as after the model's other layers: this layer's
+            # weights and queries come from HBM (the timed region is the step alone)
+            ms = graph_time(body, args.steps, pre=evict)
+            # back to back, the 16 MB of this layer's weights may stay in L2 (the cache stream is
+            # evict-first): a single-layer best case, reported beside the value
+            ms_kept = graph_time(body, args.steps)
         line = {"metric": "attention layer decode step (steps 1-3, RoPE and cache append)",
                 "value": N / (ms * 1e-3), "unit": "tokens/s", "higher_is_better": True,
-                "ms_per_step": ms, "kernels_per_step": 5 + (0 if dec.plan.launches == 2 else 1),
-                "l2": "inputs larger than L2" if cache_bytes(inp) > L2_BYTES else "L2 not flushed"}
+                "ms_per_step": ms, "ms_per_step_back_to_back": ms_kept,
+                "kernels_per_step": 5 + (0 if dec.plan.launches == 2 else 1),
+                "l2": "L2 flushed (read of 2x L2) before each step, outside the timed region"}
     line.update({"steps": args.steps, "warmup": args.warmup, "dtype": "bf16", "data": "synthetic",
                  "config": {"workload": w.name, "batch": N, "heads": H, "d_latent": d_c,
                             "d_rope": d_R, "d_head": d_head},
