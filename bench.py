@@ -575,10 +575,12 @@ def run_stage(args):
         y = torch.empty(N, H, d_head, dtype=torch.float32, device=dev)
 
         def body():
-            mlra.absorb(q_nope, w_uk, q_lat2)
+            # RoPE/append first: the absorption's weight copies then start under its tail
+            # (they precede the absorption kernel's dependency wait)
             mlra.rope_append(q_rope_in, k_new, c_new, lens_in, pt, c, kr,
                              max_seq_len=inp.max_seq_len if pt is None else None,
                              page_size=w.page_size, q_rope_out=q_rope2)
+            mlra.absorb(q_nope, w_uk, q_lat2)
             mlra.project(dec(), w_uv, y)
 
         for _ in range(args.warmup):
