@@ -41,3 +41,13 @@ def test_named_workloads_recipe():
     t = workloads.get("tiny_mlra4_f32")
     assert t.dtype == "f32" and math.isclose(t.sigma, 1 / math.sqrt(48)) and t.latent_scale == 1.0
     assert math.isclose(workloads.get("long_mlra2_l128k").latent_scale, 0.5)
+
+
+def test_tp4_shard_workload_is_one_branch_of_mlra4():
+    full, shard = workloads.get("mlra4_n8_l32k"), workloads.get("mlra4_tp4_shard_n8_l32k")
+    assert shard.num_branches == 1 and shard.d_latent == full.d_blk
+    assert shard.d_rope == full.d_rope and shard.batch == full.batch and shard.seq_len == full.seq_len
+    assert math.isclose(shard.sigma, full.sigma) and math.isclose(shard.gamma, full.gamma)
+    assert math.isclose(shard.latent_scale, full.latent_scale)
+    # bytes per cached token: 192 elements against MLRA-4's (and MLA's) 576 on one device
+    assert (shard.d_latent + shard.d_rope) * 3 == full.d_latent + full.d_rope

@@ -96,6 +96,12 @@ WORKLOADS = {
     "long_mlra2_l128k": Workload(
         name="long_mlra2_l128k", batch=1, heads=64, num_branches=2, d_latent=512, d_rope=64,
         seq_len=131072, seed=1004),
+    # One device's share of mlra4_n8_l32k when the 4 branches sit on 4 devices (tensor
+    # parallelism, one branch each): its 128-column latent block and the shared RoPE key, i.e.
+    # d_R + d_c / 4 = 192 cached elements per token instead of 576.  Same scales as MLRA-4.
+    "mlra4_tp4_shard_n8_l32k": Workload(
+        name="mlra4_tp4_shard_n8_l32k", batch=8, heads=64, num_branches=1, d_latent=128,
+        d_rope=64, seq_len=32768, seed=1006, alpha=math.sqrt(64 / 128), branch_scale=0.25),
     "serving_mlra4_n64_paged": Workload(
         name="serving_mlra4_n64_paged", batch=64, heads=64, num_branches=4, d_latent=512,
         d_rope=64, seq_len=65536, min_seq_len=1024, ragged=True, page_size=64, seed=1005),
