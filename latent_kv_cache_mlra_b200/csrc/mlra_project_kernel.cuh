@@ -227,6 +227,8 @@ mlra_project_kernel(const __grid_constant__ ProjectParams p) {
       }
     }
   }
+  if (threadIdx.x == 0 && !*issued_all)  // after a time-out: let the weight copies land (bounded)
+    for (int g = 0; g < ngroups; ++g) project_wait(bar_full + 8 * g, 0, p.timeout_ns / 8, nullptr);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
