@@ -145,3 +145,41 @@ def test_steps_1_2_3_chained():
     out_ref, _ = oracle.decode(q_lat_ref, q_rope_ref, c2, k2, lens2, None, B, sigma, gamma,
                                max_seq_len=L)
     assert_close(y, oracle.project(out_ref, w_uv.float()), "steps 1-2-3")
+
+
+def test_layer_chain_full_size_sampled():
+    """RoPE/append -> absorb -> decode -> project at the mlra4_n8_l32k shapes (8 x 32768 tokens,
+    64 heads, d_c = 512, d_head = 128) on the CUDA path, against the oracle's chain on sampled
+    sequences (their cache rows cut out: the contiguous layout keeps a sequence's rows together)."""
+    import workloads
+    w = workloads.get("mlra4_n8_l32k")
+    inp = workloads.make_inputs(w)
+    N, H, d_c, d_R, d_head, L = w.batch, w.heads, w.d_latent, w.d_rope, 128, inp.max_seq_len
+    g = torch.Generator().manual_seed(13)
+    w_uk = (torch.randn(H, d_head, d_c, generator=g) / d_head ** 0.5).to(torch.bfloat16)
+    w_uv = (torch.randn(H, d_head, d_c, generator=g) / d_c ** 0.5).to(torch.bfloat16)
+    q_nope = torch.randn(N, H, d_head, generator=g)
+    q_rope_in = torch.randn(N, H, d_R, generator=g)
+    k_new, c_new = torch.randn(N, d_R, generator=g), torch.randn(N, d_c, generator=g) * 0.7
+    lens_in = inp.seq_lens - 1  # the new token takes the last row of each sequence's space
+    # CUDA path
+    dc, dk = inp.c_kv.cuda(), inp.k_rope.cuda()
+    q_rope = mlra.rope_append(q_rope_in.cuda(), k_new.cuda(), c_new.cuda(), lens_in.cuda(), None,
+                              dc, dk, max_seq_len=L)
+    q_lat = mlra.absorb(q_nope.cuda(), mlra.pack_wuk(w_uk.cuda()))
+    out, _ = mlra.decode(q_lat, q_rope, dc, dk, inp.seq_lens.cuda(), None, num_branches=w.num_branches,
+                         softmax_scale=w.sigma, branch_scale=w.gamma, max_seq_len=L)
+    y = mlra.project(out.contiguous(), mlra.pack_wuv(w_uv.cuda())).cpu()
+    # oracle chain on the sampled sequences
+    seqs = [0, 5]
+    rows = torch.cat([torch.arange(s * L, (s + 1) * L) for s in seqs])
+    c_sub, k_sub = inp.c_kv[rows].float(), inp.k_rope[rows].float()
+    pos = lens_in[seqs].double().numpy()
+    k_ref = oracle.rope(k_new[seqs], pos, 10000.0)
+    c2, k2, lens2 = oracle.append_token(c_sub, k_sub, lens_in[seqs], None, 0, L,
+                                        c_new[seqs].to(torch.bfloat16).float(),
+                                        torch.from_numpy(k_ref).to(torch.bfloat16).float())
+    out_ref, _ = oracle.decode(oracle.absorb(q_nope[seqs], w_uk.float()),
+                               oracle.rope(q_rope_in[seqs], pos[:, None], 10000.0), c2, k2, lens2,
+                               None, w.num_branches, w.sigma, w.gamma, max_seq_len=L)
+    assert_close(y[seqs], oracle.project(out_ref, w_uv.float()), "layer chain, full size")
