@@ -151,6 +151,31 @@ def decode(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table, num_branches, sigm
     return np.stack(outs), np.stack(lses)
 
 
+def decode_multi(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table, num_branches, sigma, gamma,
+                 page_size=0, max_seq_len=0, out_mode="branches"):
+    """Decode attention for the q newest tokens of every sequence at once (a speculative or
+    chunked-prefill step; the absorbed step 2 of section 1.3 for each of them).
+
+    q_lat [N, q, H, d_c], q_rope [N, q, H, d_R]: token t of sequence s is at position
+    seq_lens[s] - q + t; all q tokens are already in the cache (seq_lens counts them).  Token t
+    attends positions 0 .. seq_lens[s] - q + t (causal among the new tokens), i.e. it is the
+    single-token decode with the length seq_lens[s] - (q - 1 - t) over the same cache rows.
+    Returns (out [N, q, H, ...], lse [N, q, H, B]).
+    """
+    q_lat, q_rope = to_f64(q_lat), to_f64(q_rope)
+    lens = np.asarray(seq_lens.tolist() if hasattr(seq_lens, "tolist") else seq_lens, dtype=np.int64)
+    q = q_lat.shape[1]
+    outs, lses = [], []
+    for t in range(q):
+        lens_t = np.maximum(lens - (q - 1 - t), 0)
+        o, l = decode(q_lat[:, t], q_rope[:, t], c_kv, k_rope, lens_t, page_table, num_branches,
+                      sigma, gamma, page_size=page_size, max_seq_len=max_seq_len,
+                      out_mode=out_mode)
+        outs.append(o)
+        lses.append(l)
+    return np.stack(outs, axis=1), np.stack(lses, axis=1)
+
+
 def branch_probabilities(q_lat_s, q_rope_s, c_rows, kr_rows, num_branches, sigma):
     """Attention weights p[b, h, j] of one sequence (for the sum-to-one checks)."""
     _, _, probs = decode_heads(to_f64(q_lat_s), to_f64(q_rope_s), to_f64(c_rows), to_f64(kr_rows),

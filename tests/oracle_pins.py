@@ -393,7 +393,59 @@ def pin_append_token(orc, seed=12):
     assert [r for r in range(rows) if (c3[r] != c_kv[r]).any()] == [2, 10, 27]
 
 
+def explicit_mlra_causal(q_nope, q_rope, c, kr, W_uk, W_uv, sigma, gamma):
+    """Like ``explicit_mlra`` for the q newest tokens of one sequence with a causal mask: query t
+    (q_nope [q, H, B, d_h], q_rope [q, H, d_R]) sees keys 0 .. L - q + t.  The mask is built as a
+    boolean matrix (the decode alignment is bottom-right, not SDPA's is_causal top-left)."""
+    q_len = q_nope.shape[0]
+    H, B, d_h, d_blk = W_uk.shape
+    L = c.shape[0]
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x))
+    mask = torch.arange(L)[None, :] <= (L - q_len + torch.arange(q_len))[:, None]   # [q, L]
+    y = torch.zeros(q_len, H, d_h, dtype=torch.float64)
+    for b in range(B):
+        cb = t(c[:, b * d_blk:(b + 1) * d_blk])
+        k_nope = torch.einsum("hkd,ld->hlk", t(W_uk[:, b]), cb)            # [H, L, d_h]
+        v = torch.einsum("hkd,ld->hlk", t(W_uv[:, b]), cb)
+        k = torch.cat([k_nope, t(kr)[None].expand(H, -1, -1)], dim=-1)     # [H, L, d_h + d_R]
+        qq = torch.cat([t(q_nope[:, :, b]), t(q_rope)], dim=-1).transpose(0, 1)  # [H, q, d_h+d_R]
+        o = F.scaled_dot_product_attention(qq[None], k[None], v[None], attn_mask=mask, scale=sigma)[0]
+        y += o.transpose(0, 1)                                               # [q, H, d_h]
+    return (gamma * y).numpy()
+
+
+def pin_multi_token_equals_explicit_causal(orc, seed=12, H=3, B=4, d_blk=8, d_R=4, d_h=5, L=29, q=3):
+    """The q newest tokens (``decode_multi``) -> step 3 == explicit decompressed attention with a
+    bottom-right causal mask; q = 1 is the single-token decode; a token ignores later positions."""
+    rng = np.random.default_rng(seed)
+    W_uk, W_uv = _rand(rng, H, B, d_h, d_blk), _rand(rng, H, B, d_h, d_blk)
+    q_nope, q_rope = _rand(rng, q, H, B, d_h), _rand(rng, q, H, d_R)
+    c, kr = _rand(rng, L, B * d_blk), _rand(rng, L, d_R)
+    sigma, gamma = 0.31, 1.0 / B
+    ref = explicit_mlra_causal(q_nope, q_rope, c, kr, W_uk, W_uv, sigma, gamma)
+    q_lat = np.stack([np.concatenate([np.einsum("hkd,hk->hd", W_uk[:, b], q_nope[t, :, b])
+                                      for b in range(B)], 1) for t in range(q)])  # [q, H, d_c]
+    w_uv = np.concatenate([W_uv[:, b] for b in range(B)], axis=2)
+    out, lse = orc.decode_multi(q_lat[None], q_rope[None], c, kr, [L], None, B, sigma, gamma,
+                                max_seq_len=L)
+    assert out.shape == (1, q, H, B * d_blk) and lse.shape == (1, q, H, B)
+    y = orc.project(out[0], w_uv)
+    err = np.abs(y - ref).max() / np.abs(ref).max()
+    assert err <= 1e-12, f"multi-token vs explicit causal rel err {err:.3e}"
+    one, _ = orc.decode_multi(q_lat[None, -1:], q_rope[None, -1:], c, kr, [L], None, B, sigma,
+                              gamma, max_seq_len=L)
+    single, _ = _one_seq(orc, q_lat[-1], q_rope[-1], c, kr, B, sigma, gamma)
+    assert np.array_equal(one[0, 0], single), "q = 1 is the single-token decode"
+    c2 = c.copy()
+    c2[L - 1] += 5.0  # the last position: seen by the last token only
+    out2, _ = orc.decode_multi(q_lat[None], q_rope[None], c2, kr, [L], None, B, sigma, gamma,
+                               max_seq_len=L)
+    assert np.array_equal(out2[0, :-1], out[0, :-1]), "earlier tokens ignore later positions"
+    assert not np.allclose(out2[0, -1], out[0, -1]), "the last token sees its own position"
+
+
 ALL_PINS = [
+    pin_multi_token_equals_explicit_causal,
     pin_absorb_equals_explicit,
     pin_rope,
     pin_append_token,

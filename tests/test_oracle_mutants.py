@@ -43,6 +43,10 @@ MUTANTS = {
     "rope_pairs_halves": ("x0, x1 = x[..., 0::2], x[..., 1::2]", "x0, x1 = x[..., : d // 2], x[..., d // 2:]"),
     "rope_frequency_exponent": ("theta = base ** (-2.0 * i / d)", "theta = base ** (-1.0 * i / d)"),
     "append_off_by_one": ("        p = int(lens[s])\n", "        p = max(int(lens[s]) - 1, 0)\n"),
+    "multi_token_causal_off_by_one": ("lens_t = np.maximum(lens - (q - 1 - t), 0)",
+                                      "lens_t = np.maximum(lens - (q - t), 0)"),
+    "multi_token_reversed": ("o, l = decode(q_lat[:, t], q_rope[:, t], c_kv, k_rope, lens_t,",
+                             "o, l = decode(q_lat[:, q - 1 - t], q_rope[:, q - 1 - t], c_kv, k_rope, lens_t,"),
     "project_head_shift": ('np.einsum("hkd,shd->shk", to_f64(w_uv), to_f64(out))',
                            'np.einsum("hkd,shd->shk", np.roll(to_f64(w_uv), 1, axis=0), to_f64(out))'),
 }
