@@ -155,6 +155,30 @@ typedef struct {
 } mlra_plan_info;
 mlra_status mlra_query_plan(const mlra_dims* dims, mlra_plan_info* info_host);
 
+/* Decode for several query tokens per sequence (a speculative-decoding or chunked-prefill step):
+ * the q_len newest tokens of every sequence attend the cache at once, each causally — token t of
+ * sequence s sits at position seq_lens[s] - q_len + t (all q_len tokens are already in the cache,
+ * seq_lens counts them) and attends positions 0 .. seq_lens[s] - q_len + t.  Per token this is the
+ * single-token decode of mlra_decode (the pages' step 2) with the length
+ * seq_lens[s] - (q_len - 1 - t) over sequence s's cache rows; the call runs dims->batch * q_len
+ * such decodes in one launch sequence (each reads its own prefix of the cache: q_len reads of it).
+ *   q_lat  [N, q_len, H, d_c], q_rope [N, q_len, H, d_R], contiguous, dtype as dims->dtype
+ *   out    [N, q_len, H, width] fp32; lse nullable [N, q_len, H, B]
+ *   dims   the caller's shapes with batch = N (not N * q_len)
+ *   workspace  at least mlra_workspace_size_multi(dims, q_len) bytes
+ * Everything else as mlra_decode.  A token whose length would be negative (seq_lens[s] < q_len - 1
+ * - t) raises MLRA_FLAG_BAD_LENGTH and gets an empty output.
+ * Errors as mlra_decode; MLRA_ERR_INVALID_ARG for q_len < 1. */
+mlra_status mlra_decode_multi(const void* q_lat, const void* q_rope, const void* c_kv,
+                              const void* k_rope, const int32_t* seq_lens,
+                              const int32_t* page_table, int q_len, int B,
+                              const mlra_scales* scales, float* out, float* lse,
+                              const mlra_dims* dims, void* workspace, size_t ws_bytes,
+                              mlra_stream_t stream);
+
+/* Workspace bytes for mlra_decode_multi with q_len query tokens per sequence (dims->batch = N). */
+mlra_status mlra_workspace_size_multi(const mlra_dims* dims, int q_len, size_t* bytes_host);
+
 /* mlra_decode for callers that cannot hand the library any device memory: hosts that own every
  * device allocation through their own pool and give plug-ins no allocator, or serving paths that
  * must not allocate at all.  It takes the same arguments as mlra_decode minus the workspace and

@@ -79,10 +79,13 @@ mlra_status check_dims(const mlra_dims* d, bool paged) {
   return MLRA_OK;
 }
 
-// Kernel variant and workspace layout.  sms == 0 requires dims->num_ranges > 0.
-mlra_status make_plan(const mlra_dims* d, bool paged, int sms, Plan* pl) {
+// Kernel variant and workspace layout.  sms == 0 requires dims->num_ranges > 0.  With q_len > 1
+// query tokens per sequence the plan covers d->batch * q_len virtual sequences (virtual_len).
+mlra_status make_plan(const mlra_dims* d, bool paged, int sms, Plan* pl, int q_len = 1) {
   mlra_status st = check_dims(d, paged);
   if (st != MLRA_OK) return st;
+  if (q_len < 1 || (int64_t)d->batch * q_len > INT_MAX / 2) return MLRA_ERR_INVALID_ARG;
+  const int64_t Nv = (int64_t)d->batch * q_len;
   const int B = d->num_branches, dblk = d->d_latent / B;
   const int dk = dblk <= 64 ? 64 : dblk <= 128 ? 128 : dblk <= 256 ? 256 : 512;
   if (B * dk > 512) return MLRA_ERR_UNSUPPORTED;
@@ -101,16 +104,16 @@ mlra_status make_plan(const mlra_dims* d, bool paged, int sms, Plan* pl) {
     pl->R = sms / pl->n_groups > 0 ? sms / pl->n_groups : 1;
   }
   if ((int64_t)pl->R * pl->n_groups > INT_MAX / 2) return MLRA_ERR_INVALID_ARG;
-  pl->slots = (int64_t)pl->R + d->batch - 1;
+  pl->slots = (int64_t)pl->R + Nv - 1;
   pl->limit = paged ? d->max_pages_per_seq * d->page_size : d->max_seq_len;
   if (!paged) pl->limit = d->max_seq_len;
   else if (d->max_seq_len > 0 && d->max_seq_len < pl->limit) pl->limit = d->max_seq_len;
   pl->seg_cost = kSegmentCostTiles;
   // the plan's (virtual) tile prefix must fit int32
-  if ((int64_t)d->batch * ((pl->limit + pl->tile - 1) / pl->tile + pl->seg_cost) > INT_MAX)
+  if (Nv * ((pl->limit + pl->tile - 1) / pl->tile + pl->seg_cost) > INT_MAX)
     return MLRA_ERR_INVALID_ARG;
 
-  const int64_t N = d->batch, H = d->heads;
+  const int64_t N = Nv, H = d->heads;
   size_t off = kAlign;  // status word + padding
   pl->self_plan = N <= kSelfPlanMaxSeqs;
   pl->off_scratch = off; off = align_up(off + 4 * (5 * (size_t)N + 2));
@@ -257,12 +260,15 @@ mlra_status mlra_decode(const void* q_lat, const void* q_rope, const void* c_kv,
                               lse, dims, workspace, ws_bytes, stream, nullptr, nullptr);
 }
 
-mlra_status mlra_decode_profiled(const void* q_lat, const void* q_rope, const void* c_kv,
-                                 const void* k_rope, const int32_t* seq_lens,
-                                 const int32_t* page_table, int B, const mlra_scales* scales,
-                                 float* out, float* lse, const mlra_dims* dims, void* workspace,
-                                 size_t ws_bytes, mlra_stream_t stream, mlra_event_t k1_begin,
-                                 mlra_event_t k1_end) {
+namespace {
+// The decode call: q_len query tokens per caller sequence (1: single-token decode), run as
+// dims->batch * q_len virtual sequences (virtual_len).
+mlra_status decode_impl(const void* q_lat, const void* q_rope, const void* c_kv,
+                        const void* k_rope, const int32_t* seq_lens, const int32_t* page_table,
+                        int B, const mlra_scales* scales, float* out, float* lse,
+                        const mlra_dims* dims, void* workspace, size_t ws_bytes,
+                        mlra_stream_t stream, mlra_event_t k1_begin, mlra_event_t k1_end,
+                        int q_len) {
   if (!q_lat || !q_rope || !c_kv || !k_rope || !seq_lens || !scales || !out || !dims)
     return MLRA_ERR_INVALID_ARG;
   if (B != dims->num_branches) return MLRA_ERR_INVALID_ARG;
@@ -277,7 +283,7 @@ mlra_status mlra_decode_profiled(const void* q_lat, const void* q_rope, const vo
     if (st != MLRA_OK) return st;
   }
   Plan pl;
-  st = make_plan(dims, paged, sms, &pl);
+  st = make_plan(dims, paged, sms, &pl, q_len);
   if (st != MLRA_OK) return st;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || ws_bytes < pl.total)
     return MLRA_ERR_WORKSPACE;
@@ -294,7 +300,7 @@ mlra_status mlra_decode_profiled(const void* q_lat, const void* q_rope, const vo
   RangeInfo* ranges = reinterpret_cast<RangeInfo*>(ws + pl.off_ranges);
   SegDesc* segs = reinterpret_cast<SegDesc*>(ws + pl.off_segs);
   SeqInfo* seqs = reinterpret_cast<SeqInfo*>(ws + pl.off_seqs);
-  const int N = dims->batch, H = dims->heads, dblk = dims->d_latent / B;
+  const int N = dims->batch * q_len, H = dims->heads, dblk = dims->d_latent / B;  // virtual
   const int64_t rows = dims->cache_rows;
 
   const void* kq = q_lat; const void* kqr = q_rope; const void* kc = c_kv; const void* kkr = k_rope;
@@ -352,7 +358,7 @@ mlra_status mlra_decode_profiled(const void* q_lat, const void* q_rope, const vo
   if (!pl.self_plan) {
     PrepParams pp;
     pp.seq_lens = seq_lens; pp.N = N; pp.limit = pl.limit; pp.tile = pl.tile; pp.num_ranges = pl.R;
-    pp.seg_cost = pl.seg_cost; pp.scratch = plan_scratch;
+    pp.seg_cost = pl.seg_cost; pp.scratch = plan_scratch; pp.q_per_seq = q_len;
     pp.ranges = ranges; pp.segs = segs; pp.seqs = seqs;
     pp.flags = cta_flags + grid;
     pp.out = out; pp.lse = lse; pp.H = H; pp.B = B; pp.out_width = out_width;
@@ -373,6 +379,7 @@ mlra_status mlra_decode_profiled(const void* q_lat, const void* q_rope, const vo
   p.max_seq_len = dims->max_seq_len;
   p.n_pages = paged ? rows / dims->page_size : 0;
   p.oob_row = static_cast<int>(rows);
+  p.q_per_seq = q_len;
   p.scale_log2 = scales->softmax_scale * 1.4426950408889634f;
   p.gamma = scales->branch_scale;
   p.write_final = summed ? 0 : 1;
@@ -401,6 +408,44 @@ mlra_status mlra_decode_profiled(const void* q_lat, const void* q_rope, const vo
   cp.final_written = summed ? 0 : 1;
   cp.gamma = scales->branch_scale;
   if (launch_combine(cp, s) != cudaSuccess) return MLRA_ERR_CUDA;
+  return MLRA_OK;
+}
+}  // namespace
+
+mlra_status mlra_decode_profiled(const void* q_lat, const void* q_rope, const void* c_kv,
+                                 const void* k_rope, const int32_t* seq_lens,
+                                 const int32_t* page_table, int B, const mlra_scales* scales,
+                                 float* out, float* lse, const mlra_dims* dims, void* workspace,
+                                 size_t ws_bytes, mlra_stream_t stream, mlra_event_t k1_begin,
+                                 mlra_event_t k1_end) {
+  return decode_impl(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table, B, scales, out, lse, dims,
+                     workspace, ws_bytes, stream, k1_begin, k1_end, 1);
+}
+
+mlra_status mlra_decode_multi(const void* q_lat, const void* q_rope, const void* c_kv,
+                              const void* k_rope, const int32_t* seq_lens,
+                              const int32_t* page_table, int q_len, int B,
+                              const mlra_scales* scales, float* out, float* lse,
+                              const mlra_dims* dims, void* workspace, size_t ws_bytes,
+                              mlra_stream_t stream) {
+  if (q_len < 1) return MLRA_ERR_INVALID_ARG;
+  return decode_impl(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table, B, scales, out, lse, dims,
+                     workspace, ws_bytes, stream, nullptr, nullptr, q_len);
+}
+
+mlra_status mlra_workspace_size_multi(const mlra_dims* dims, int q_len, size_t* bytes_host) {
+  if (!dims || !bytes_host || q_len < 1) return MLRA_ERR_INVALID_ARG;
+  const bool paged = dims->max_pages_per_seq > 0 && dims->page_size > 0;
+  int sms = 0;
+  if (dims->num_ranges == 0) {
+    mlra_status st;
+    sms = device_sm_count(&st);
+    if (st != MLRA_OK) return st;
+  }
+  Plan pl;
+  mlra_status st = make_plan(dims, paged, sms, &pl, q_len);
+  if (st != MLRA_OK) return st;
+  *bytes_host = pl.total;
   return MLRA_OK;
 }
 

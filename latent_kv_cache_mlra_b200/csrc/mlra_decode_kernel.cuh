@@ -147,7 +147,10 @@ __device__ __noinline__ int plan_in_kernel(const DecodeParams& p, int range, int
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const int i = 32 * c + lane;
-      L[c] = i < N ? __ldcg(p.seq_lens + i) : 0;
+      L[c] = i < N ? (p.q_per_seq == 1 ? __ldcg(p.seq_lens + i)
+                                         : __ldcg(p.seq_lens + i / p.q_per_seq) -
+                                               (p.q_per_seq - 1 - i % p.q_per_seq))
+                   : 0;
     }
     int carry_t = 0, carry_v = 0;
 #pragma unroll
@@ -326,7 +329,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (p.self_plan && warp == 0 && 32 * lane < p.N)
+  if (p.self_plan && warp == 0 && 32 * lane < p.N / p.q_per_seq)  // the caller's lengths
     prefetch_l2(p.seq_lens + 32 * lane);  // warms L2 and the TLB for the plan below
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&tm_q);
@@ -382,7 +385,8 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           const int t64 = (seg.tile0 + i) * C::TB + l;
           rows[l] = (t64 * kTile < L)
                         ? tile_row(p.page_table, p.max_pages, p.page_size, p.max_seq_len, p.n_pages,
-                                   p.oob_row, seg.seq, t64, lane == 0 ? flags : nullptr)
+                                   p.oob_row, seg.seq / p.q_per_seq, t64,
+                                   lane == 0 ? flags : nullptr)
                         : p.oob_row;
         }
         const int st = it % NS;

@@ -25,9 +25,19 @@ struct alignas(16) SegDesc {
 };
 struct alignas(8) SeqInfo { int32_t r0, r1; };
 
+// Several query tokens per sequence (a speculative or chunked-prefill step): the decode runs
+// N = (caller sequences) x q_per_seq virtual sequences, v = s q_per_seq + t for token t of caller
+// sequence s, over s's cache rows; token t is at position seq_lens[s] - q_per_seq + t and sees the
+// positions up to its own (causal), so v's length is seq_lens[s] - (q_per_seq - 1 - t).
+__host__ __device__ inline int virtual_len(const int32_t* seq_lens, int v, int q_per_seq) {
+  if (q_per_seq == 1) return seq_lens[v];
+  return seq_lens[v / q_per_seq] - (q_per_seq - 1 - v % q_per_seq);
+}
+
 struct PrepParams {
-  const int32_t* seq_lens;    // caller lengths [N]
+  const int32_t* seq_lens;    // caller lengths [N / q_per_seq]
   int N, limit, tile, num_ranges;
+  int q_per_seq;              // query tokens per caller sequence (virtual_len)
   int seg_cost;               // tiles a sequence start costs a CTA (plan balance)
   int32_t* scratch;           // [5 N + 2] plan arrays when N is too large for shared memory
   RangeInfo* ranges;          // [num_ranges]
@@ -63,6 +73,8 @@ struct DecodeParams {
   int page_size, max_pages, max_seq_len;
   int64_t n_pages;            // pages in the pool (paged layout)
   int oob_row;                // tile row used for an invalid page id (reads zeros)
+  int q_per_seq;              // query tokens per caller sequence: virtual sequence v reads the
+                              // cache rows of caller sequence v / q_per_seq (virtual_len)
   float scale_log2;           // softmax_scale * log2(e)
   float gamma;                // branch_scale
   int write_final;            // whole-sequence segments write `out` directly

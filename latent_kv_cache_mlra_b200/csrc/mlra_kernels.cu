@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(1024) mlra_prep_kernel(const PrepParams p) {
     const int i = b0 + tid;
     int x[2] = {0, 0};  // tiles, virtual tiles
     if (i < N) {
-      int L = p.seq_lens[i];
+      int L = virtual_len(p.seq_lens, i, p.q_per_seq);
       if (L < 0 || L > p.limit) {
         atomicOr(&flags, kFlagBadLength);
         L = L < 0 ? 0 : p.limit;

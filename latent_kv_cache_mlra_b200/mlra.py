@@ -28,7 +28,8 @@ EXPORTS = ("mlra_workspace_size", "mlra_decode", "mlra_decode_profiled", "mlra_q
            "mlra_decode_static_scratch",
            "mlra_read_status", "mlra_debug_resolve_rows", "mlra_plan_host",
            "mlra_plan_segments_host", "mlra_project", "mlra_pack_wuv", "mlra_absorb",
-           "mlra_pack_wuk", "mlra_rope_append", "mlra_status_string", "mlra_version")
+           "mlra_pack_wuk", "mlra_rope_append", "mlra_decode_multi", "mlra_workspace_size_multi",
+           "mlra_status_string", "mlra_version")
 
 
 class Dims(ctypes.Structure):
@@ -90,6 +91,11 @@ def lib() -> ctypes.CDLL:
         L.mlra_pack_wuk.argtypes = L.mlra_pack_wuv.argtypes
         L.mlra_rope_append.argtypes = [vp, vp, vp, vp, vp, ctypes.POINTER(Dims), vp, vp, vp,
                                        ctypes.c_double, vp, vp]
+        L.mlra_decode_multi.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int,
+                                        ctypes.POINTER(Scales), vp, vp, ctypes.POINTER(Dims), vp,
+                                        ctypes.c_size_t, vp]
+        L.mlra_workspace_size_multi.argtypes = [ctypes.POINTER(Dims), ctypes.c_int,
+                                                ctypes.POINTER(ctypes.c_size_t)]
         L.mlra_status_string.argtypes = [ctypes.c_int]
         L.mlra_status_string.restype = ctypes.c_char_p
         L.mlra_version.argtypes = []
@@ -97,7 +103,8 @@ def lib() -> ctypes.CDLL:
                   "mlra_decode_static_scratch",
                   "mlra_read_status", "mlra_debug_resolve_rows", "mlra_plan_host",
                   "mlra_plan_segments_host", "mlra_project", "mlra_pack_wuv", "mlra_absorb",
-                  "mlra_pack_wuk", "mlra_rope_append"):
+                  "mlra_pack_wuk", "mlra_rope_append", "mlra_decode_multi",
+                  "mlra_workspace_size_multi"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -274,6 +281,47 @@ def decode(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table=None, *, num_branch
                              _ptr(page_table), num_branches, ctypes.byref(scales), _ptr(out),
                              _ptr(lse), ctypes.byref(dims), _ptr(workspace), workspace.numel(),
                              ctypes.c_void_p(st)), "mlra_decode")
+    return out, lse
+
+
+def workspace_size_multi(dims: Dims, q_len: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().mlra_workspace_size_multi(ctypes.byref(dims), q_len, ctypes.byref(n)),
+           "mlra_workspace_size_multi")
+    return n.value
+
+
+def decode_multi(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table=None, *, num_branches: int,
+                 softmax_scale: float, branch_scale: Optional[float] = None, out_mode="branches",
+                 max_seq_len=None, page_size=0, with_lse=False, out=None, lse=None,
+                 workspace=None, num_ranges=0, stream=None):
+    """Decode for the q newest tokens of every sequence through ``mlra_decode_multi``.
+
+    q_lat [N, q, H, d_c], q_rope [N, q, H, d_R] contiguous: token t of sequence s sits at position
+    seq_lens[s] - q + t (all q tokens already in the cache) and attends positions up to its own.
+    Returns (out [N, q, H, width], lse [N, q, H, B] or None)."""
+    N, q, H, d_c = q_lat.shape
+    gamma = 1.0 / num_branches if branch_scale is None else branch_scale
+    dims = dims_for(q_lat[:, 0], q_rope[:, 0], c_kv, k_rope, seq_lens, page_table, num_branches,
+                    max_seq_len=max_seq_len, page_size=page_size, out_mode=out_mode,
+                    num_ranges=num_ranges)
+    if not (q_lat.is_contiguous() and q_rope.is_contiguous()):
+        raise ValueError("decode_multi: contiguous queries expected")
+    width = d_c if out_mode == "branches" else d_c // num_branches
+    dev = q_lat.device
+    if out is None:
+        out = torch.empty(N, q, H, width, dtype=torch.float32, device=dev)
+    if with_lse and lse is None:
+        lse = torch.empty(N, q, H, num_branches, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(workspace_size_multi(dims, q), dtype=torch.uint8, device=dev)
+    st = stream if stream is not None else torch.cuda.current_stream(dev).cuda_stream
+    scales = Scales(softmax_scale, gamma)
+    _check(lib().mlra_decode_multi(_ptr(q_lat), _ptr(q_rope), _ptr(c_kv), _ptr(k_rope),
+                                   _ptr(seq_lens), _ptr(page_table), q, num_branches,
+                                   ctypes.byref(scales), _ptr(out), _ptr(lse), ctypes.byref(dims),
+                                   _ptr(workspace), workspace.numel(), ctypes.c_void_p(st)),
+           "mlra_decode_multi")
     return out, lse
 
 
