@@ -377,6 +377,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         tma_load_3d(sQ + C::NCB * C::BOX, &tm_qr, bar_q_full, 0, 0, seg.seq);
       }
       __syncwarp();
+      const int cache_seq = seg.seq / p.q_per_seq;  // whose cache rows (once per segment)
       for (int i = 0; i < seg.ntiles; ++i, ++it) {
         // cache rows of the tile's 64-position sub-boxes (past the sequence end: zeros)
         int rows[C::TB];
@@ -385,8 +386,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           const int t64 = (seg.tile0 + i) * C::TB + l;
           rows[l] = (t64 * kTile < L)
                         ? tile_row(p.page_table, p.max_pages, p.page_size, p.max_seq_len, p.n_pages,
-                                   p.oob_row, seg.seq / p.q_per_seq, t64,
-                                   lane == 0 ? flags : nullptr)
+                                   p.oob_row, cache_seq, t64, lane == 0 ? flags : nullptr)
                         : p.oob_row;
         }
         const int st = it % NS;
