@@ -526,7 +526,8 @@ def run_stage(args):
       absorb:  step 1 (query absorption of W^UK) alone, W^UK evicted from L2 each call;
       layer:   one attention layer's whole decode step -- step 1, the new token's RoPE and cache
                append, step 2 (the path's two kernels) and step 3 -- with L2 evicted before each
-               step (and, for reference, back to back).
+               step (and, for reference, back to back);
+      multi:   step 2 for --q-len query tokens per sequence (mlra_decode_multi).
     Weights are N(0, 1/fan-in) bf16 draws, packed once.  Prints one JSON line."""
     from latent_kv_cache_mlra_b200 import mlra
 
@@ -577,6 +578,42 @@ def run_stage(args):
                                                          PROJECT_SOURCES),
                              "tensor_tflops": flops / (ms * 1e-3) / 1e12},
                 "l2": "L2 flushed (read of 2x L2) before each launch"}
+    elif args.stage == "multi":
+        # q query tokens per sequence (speculative / chunked-prefill step), causal among them
+        q = args.q_len
+        gq = torch.Generator().manual_seed(w.seed + 78)
+        qm = torch.randn(N, q, H, d_c, generator=gq).to(torch.bfloat16).to(dev)
+        qrm = torch.randn(N, q, H, d_R, generator=gq).to(torch.bfloat16).to(dev)
+        dims = mlra.dims_for(qm[:, 0], qrm[:, 0], c, kr, lens, pt, w.num_branches,
+                             max_seq_len=inp.max_seq_len, page_size=w.page_size)
+        ws = torch.empty(mlra.workspace_size_multi(dims, q), dtype=torch.uint8, device=dev)
+        outm = torch.empty(N, q, H, d_c, dtype=torch.float32, device=dev)
+        body = lambda: mlra.decode_multi(qm, qrm, c, kr, lens, pt, num_branches=w.num_branches,  # noqa: E731
+                                         softmax_scale=w.sigma, branch_scale=w.gamma,
+                                         max_seq_len=inp.max_seq_len, page_size=w.page_size,
+                                         out=outm, workspace=ws)
+        for _ in range(args.warmup):
+            body()
+        big = cache_bytes(inp) > L2_BYTES
+        with ClockSampler(0) as clk:
+            ms = graph_time(body, args.steps, pre=None if big else evict)
+        once = cache_bytes(inp)  # the cache read once: what a fused multi-token kernel needs
+        token_bytes = once // max(1, int(inp.seq_lens.sum()))
+        read = sum(max(0, int(L) - (q - 1 - t)) for L in inp.seq_lens.tolist()
+                   for t in range(q)) * token_bytes
+        gbs = once / (ms * 1e-3) / 1e9
+        line = {"metric": f"multi-token decode ({q} query tokens per sequence) query tokens/s",
+                "value": N * q / (ms * 1e-3), "unit": "tokens/s", "higher_is_better": True,
+                "ms_per_step": ms, "q_len": q,
+                "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                             "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                             "kernel": "mlra_decode_kernel (whole call)",
+                             "algorithmic_bytes_per_launch": once,
+                             "bytes_read_per_step": read,
+                             "note": "algorithmic = the cache read once; this path reads each "
+                                     "token's causal prefix, about q times the cache"},
+                "l2": "inputs larger than L2" if big else
+                      "L2 flushed (read of 2x L2) before each step, outside the timed region"}
     else:  # layer
         q_rope_in = torch.randn(N, H, d_R, generator=g).to(dev)
         k_new, c_new = torch.randn(N, d_R, generator=g).to(dev), torch.randn(N, d_c, generator=g).to(dev)
@@ -627,9 +664,13 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--stage", choices=["decode", "project", "absorb", "layer"], default="decode",
+    ap.add_argument("--q-len", type=int, default=2,
+                    help="query tokens per sequence for --stage multi")
+    ap.add_argument("--stage", choices=["decode", "project", "absorb", "layer", "multi"],
+                    default="decode",
                     help="decode: the attention path (the default line); project / absorb: step 3 "
-                         "/ step 1 alone; layer: steps 1-3 with RoPE and the cache append")
+                         "/ step 1 alone; layer: steps 1-3 with RoPE and the cache append; multi: "
+                         "--q-len query tokens per sequence")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
