@@ -79,7 +79,7 @@ typedef struct {
 
 typedef struct {
   int batch;              /* N >= 1 sequences, one query token each */
-  int heads;              /* H, 1..64 */
+  int heads;              /* H, 1..128 (groups of 64 heads per CTA) */
   int num_branches;       /* B >= 1, divides d_latent */
   int d_latent;           /* d_c = B * d_blk, <= 512 */
   int d_rope;             /* d_R, 1..64 */

@@ -29,7 +29,7 @@ struct Plan {
   Variant variant = kV128;
   int dblk_k = 0;      // padded branch width seen by the kernel
   int tile = 0;        // KV positions per tile
-  int n_groups = 1;    // CTAs per range (one per branch)
+  int n_groups = 1;    // CTAs per range (one per branch and 64-head group)
   int dck = 0;         // B * dblk_k
   int R = 0;           // work ranges
   int64_t slots = 0;   // partial slots = R + N - 1
@@ -72,7 +72,7 @@ mlra_status check_dims(const mlra_dims* d, bool paged) {
   } else {
     if ((int64_t)d->batch * d->max_seq_len > d->cache_rows) return MLRA_ERR_INVALID_ARG;
   }
-  if (d->heads > 64 || d->d_latent > 512 || d->d_rope > 64) return MLRA_ERR_UNSUPPORTED;
+  if (d->heads > kMaxHeads || d->d_latent > 512 || d->d_rope > 64) return MLRA_ERR_UNSUPPORTED;
   if (paged && d->page_size % kTile != 0) return MLRA_ERR_UNSUPPORTED;
   if (d->cache_rows > (int64_t)INT_MAX - 2 * kTile) return MLRA_ERR_UNSUPPORTED;
   if (d->num_branches > 64) return MLRA_ERR_UNSUPPORTED;
@@ -96,7 +96,8 @@ mlra_status make_plan(const mlra_dims* d, bool paged, int sms, Plan* pl, int q_l
   pl->dblk_k = dk;
   pl->variant = dk == 64 ? kV64 : dk == 128 ? kV128 : dk == 256 ? kV256 : kV512;
   pl->tile = variant_tile(pl->variant);
-  pl->n_groups = B;
+  pl->n_groups = B * ((d->heads + 63) / 64);  // CTAs per range: (64-head group, branch)
+  if (pl->n_groups > 148) return MLRA_ERR_UNSUPPORTED;
   pl->dck = B * dk;
   if (d->num_ranges > 0) pl->R = d->num_ranges;
   else {

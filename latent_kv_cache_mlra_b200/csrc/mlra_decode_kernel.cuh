@@ -5,9 +5,10 @@
 // scores of the absorbed query block against latent block c_b plus the shared RoPE term,
 // an online softmax of its own over positions, and the probability-weighted sum of c_b.
 //
-// One persistent CTA per (work range, branch).  A work range is a contiguous run of KV tiles
-// (T positions each) of the batch (see mlra_plan.cuh).  Heads are the M = 64 rows of every
-// tcgen05 MMA, the tile's T positions the N of the score product:
+// One persistent CTA per (work range, branch, group of 64 heads).  A work range is a contiguous
+// run of KV tiles (T positions each) of the batch (see mlra_plan.cuh).  A group's 64 heads are
+// the M = 64 rows of every tcgen05 MMA (more than 64 heads: several groups read the same tiles,
+// which mostly meet in L2), the tile's T positions the N of the score product:
 //   score:  S[64 x T]     = Q~_b[64 x d] . C_b^T  +  Q^R[64 x 64] . K^R^T     (TMEM, fp32)
 //   output: O[64 x d]    += P[64 x T] . C_b[T x d]                           (TMEM, fp32)
 // The RoPE product is accumulated into the same score tile by the MMA chain.  An MMA costs at
@@ -133,10 +134,10 @@ constexpr int kDecodeThreads = 224;
 // lane and lane + 32: it clamps their lengths, scans the real and virtual tile prefixes
 // (mlra_plan.cuh) across the warp, finds the sequence holding each of the range's two virtual
 // boundaries with one ballot, and lets every sequence that overlaps the range write its own
-// segment at its rank in the warp.  The CTAs of branch 0 also record, for the combine kernel, the
+// segment at its rank in the warp.  The CTAs of group 0 also record, for the combine kernel, the
 // ranges holding each sequence's first and last tile; CTA 0 writes the records and outputs of
 // empty sequences.  Returns the segment count.
-__device__ __noinline__ int plan_in_kernel(const DecodeParams& p, int range, int branch,
+__device__ __noinline__ int plan_in_kernel(const DecodeParams& p, int range, int group,
                                            uint8_t* plan, uint32_t* flags) {
   int4* list = reinterpret_cast<int4*>(plan);                       // [kSelfPlanMaxSeqs]
   int32_t* lens = reinterpret_cast<int32_t*>(list + kSelfPlanMaxSeqs);
@@ -213,7 +214,7 @@ __device__ __noinline__ int plan_in_kernel(const DecodeParams& p, int range, int
           list[base + __popc(m & ((1u << lane) - 1u))] =
               make_int4(i, static_cast<int>(a - lo[c]), static_cast<int>(e - a),
                         L[c] | (whole ? (int32_t)0x80000000u : 0));
-          if (branch == 0) {
+          if (group == 0) {
             if (a == lo[c]) p.seqs[i].r0 = range;  // the sequence's first tile is in this range
             if (e == hi[c]) p.seqs[i].r1 = range;  // ... its last tile
           }
@@ -302,7 +303,9 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int range = blockIdx.x / p.n_groups;
-  const int branch = blockIdx.x % p.n_groups;
+  const int group = blockIdx.x % p.n_groups;  // (64-head group, branch) of this CTA
+  const int branch = group % p.B;
+  const int h0 = 64 * (group / p.B);          // first head of this CTA's group
   const uint64_t tmo = p.timeout_ns;
   // The combine kernel may be scheduled now; it waits for this grid before reading anything.
   pdl_launch_dependents();
@@ -350,7 +353,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const int4* seg_list;
   int seg_count;
   if (p.self_plan) {
-    seg_count = plan_in_kernel(p, range, branch, smem + C::OFF_PLAN, flags);
+    seg_count = plan_in_kernel(p, range, group, smem + C::OFF_PLAN, flags);
     seg_list = reinterpret_cast<const int4*>(smem + C::OFF_PLAN);
   } else {
     const int2 r2 = __ldcg(reinterpret_cast<const int2*>(p.ranges + range));
@@ -373,8 +376,8 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         mbar_arrive_expect_tx(bar_q_full, C::QBYTES);
 #pragma unroll
         for (int k = 0; k < C::NCB; ++k)
-          tma_load_3d(sQ + k * C::BOX, &tm_q, bar_q_full, col0 + 64 * k, 0, seg.seq);
-        tma_load_3d(sQ + C::NCB * C::BOX, &tm_qr, bar_q_full, 0, 0, seg.seq);
+          tma_load_3d(sQ + k * C::BOX, &tm_q, bar_q_full, col0 + 64 * k, h0, seg.seq);
+        tma_load_3d(sQ + C::NCB * C::BOX, &tm_qr, bar_q_full, 0, h0, seg.seq);
       }
       __syncwarp();
       const int cache_seq = seg.seq / p.q_per_seq;  // whose cache rows (once per segment)
@@ -508,7 +511,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   } else {
     // ------------------------------------------------------------------ softmax warps 0-3
     const int q = lane >> 4;                   // which half of the row's columns
-    const int h = 16 * warp + (lane & 15);     // head
+    const int h = h0 + 16 * warp + (lane & 15);  // head
     const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
     uint8_t* stg = smem + C::OFF_STG + warp * C::STG_BYTES;  // this warp's store staging box
     const uint32_t stg_u = smem_u32(stg);
@@ -631,7 +634,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         scale = 1.f;
         ncols_out = DBLK;
       }
-      if (16 * warp >= p.H) {
+      if (h0 + 16 * warp >= p.H) {
         // no head of this warp exists: nothing to store
       } else if (!to_final || p.tma_out) {
         // Through shared memory and the TMA: each [16 heads x 32 columns] box is staged in the
@@ -671,7 +674,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           __syncwarp();
           if (lane == 0) {
             for (int col = 0; col < ncols_out && col < DBLK; col += 32)
-              tma_store_3d(map, smem_u32(ring + (col / 32) * C::STG_BYTES), x0 + col, 16 * warp, z);
+              tma_store_3d(map, smem_u32(ring + (col / 32) * C::STG_BYTES), x0 + col, h0 + 16 * warp, z);
             bulk_commit();
           }
         } else {
@@ -698,7 +701,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 fence_proxy_async_smem();  // the staged box is read by the bulk copy (async proxy)
                 __syncwarp();
                 if (lane == 0) {
-                  tma_store_3d(map, stg_u, x0 + col, 16 * warp, z);
+                  tma_store_3d(map, stg_u, x0 + col, h0 + 16 * warp, z);
                   bulk_commit();
                 }
                 stg_pending = true;

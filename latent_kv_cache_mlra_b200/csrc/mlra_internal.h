@@ -12,6 +12,7 @@ constexpr uint32_t kFlagBadPage = 0x2u;
 constexpr uint32_t kFlagBadLength = 0x4u;
 // Up to this many sequences the decode kernel plans its work range itself (no prep kernel).
 constexpr int kSelfPlanMaxSeqs = 64;
+constexpr int kMaxHeads = 128;        // query heads: groups of 64 per CTA
 constexpr int kMaxRopePairs = 32;     // d_rope <= 64
 
 // The split plan as the prep kernel writes it for the decode and combine kernels.
@@ -68,7 +69,7 @@ struct DecodeParams {
   int d_blk_out;              // branch width of the caller's output
   int out_width;              // row width of out (d_latent)
   int dck;                    // latent width seen by the kernel (B * padded d_blk)
-  int n_groups;               // CTAs per work range (branch groups)
+  int n_groups;               // CTAs per work range: B x (64-head groups), group g = (g / B, g % B)
   int num_ranges;
   int page_size, max_pages, max_seq_len;
   int64_t n_pages;            // pages in the pool (paged layout)

@@ -295,7 +295,18 @@ def _sampled(name, seqs, heads, R=0):
     return out
 
 
+@pytest.mark.parametrize("B,heads,page_size", [(1, 128, 0), (4, 128, 0), (2, 96, 64), (1, 72, 0)])
+def test_head_groups(B, heads, page_size):
+    """More than 64 heads: one CTA per (range, branch, 64-head group); a partial last group."""
+    inp = small_inputs(B=B, heads=heads, lens=[300, 1, 129, 700], page_size=page_size, seed=71)
+    out, lse = run_gpu(inp)
+    ref, ref_lse = run_oracle(inp)
+    assert_close(out, ref, f"B={B} H={heads}")
+    assert_lse_close(lse, ref_lse, f"B={B} H={heads}")
+
+
 @pytest.mark.parametrize("name,seqs,heads", [
+    ("mla_h128_n8_l32k", [0, 7], [0, 63, 64, 127]),
     ("mlra4_n8_l32k", [0, 5, 7], [0, 17, 33, 63]),
     ("mla_n8_l32k", [1, 6], [2, 40, 63]),
     ("long_mlra4_l128k", [0], [0, 9, 31, 62]),

@@ -65,7 +65,7 @@ def test_workspace_size_layout():
     (dict(num_branches=3), mlra.MLRA_ERR_INVALID_ARG),          # 3 does not divide 512
     (dict(cache_rows=100), mlra.MLRA_ERR_INVALID_ARG),          # contiguous rows too few
     (dict(c_row_stride=100), mlra.MLRA_ERR_INVALID_ARG),        # stride below the width
-    (dict(heads=65), mlra.MLRA_ERR_UNSUPPORTED),
+    (dict(heads=129), mlra.MLRA_ERR_UNSUPPORTED),
     (dict(d_latent=1024, num_branches=8), mlra.MLRA_ERR_UNSUPPORTED),
     (dict(d_rope=128, kr_row_stride=128), mlra.MLRA_ERR_UNSUPPORTED),
     (dict(page_size=32, max_pages_per_seq=1024), mlra.MLRA_ERR_UNSUPPORTED),
@@ -303,3 +303,12 @@ def test_rope_append_argument_errors_without_a_gpu():
     for name in ("q_in", "kr", "c", "q_out", "krc", "ckv"):
         assert call(mlra.make_dims(**good), **{name: ctypes.c_void_p(4104)}) == mlra.MLRA_ERR_UNSUPPORTED, name
     assert call(mlra.make_dims(**dict(good, cache_rows=100))) == mlra.MLRA_ERR_INVALID_ARG  # 2 x 64 rows
+
+
+def test_head_groups_in_the_plan():
+    """More than 64 heads: one CTA per (range, branch, 64-head group)."""
+    info = mlra.query_plan(dims(heads=128, num_branches=1))
+    assert info.ctas == info.num_ranges * 2
+    info4 = mlra.query_plan(dims(heads=96, num_branches=4))
+    assert info4.ctas == info4.num_ranges * 8
+    assert mlra.query_plan(dims(heads=64, num_branches=4)).ctas == 74 * 4

@@ -102,6 +102,10 @@ WORKLOADS = {
     "mlra4_tp4_shard_n8_l32k": Workload(
         name="mlra4_tp4_shard_n8_l32k", batch=8, heads=64, num_branches=1, d_latent=128,
         d_rope=64, seq_len=32768, seed=1006, alpha=math.sqrt(64 / 128), branch_scale=0.25),
+    # MLA with 128 query heads (DeepSeek-V3-like attention: latent 512, RoPE key 64, head dim 128).
+    "mla_h128_n8_l32k": Workload(
+        name="mla_h128_n8_l32k", batch=8, heads=128, num_branches=1, d_latent=512, d_rope=64,
+        seq_len=32768, seed=1007),
     "serving_mlra4_n64_paged": Workload(
         name="serving_mlra4_n64_paged", batch=64, heads=64, num_branches=4, d_latent=512,
         d_rope=64, seq_len=65536, min_seq_len=1024, ragged=True, page_size=64, seed=1005),
