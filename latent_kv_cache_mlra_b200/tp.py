@@ -56,7 +56,9 @@ class BranchShardStep:
     q_lat_b [N, H, d_c / B] and c_b [rows, d_c / B] are this device's blocks (``shard_queries``,
     ``shard_latent``); q_rope, k_rope, seq_lens and page_table are the full (replicated) arrays;
     w_uv_b [H, d_head, d_c / B] bf16 is ``shard_wuv``'s block, packed here once.  ``group`` is the
-    process group of the B branch devices (None: no reduction, the caller sums).
+    process group of the B branch devices (None: the default group); with ``reduce=False`` the
+    call returns this device's share and leaves the sum to the caller.  The returned tensor is the
+    step's output buffer, overwritten by the next call.
     """
 
     def __init__(self, q_lat_b, q_rope, c_b, k_rope, seq_lens, page_table, w_uv_b, *,
