@@ -296,6 +296,20 @@ def pin_golden_hand_worked(orc):
         assert np.allclose(summed[:, 0], f[f"summed_{tag}"], rtol=0, atol=1e-14), f"golden sum {tag}"
 
 
+def pin_golden_multi_token(orc):
+    """Hand-derived example of two new tokens attending causally
+    (tests/golden/hand_worked_multi_token.txt)."""
+    f = read_fixture("hand_worked_multi_token.txt")
+    c, kr = np.array(f["c_kv"], float), np.array(f["k_rope"], float)
+    q_rope = np.array(f["q_rope"], float)[None, :, None, :]            # [1, q, 1, d_R]
+    for tag in ("a", "b"):
+        q_lat = np.array(f[f"q_lat_{tag}"], float)[None, :, None, :]    # [1, q, 1, d_c]
+        out, lse = orc.decode_multi(q_lat, q_rope, c, kr, [c.shape[0]], None, 1, f["sigma"],
+                                    f["gamma"], max_seq_len=c.shape[0])
+        assert np.allclose(out[0, :, 0, 0], f[f"out_{tag}"], rtol=0, atol=1e-14), f"golden out {tag}"
+        assert np.allclose(lse[0, :, 0, 0], f[f"lse_{tag}"], rtol=0, atol=1e-14), f"golden lse {tag}"
+
+
 def pin_golden_rows(orc):
     """Hand-written page-resolution example (tests/golden/page_rows.txt)."""
     f = read_fixture("page_rows.txt")
@@ -460,5 +474,6 @@ ALL_PINS = [
     pin_position_permutation,
     pin_batch_rows_and_paging,
     pin_golden_hand_worked,
+    pin_golden_multi_token,
     pin_golden_rows,
 ]
