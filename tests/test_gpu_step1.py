@@ -13,7 +13,8 @@ pytestmark = pytest.mark.gpu
 BF16_REL = 2.0 ** -8   # one bf16 rounding of the result
 
 
-@pytest.mark.parametrize("N,H,d_head,d_latent", [(8, 64, 128, 512), (3, 5, 64, 192), (70, 2, 128, 256)])
+@pytest.mark.parametrize("N,H,d_head,d_latent", [(8, 64, 128, 512), (3, 5, 64, 192), (70, 2, 128, 256),
+                                                  (5, 32, 128, 512), (64, 64, 128, 512)])
 def test_absorb_matches_oracle(N, H, d_head, d_latent):
     g = torch.Generator().manual_seed(N + H)
     q = torch.randn(N, H, d_head, generator=g)
