@@ -25,7 +25,7 @@ table or the contiguous layout):
     p        = softmax over j of score          (independent per branch)
     out[s,h,b-block] = gamma * sum_j p[j] * c[row, b-block]
 
-Readings where the pages are silent (each listed in the design doc): one RoPE query
+Readings where the pages are silent: one RoPE query
 per head shared by all branches; ``sigma`` and ``gamma`` are parameters; the
 current token is already in the cache and no other mask applies; an empty
 sequence gives a zero output and ``lse = -inf``; ``lse = log sum_j exp(score_j)``
