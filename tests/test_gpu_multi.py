@@ -48,6 +48,20 @@ def test_multi_token_matches_oracle(q, lens, B, page_size):
     assert_lse_close(lse, ref_lse, f"q={q} lse")  # empty tokens: -inf on both sides
 
 
+def test_multi_token_through_the_prep_kernel():
+    """40 sequences x 2 tokens = 80 virtual sequences: more than the attention kernel plans itself,
+    so the prep kernel plans them (virtual lengths from the caller's lengths there too)."""
+    g = torch.Generator().manual_seed(91)
+    lens = (torch.randint(2, 400, (40,), generator=g)).tolist()
+    w, inp, q_lat, q_rope = multi_inputs(2, lens, B=4, heads=8, d_latent=256, seed=92)
+    out, lse = run_multi(w, inp, q_lat, q_rope)
+    torch.cuda.synchronize()
+    ref, ref_lse = oracle.decode_multi(q_lat, q_rope, inp.c_kv, inp.k_rope, inp.seq_lens, None,
+                                       w.num_branches, w.sigma, w.gamma, max_seq_len=inp.max_seq_len)
+    assert_close(out, ref, "80 virtual sequences")
+    assert_lse_close(lse, ref_lse, "80 virtual sequences lse")
+
+
 def test_short_sequence_is_flagged():
     """seq_lens[s] < q - 1 leaves some tokens with a negative length: MLRA_FLAG_BAD_LENGTH, and
     their outputs are empty (zeros); the other sequences are unaffected."""
