@@ -1,11 +1,13 @@
 /*
- * mlra.h -- C ABI of the B200 (sm_100a) MLRA single-token decode-attention library.
+ * mlra.h -- C ABI of the B200 (sm_100a) MLRA decode-attention library.
  *
  * The operation ("Multi-Head Low-Rank Attention", yunpan.plus page):
  *   section 1.3  MLA's efficient decode in three steps -- (1) absorb the key up-projection
  *                into the query, (2) run MQA-style attention of the absorbed query against the
- *                cached latent vectors, (3) apply the value up-projection.  This library is
- *                step 2.
+ *                cached latent vectors, (3) apply the value up-projection.  The core of this
+ *                library is step 2 (mlra_decode, below); steps 1 and 3 (mlra_absorb,
+ *                mlra_project), the new token's RoPE and cache append (mlra_rope_append) and
+ *                several query tokens per sequence (mlra_decode_multi) follow further down.
  *   section 2    the per-head NoPE key is a sum of B block projections of the latent, so the
  *                latent c_t splits into B column blocks c_{t,b} of width d_blk = d_latent / B;
  *   section 3.1  MLRA moves that sum behind the attention: every branch b runs its own
