@@ -312,3 +312,15 @@ def test_head_groups_in_the_plan():
     info4 = mlra.query_plan(dims(heads=96, num_branches=4))
     assert info4.ctas == info4.num_ranges * 8
     assert mlra.query_plan(dims(heads=64, num_branches=4)).ctas == 74 * 4
+
+
+def test_workspace_size_multi_covers_the_virtual_sequences():
+    """q query tokens per sequence plan N * q virtual sequences: the workspace equals that of a
+    single-token call with N * q sequences (paged, so the cache geometry is the same)."""
+    kw = dict(heads=64, num_branches=4, d_latent=512, d_rope=64, max_seq_len=4096,
+              cache_rows=64 * 1024, page_size=64, max_pages_per_seq=64, num_ranges=37)
+    d = mlra.make_dims(batch=8, **kw)
+    for q in (1, 2, 4):
+        assert mlra.workspace_size_multi(d, q) == mlra.workspace_size(mlra.make_dims(batch=8 * q, **kw))
+    with pytest.raises(mlra.MlraError):
+        mlra.workspace_size_multi(d, 0)
