@@ -122,7 +122,7 @@ mlra_status mlra_workspace_size(const mlra_dims* dims, size_t* bytes_host);
  * bf16 inputs with d_blk in {64, 128, 256, 512}, d_rope == 64, 16-byte aligned rows and
  * base pointers are read in place.  Other shapes (and fp32 inputs) are first repacked into
  * padded bf16 copies inside the workspace (a full copy of the cache per call: meant for
- * small problems).  MLRA_ERR_UNSUPPORTED: H > 64, d_latent > 512, d_rope > 64, page_size not
+ * small problems).  MLRA_ERR_UNSUPPORTED: H > 128, d_latent > 512, d_rope > 64, page_size not
  * a multiple of 64, misaligned bf16 rows.  Launch failures return MLRA_ERR_CUDA. */
 mlra_status mlra_decode(const void* q_lat, const void* q_rope, const void* c_kv, const void* k_rope,
                         const int32_t* seq_lens, const int32_t* page_table, int B,

@@ -331,8 +331,9 @@ def decode_static_scratch(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table=None
                           max_seq_len=None, page_size=0, out=None, lse=None, num_ranges=0,
                           stream=None):
     """``mlra_decode_static_scratch``: the decode without a workspace argument; the library uses
-    its built-in scratch array.  ``out`` / ``lse`` are allocated here when not given (the C entry
-    point itself allocates nothing).  Returns (out, lse or None)."""
+    its built-in scratch array.  ``out`` is allocated here when not given (the C entry point itself
+    allocates nothing); ``lse`` is written only when the caller passes an fp32 [N, H, B] tensor,
+    else no LSE is computed.  Returns (out, lse or None)."""
     gamma = 1.0 / num_branches if branch_scale is None else branch_scale
     dims = dims_for(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table, num_branches,
                     max_seq_len=max_seq_len, page_size=page_size, out_mode=out_mode,

@@ -2,9 +2,14 @@
 
 Some hosts own every device allocation through their own pool and offer plug-ins no allocator;
 some serving paths must not allocate at all.  This entry point takes no workspace and runs the
-decode on a scratch array built into the library.  Called here through the C ABI, twice in a row
-(the array keeps the previous call's contents), it must give what mlra_decode gives with a
-caller workspace, within the parity tolerance of the GPU tests.  The file is named to run last.
+decode on a scratch array built into the library, which every call shares and which keeps the
+previous call's contents.
+
+Called here through the C ABI several times in a row with problems of different shapes (a small
+contiguous batch planned inside the attention kernel, then 80 ragged paged sequences planned by
+the prep kernel, then the first problem again over the scratch the second one left), each result
+must match the CPU oracle within the parity tolerance of the GPU tests, and also what mlra_decode
+gives with a caller workspace.  The file is named to run last.
 """
 import ctypes
 
@@ -12,6 +17,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import workloads
 from latent_kv_cache_mlra_b200 import mlra
 
@@ -20,11 +26,21 @@ pytestmark = pytest.mark.gpu
 MAX_REL, MEAN_ABS = 1e-2, 2e-3
 
 
-def _close(a, b):
-    a, b = a.detach().cpu().double().numpy(), b.detach().cpu().double().numpy()
+def _close(a, b, what):
+    a = a.detach().cpu().double().numpy() if hasattr(a, "detach") else np.asarray(a)
+    b = b.detach().cpu().double().numpy() if hasattr(b, "detach") else np.asarray(b)
+    assert a.shape == b.shape, (what, a.shape, b.shape)
+    assert np.isfinite(a).all(), f"{what}: non-finite output"
     err = np.abs(a - b)
-    assert np.isfinite(a).all()
-    assert err.max() <= MAX_REL * max(np.abs(b).max(), 1e-30) and err.mean() <= MEAN_ABS
+    assert err.max() <= MAX_REL * max(np.abs(b).max(), 1e-30), f"{what}: max err {err.max():.3e}"
+    assert err.mean() <= MEAN_ABS, f"{what}: mean err {err.mean():.3e}"
+
+
+def _lse_close(a, b, what):
+    a = a.detach().cpu().double().numpy()
+    fin = np.isfinite(b)
+    assert (np.isneginf(a) == np.isneginf(b)).all(), f"{what}: -inf pattern"
+    assert (np.abs(a[fin] - b[fin]) <= 1e-3 + 1e-4 * np.abs(b[fin])).all(), what
 
 
 def _call(lib, dev, w, dims, out, lse):
@@ -39,25 +55,50 @@ def _call(lib, dev, w, dims, out, lse):
         ctypes.byref(dims), ctypes.c_void_p(st))
 
 
-@pytest.mark.parametrize("paged", [False, True])
-def test_static_scratch_matches_workspace_entry_point(paged):
-    w = workloads.small(batch=5, seq_len=3000, ragged=True, min_seq_len=1,
-                        page_size=64 if paged else 0, seed=31)
-    inp = workloads.make_inputs(w)
-    dev = [t.cuda() for t in (inp.q_lat, inp.q_rope, inp.c_kv, inp.k_rope, inp.seq_lens)]
-    dev.append(None if inp.page_table is None else inp.page_table.cuda())
-    ref, ref_lse = mlra.decode(*dev, num_branches=w.num_branches, softmax_scale=w.sigma,
-                               branch_scale=w.gamma, max_seq_len=inp.max_seq_len,
-                               page_size=w.page_size, with_lse=True)
-    dims = mlra.dims_for(*dev, w.num_branches, max_seq_len=inp.max_seq_len, page_size=w.page_size)
-    lib = mlra.lib()
-    for _ in range(2):  # two calls in a row share the built-in scratch
-        out = torch.full_like(ref, float("nan"))
-        lse = torch.full_like(ref_lse, float("nan"))
-        assert _call(lib, dev, w, dims, out, lse) == mlra.MLRA_OK
+class _Problem:
+    """One decode problem: device inputs, the oracle's answer and mlra_decode's answer."""
+
+    def __init__(self, w, seq_lens=None):
+        self.w = w
+        inp = workloads.make_inputs(w, seq_lens=seq_lens)
+        self.inp = inp
+        self.dev = [t.cuda() for t in (inp.q_lat, inp.q_rope, inp.c_kv, inp.k_rope, inp.seq_lens)]
+        self.dev.append(None if inp.page_table is None else inp.page_table.cuda())
+        self.ref, self.ref_lse = oracle.decode(
+            inp.q_lat, inp.q_rope, inp.c_kv, inp.k_rope, inp.seq_lens, inp.page_table,
+            w.num_branches, w.sigma, w.gamma, page_size=w.page_size, max_seq_len=inp.max_seq_len)
+        self.ws_out, self.ws_lse = mlra.decode(
+            *self.dev, num_branches=w.num_branches, softmax_scale=w.sigma, branch_scale=w.gamma,
+            max_seq_len=inp.max_seq_len, page_size=w.page_size, with_lse=True)
+        self.dims = mlra.dims_for(*self.dev, w.num_branches, max_seq_len=inp.max_seq_len,
+                                  page_size=w.page_size)
+
+    def check(self, lib, what):
+        out = torch.full_like(self.ws_out, float("nan"))
+        lse = torch.full_like(self.ws_lse, float("nan"))
+        assert _call(lib, self.dev, self.w, self.dims, out, lse) == mlra.MLRA_OK
         torch.cuda.synchronize()
-        _close(out, ref)
-        _close(lse, ref_lse)
+        _close(out, self.ref, f"{what} vs oracle")
+        _lse_close(lse, self.ref_lse, f"{what} lse vs oracle")
+        _close(out, self.ws_out, f"{what} vs mlra_decode")
+        _lse_close(lse, self.ws_lse, f"{what} lse vs mlra_decode")
+
+
+def test_static_scratch_consecutive_calls_of_different_shapes():
+    small = _Problem(workloads.small(batch=5, seq_len=3000, ragged=True, min_seq_len=1, seed=31))
+    # more than 64 sequences: the prep kernel plans the call; paged, ragged, one empty sequence
+    lens = workloads.draw_seq_lens(
+        workloads.small(batch=80, seq_len=900, ragged=True, min_seq_len=1, seed=32),
+        torch.Generator().manual_seed(32))
+    lens[17] = 0
+    big = _Problem(workloads.small(batch=80, seq_len=900, ragged=True, min_seq_len=1,
+                                   page_size=64, seed=33), seq_lens=lens)
+    assert mlra.query_plan(big.dims).launches == 3  # prep kernel in the call
+
+    lib = mlra.lib()
+    small.check(lib, "first call (5 contiguous sequences)")
+    big.check(lib, "second call (80 paged sequences)")
+    small.check(lib, "third call (the first problem again)")
 
 
 def test_static_scratch_rejects_problems_beyond_its_size():
