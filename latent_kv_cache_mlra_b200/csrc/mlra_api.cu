@@ -6,6 +6,7 @@
 #include <climits>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <array>
 #include <mutex>
@@ -387,6 +388,9 @@ mlra_status decode_impl(const void* q_lat, const void* q_rope, const void* c_kv,
   p.write_final = summed ? 0 : 1;
   p.tma_out = tma_out ? 1 : 0;
   p.timeout_ns = kTimeoutNs;
+  // Test hook: with MLRA_TEST_FORCE_REPLAN set in the environment, the attention kernel treats
+  // its speculative plan as stale and takes the re-plan path (results are unchanged).
+  p.force_replan = std::getenv("MLRA_TEST_FORCE_REPLAN") != nullptr ? 1 : 0;
   if (k1_begin && cudaEventRecord(reinterpret_cast<cudaEvent_t>(k1_begin), s) != cudaSuccess)
     return MLRA_ERR_CUDA;
   if (launch_decode(pl.variant, tq, tqr, tc, tkr, tout, tpart, p, grid, s) != cudaSuccess)

@@ -15,12 +15,15 @@
 // least ~57 cycles and N/2 cycles for N >= 128, so T = 128 keeps the score products efficient.
 //
 // TMEM.  An M = 64 accumulator occupies 16 of the 32 lanes of each sub-partition (rows 16k..16k+15
-// in lanes 32k + [0,16) + 16h for lane half h).  O is cut into chunks of up to 128 columns: chunk
-// j lives in lane half j % 2 at columns 128 (j / 2); score buffers follow in lane half 0.
+// in lanes 32k + [0,16) + 16h for lane half h).  The score buffers (one per stage, T columns
+// each) fill lane half 0; O, cut into chunks of up to 128 columns, sits in lane half 1.
 //
 // Shared memory: the branch's queries (per segment), an NS-deep ring of cache tiles
-// [latent blocks | RoPE block].  The bf16 probabilities P of a tile overwrite the front of the
-// tile's own score buffer in TMEM, from where the output MMA reads them as its A operand.
+// [latent blocks | RoPE block].  The RoPE block is read only by the score product, so the bf16
+// probabilities P of the tile overwrite it ([64 heads x T positions], K-major, the 128-byte
+// swizzled image of an MMA operand) and the output product reads them from there as its A
+// operand.  P is released in 64-position halves: the output product of the first half starts
+// while the softmax still computes the second.
 //
 // Warp roles (224 threads): warps 0-3 softmax / rescale / epilogue, warp 4 TMA producer,
 // warp 5 score-MMA issuer and TMEM owner, warp 6 output-MMA issuer.  The two issuers feed the
@@ -30,11 +33,11 @@
 //
 // Ordering facts the parity waits rely on (a parity wait is only safe when the barrier is at
 // most one phase past the previous phase awaited):
-//   * the score of tile s is issued only after the output product of tile s - NSB completed
-//     (its P sits in the score buffer being reused), so neither issuer can run more than NSB
-//     tiles ahead of the other;
-//   * tile s is loaded only after the output product of tile s - NS completed (stage reuse),
-//     so once the score of tile s is done, every output product up to s - NS is done: the
+//   * tile s is loaded only after the output product of tile s - NS completed (stage reuse), and
+//     there are as many score buffers as stages (NSB = NS), so the score of tile s, issued after
+//     tile s landed, never overwrites a score buffer the softmax still reads; neither issuer runs
+//     more than NS tiles ahead of the other;
+//   * once the score of tile s is done, every output product up to s - NS is done: the
 //     output-completion ring bar_pv_done has NS entries.
 #pragma once
 #include <cstdint>
@@ -57,17 +60,16 @@ struct DecodeCfg {
   static constexpr int QBYTES = (NCB + 1) * BOX;    // query blocks + RoPE-query block
   static constexpr int OCW = DBLK < 128 ? DBLK : 128;   // O chunk width (columns)
   static constexpr int OCH = DBLK / OCW;                // O chunks
-  static constexpr int O_COLS = ((OCH + 1) / 2) * OCW;  // TMEM columns used by O
-  static constexpr int NSB_TMEM = (512 - O_COLS) / T;
-  static constexpr int NSB = NSB_TMEM < 3 ? NSB_TMEM : (NS < 3 ? NS : 3);  // score buffers
+  static constexpr int O_COLS = OCH * OCW;              // TMEM columns of O (lane half 1)
+  static constexpr int NSB = NS;                        // score buffers (lane half 0)
   static constexpr int NPV = NS;                    // ring of output-MMA completion barriers
-  static constexpr int TMEM_USED = O_COLS + NSB * T;
+  static constexpr int TMEM_USED = O_COLS > NSB * T ? O_COLS : NSB * T;
   static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 :
                                    TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_STAGE = QBYTES;
   static constexpr int OFF_BAR = OFF_STAGE + NS * STAGE;
-  static constexpr int NBAR = 2 * NS + 2 + 2 * NSB + NPV + 2;
+  static constexpr int NBAR = 2 * NS + 2 + NSB + TB * NSB + NPV + 2;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // TMEM address, abort flag, status bits
   static constexpr int OFF_PLAN = OFF_MISC + 16;       // in-kernel plan (self_plan)
   static constexpr int PLAN_BYTES = 16 * kSelfPlanMaxSeqs +     // segment list
@@ -79,7 +81,8 @@ struct DecodeCfg {
   static constexpr int SMEM_ALLOC = SMEM + 1024;    // slack to align the base to 1024 B
   static_assert(DBLK % 64 == 0 && DBLK <= 512, "branch width must be a multiple of 64, <= 512");
   static_assert(T == 64 || T == 128, "tile of 64 or 128 positions");
-  static_assert(NSB >= 2 && NSB <= NS, "score buffers: at least 2, at most the stage count");
+  static_assert(NSB >= 2 && NSB == NS, "score buffers: one per stage, at least 2");
+  static_assert(TB * BOX == CBLK, "P of a tile fills the RoPE block of its stage");
   static_assert(TMEM_USED <= 512, "TMEM budget");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
@@ -130,119 +133,144 @@ __device__ __forceinline__ int tile_row(const int32_t* page_table, int max_pages
 
 constexpr int kDecodeThreads = 224;
 
-// In-kernel plan for N <= kSelfPlanMaxSeqs = 64 (all threads call it).  Warp 0 holds sequences
-// lane and lane + 32: it clamps their lengths, scans the real and virtual tile prefixes
-// (mlra_plan.cuh) across the warp, finds the sequence holding each of the range's two virtual
-// boundaries with one ballot, and lets every sequence that overlaps the range write its own
-// segment at its rank in the warp.  The CTAs of group 0 also record, for the combine kernel, the
-// ranges holding each sequence's first and last tile; CTA 0 writes the records and outputs of
-// empty sequences.  Returns the segment count.
-__device__ __noinline__ int plan_in_kernel(const DecodeParams& p, int range, int group,
-                                           uint8_t* plan, uint32_t* flags) {
+// In-kernel plan for N <= kSelfPlanMaxSeqs = 64.  Warp 0 holds sequences lane and lane + 32.
+//
+// plan_read_lengths: the lengths (virtual lengths for several tokens per sequence), clamped to
+// [0, limit]; bit 6 of `bits` reports a length outside that range.
+//
+// plan_segments: scans the real and virtual tile prefixes (mlra_plan.cuh) across the warp, finds
+// the sequence holding each of the range's two virtual boundaries with one ballot, and lets every
+// sequence that overlaps the range write its own segment at its rank in the warp (shared memory
+// only).  Per lane it returns in `bits`: bit c (c = 0, 1) sequence 32 c + lane has its first tile
+// in this range, bit 2 + c its last tile, bit 4 + c it is empty.  Returns the segment count.
+//
+// plan_commit: the plan's global records, written once the lengths are final: the CTAs of group 0
+// record for the combine kernel the ranges holding each sequence's first and last tile, CTA 0
+// the records of empty sequences, and the bad-length status bit.
+//
+// The decode kernel runs the first two before its dependency wait on the lengths as they are then
+// (a speculative plan), reads the lengths again after the wait and keeps the plan when they are
+// unchanged (plan_verify).
+__device__ __forceinline__ void plan_read_lengths(const DecodeParams& p, int lane, int (&L)[2],
+                                                  uint32_t& bits) {
+  bits = 0;
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    const int i = 32 * c + lane;
+    int x = i < p.N ? (p.q_per_seq == 1 ? __ldcg(p.seq_lens + i)
+                                        : __ldcg(p.seq_lens + i / p.q_per_seq) -
+                                              (p.q_per_seq - 1 - i % p.q_per_seq))
+                    : 0;
+    if (i < p.N && (x < 0 || x > p.limit)) {
+      bits |= 64u;
+      x = x < 0 ? 0 : p.limit;
+    }
+    L[c] = x;
+  }
+}
+
+__device__ __noinline__ int plan_segments(const DecodeParams& p, int range, const int (&L)[2],
+                                          uint8_t* plan, uint32_t& bits) {
   int4* list = reinterpret_cast<int4*>(plan);                       // [kSelfPlanMaxSeqs]
   int32_t* lens = reinterpret_cast<int32_t*>(list + kSelfPlanMaxSeqs);
-  int32_t* count = lens + kSelfPlanMaxSeqs;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, N = p.N;
-  if (warp == 0) {
-    int L[2], t[2], lo[2], hi[2], vlo[2], vhi[2];
+  const int lane = threadIdx.x & 31, N = p.N;
+  int t[2], lo[2], hi[2], vlo[2], vhi[2];
+  int carry_t = 0, carry_v = 0;
+  bits &= 64u;
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    const int i = 32 * c + lane;
+    t[c] = i < N ? (L[c] + p.tile - 1) / p.tile : 0;
+    if (i < N && t[c] == 0) bits |= 16u << c;
+    int x = t[c], v = t[c] > 0 ? t[c] + p.seg_cost : 0;
+    const int vt = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {  // inclusive scans
+      const int yx = __shfl_up_sync(kFull, x, o), yv = __shfl_up_sync(kFull, v, o);
+      if (lane >= o) {
+        x += yx;
+        v += yv;
+      }
+    }
+    hi[c] = x + carry_t;
+    lo[c] = hi[c] - t[c];
+    vhi[c] = v + carry_v;
+    vlo[c] = vhi[c] - vt;
+    carry_t += __shfl_sync(kFull, x, 31);
+    carry_v += __shfl_sync(kFull, v, 31);
+    if (i < N) lens[i] = L[c];
+  }
+  const int64_t total = carry_t, vtotal = carry_v;
+  const int64_t R = effective_ranges(p.num_ranges, total);
+  int n = 0;
+  if (range < R && total > 0) {
+    // real tile of a virtual position: the sequence whose virtual interval holds it
+    auto tile_of = [&](int64_t v) -> int64_t {
+      int64_t g = 0;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const bool own = t[c] > 0 && vlo[c] <= v && v < vhi[c];
+        const uint32_t m = __ballot_sync(kFull, own);
+        if (m) {
+          const int src = __ffs(m) - 1;
+          const int64_t o = v - vlo[c] - p.seg_cost;
+          const int64_t mine = lo[c] + (o > 0 ? o : 0);
+          g = __shfl_sync(kFull, mine, src);
+        }
+      }
+      return g;
+    };
+    const int64_t g0 = tile_of((range * vtotal) / R);
+    const int64_t g1 = range + 1 < R ? tile_of(((range + 1) * vtotal) / R) : total;
+    int base = 0;
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const int i = 32 * c + lane;
-      L[c] = i < N ? (p.q_per_seq == 1 ? __ldcg(p.seq_lens + i)
-                                         : __ldcg(p.seq_lens + i / p.q_per_seq) -
-                                               (p.q_per_seq - 1 - i % p.q_per_seq))
-                   : 0;
-    }
-    int carry_t = 0, carry_v = 0;
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const int i = 32 * c + lane;
-      if (i < N && (L[c] < 0 || L[c] > p.limit)) {
-        atomicOr(flags, kFlagBadLength);
-        L[c] = L[c] < 0 ? 0 : p.limit;
+      const bool ov = t[c] > 0 && lo[c] < g1 && hi[c] > g0;
+      const uint32_t m = __ballot_sync(kFull, ov);
+      if (ov) {
+        const int64_t a = g0 > lo[c] ? g0 : lo[c], e = g1 < hi[c] ? g1 : hi[c];
+        const bool whole = a == lo[c] && e == hi[c];
+        list[base + __popc(m & ((1u << lane) - 1u))] =
+            make_int4(i, static_cast<int>(a - lo[c]), static_cast<int>(e - a),
+                      L[c] | (whole ? (int32_t)0x80000000u : 0));
+        if (a == lo[c]) bits |= 1u << c;  // the sequence's first tile is in this range
+        if (e == hi[c]) bits |= 4u << c;  // ... its last tile
       }
-      t[c] = i < N ? (L[c] + p.tile - 1) / p.tile : 0;
-      int x = t[c], v = t[c] > 0 ? t[c] + p.seg_cost : 0;
-      const int vt = v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {  // inclusive scans
-        const int yx = __shfl_up_sync(kFull, x, o), yv = __shfl_up_sync(kFull, v, o);
-        if (lane >= o) {
-          x += yx;
-          v += yv;
-        }
-      }
-      hi[c] = x + carry_t;
-      lo[c] = hi[c] - t[c];
-      vhi[c] = v + carry_v;
-      vlo[c] = vhi[c] - vt;
-      carry_t += __shfl_sync(kFull, x, 31);
-      carry_v += __shfl_sync(kFull, v, 31);
-      if (i < N) lens[i] = L[c];
+      base += __popc(m);
     }
-    const int64_t total = carry_t, vtotal = carry_v;
-    const int64_t R = effective_ranges(p.num_ranges, total);
-    int n = 0;
-    if (range < R && total > 0) {
-      // real tile of a virtual position: the sequence whose virtual interval holds it
-      auto tile_of = [&](int64_t v) -> int64_t {
-        int64_t g = 0;
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const bool own = t[c] > 0 && vlo[c] <= v && v < vhi[c];
-          const uint32_t m = __ballot_sync(kFull, own);
-          if (m) {
-            const int src = __ffs(m) - 1;
-            const int64_t o = v - vlo[c] - p.seg_cost;
-            const int64_t mine = lo[c] + (o > 0 ? o : 0);
-            g = __shfl_sync(kFull, mine, src);
-          }
-        }
-        return g;
-      };
-      const int64_t g0 = tile_of((range * vtotal) / R);
-      const int64_t g1 = range + 1 < R ? tile_of(((range + 1) * vtotal) / R) : total;
-      int base = 0;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int i = 32 * c + lane;
-        const bool ov = t[c] > 0 && lo[c] < g1 && hi[c] > g0;
-        const uint32_t m = __ballot_sync(kFull, ov);
-        if (ov) {
-          const int64_t a = g0 > lo[c] ? g0 : lo[c], e = g1 < hi[c] ? g1 : hi[c];
-          const bool whole = a == lo[c] && e == hi[c];
-          list[base + __popc(m & ((1u << lane) - 1u))] =
-              make_int4(i, static_cast<int>(a - lo[c]), static_cast<int>(e - a),
-                        L[c] | (whole ? (int32_t)0x80000000u : 0));
-          if (group == 0) {
-            if (a == lo[c]) p.seqs[i].r0 = range;  // the sequence's first tile is in this range
-            if (e == hi[c]) p.seqs[i].r1 = range;  // ... its last tile
-          }
-        }
-        base += __popc(m);
-      }
-      n = base;
-    }
-    if (blockIdx.x == 0) {
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int i = 32 * c + lane;
-        if (i < N && t[c] == 0) p.seqs[i] = SeqInfo{0, -1};
-      }
-    }
-    if (lane == 0) *count = n;
+    n = base;
   }
-  __syncthreads();
-  if (blockIdx.x == 0 && warp >= 1) {
-    for (int sq = warp - 1; sq < N; sq += kDecodeThreads / 32 - 1) {  // empty: out = 0, lse = -inf
-      if (lens[sq] != 0) continue;
-      float* row = p.out + (int64_t)sq * p.H * p.out_width;
-      for (int i = lane; i < p.H * p.out_width; i += 32) row[i] = 0.f;
-      if (p.lse)
-        for (int i = lane; i < p.H * p.B; i += 32) p.lse[(int64_t)sq * p.H * p.B + i] = -CUDART_INF_F;
+  return n;
+}
+
+__device__ __forceinline__ void plan_commit(const DecodeParams& p, int range, int group,
+                                            uint32_t bits, uint32_t* flags) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    const int i = 32 * c + lane;
+    if (group == 0) {
+      if (bits & (1u << c)) p.seqs[i].r0 = range;
+      if (bits & (4u << c)) p.seqs[i].r1 = range;
     }
+    if (blockIdx.x == 0 && (bits & (16u << c))) p.seqs[i] = SeqInfo{0, -1};
   }
-  return *count;
+  if (bits & 64u) atomicOr(flags, kFlagBadLength);
+}
+
+// Outputs of empty sequences (out = 0, lse = -inf), written by CTA 0's warps 1.. after the plan.
+__device__ __forceinline__ void plan_empty_outputs(const DecodeParams& p, const uint8_t* plan) {
+  const int32_t* lens =
+      reinterpret_cast<const int32_t*>(reinterpret_cast<const int4*>(plan) + kSelfPlanMaxSeqs);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int sq = warp - 1; sq < p.N; sq += kDecodeThreads / 32 - 1) {
+    if (lens[sq] != 0) continue;
+    float* row = p.out + (int64_t)sq * p.H * p.out_width;
+    for (int i = lane; i < p.H * p.out_width; i += 32) row[i] = 0.f;
+    if (p.lse)
+      for (int i = lane; i < p.H * p.B; i += 32) p.lse[(int64_t)sq * p.H * p.B + i] = -CUDART_INF_F;
+  }
 }
 
 // The segments of one work range, read one ahead of use: from the prep kernel's descriptors in
@@ -293,13 +321,17 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const uint32_t bar_q_full = bar0 + 16 * NS;               //       TMA -> MMA
   const uint32_t bar_q_empty = bar_q_full + 8;              //       MMA (last score) -> TMA
   const uint32_t bar_s_full = bar_q_full + 16;              // [NSB] MMA (score) -> softmax
-  const uint32_t bar_p_full = bar_s_full + 8 * NSB;         // [NSB] softmax -> MMA
-  const uint32_t bar_pv_done = bar_p_full + 8 * NSB;       // [NPV] MMA (PV done) -> softmax, score issuer
+  const uint32_t bar_p_full = bar_s_full + 8 * NSB;         // [TB][NSB] softmax (P half) -> MMA
+  const uint32_t bar_pv_done = bar_p_full + 8 * C::TB * NSB; // [NPV] MMA (PV done) -> softmax
   const uint32_t bar_final_s = bar_pv_done + 8 * NPV;       // drains of the two issuers
   const uint32_t bar_final_pv = bar_final_s + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  uint32_t* spec_flags = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC + 8);  // see below
   uint32_t* flags = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC + 12);  // this CTA's status bits
+  uint8_t* plan = smem + C::OFF_PLAN;
+  volatile int32_t* plan_count = reinterpret_cast<volatile int32_t*>(plan + 20 * kSelfPlanMaxSeqs);
+  volatile int32_t* plan_stale = plan_count + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int range = blockIdx.x / p.n_groups;
@@ -310,21 +342,23 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   // The combine kernel may be scheduled now; it waits for this grid before reading anything.
   pdl_launch_dependents();
 
-  if (threadIdx.x == 0) {
+  auto init_barriers = [&]() {
     for (int k = 0; k < NS; ++k) {
       mbar_init(bar_stage_full + 8 * k, 1);
       mbar_init(bar_stage_empty + 8 * k, 1);
     }
     mbar_init(bar_q_full, 1);
     mbar_init(bar_q_empty, 1);
-    for (int k = 0; k < NSB; ++k) {
-      mbar_init(bar_s_full + 8 * k, 1);
-      mbar_init(bar_p_full + 8 * k, 128);
-    }
+    for (int k = 0; k < NSB; ++k) mbar_init(bar_s_full + 8 * k, 1);
+    for (int k = 0; k < C::TB * NSB; ++k) mbar_init(bar_p_full + 8 * k, 128);
     for (int k = 0; k < NPV; ++k) mbar_init(bar_pv_done + 8 * k, 1);
     mbar_init(bar_final_s, 1);
     mbar_init(bar_final_pv, 1);
+  };
+  if (threadIdx.x == 0) {
+    init_barriers();
     *abort_flag = 0;
+    *spec_flags = 0;
     *flags = 0;
     fence_barrier_init();
   }
@@ -332,8 +366,6 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (p.self_plan && warp == 0 && 32 * lane < p.N / p.q_per_seq)  // the caller's lengths
-    prefetch_l2(p.seq_lens + 32 * lane);  // warms L2 and the TLB for the plan below
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_qr);
@@ -342,19 +374,125 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tma_prefetch_desc(&tm_part);
     if (p.tma_out) tma_prefetch_desc(&tm_out);
   }
+  // Speculative plan (N <= kSelfPlanMaxSeqs): made from the lengths as they are before the
+  // dependency wait, while the previous kernel on the stream may still run.  It is used only if
+  // the lengths read again after the wait are the same (below); nothing global is written here.
+  int spec_len[2] = {0, 0};
+  uint32_t plan_bits = 0;
+  if (p.self_plan && warp == 0) {
+    plan_read_lengths(p, lane, spec_len, plan_bits);
+    const int n = plan_segments(p, range, spec_len, plan, plan_bits);
+    if (lane == 0) *plan_count = n;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int col0 = branch * DBLK;  // first latent column of this CTA's branch
+  int4 first_seg = make_int4(0, 0, 0, 0);  // the producer's copy of the first speculative segment
+  const bool speculate = p.self_plan && warp == 4 && *plan_count > 0;
+  if (speculate) first_seg = reinterpret_cast<const int4*>(plan)[0];
+
+  // Loads of one tile into stage st (lane 0 of the producer): the latent block's 64-row
+  // sub-boxes and the RoPE block, counted on the stage's full barrier.
+  const uint64_t once = l2_policy_evict_first();
+  auto issue_tile = [&](int st, const int (&rows)[C::TB]) {
+    const uint32_t full = bar_stage_full + 8 * st;
+    const uint32_t dst = sStage + st * C::STAGE;
+    mbar_arrive_expect_tx(full, C::STAGE);
+    // the latent rows are read once per call (by this CTA alone): first out of L2, so the
+    // queries, RoPE rows (shared by the branch CTAs) and partial results stay
+#pragma unroll
+    for (int l = 0; l < C::TB; ++l) {
+#pragma unroll
+      for (int k = 0; k < C::NCB; ++k)
+        tma_load_2d_hint(dst + k * C::CBLK + l * C::BOX, &tm_c, full, col0 + 64 * k, rows[l], once);
+      tma_load_2d(dst + C::NCB * C::CBLK + l * C::BOX, &tm_kr, full, 0, rows[l]);
+    }
+  };
+  auto issue_queries = [&](int seq) {
+    mbar_arrive_expect_tx(bar_q_full, C::QBYTES);
+#pragma unroll
+    for (int k = 0; k < C::NCB; ++k)
+      tma_load_3d(sQ + k * C::BOX, &tm_q, bar_q_full, col0 + 64 * k, h0, seq);
+    tma_load_3d(sQ + C::NCB * C::BOX, &tm_qr, bar_q_full, 0, h0, seq);
+  };
+  // cache rows of tile t of virtual sequence v's cache (length len; past the end: zeros)
+  auto tile_rows = [&](int cache_seq, int t, int len, uint32_t* status, int (&rows)[C::TB]) {
+#pragma unroll
+    for (int l = 0; l < C::TB; ++l) {
+      const int t64 = t * C::TB + l;
+      rows[l] = (t64 * kTile < len)
+                    ? tile_row(p.page_table, p.max_pages, p.page_size, p.max_seq_len, p.n_pages,
+                               p.oob_row, cache_seq, t64, lane == 0 ? status : nullptr)
+                    : p.oob_row;
+    }
+  };
+
   // Everything above overlapped the previous kernel on the stream (the prep kernel, or the
-  // previous call's combine); the lengths or the prep kernel's plan are read only after it.
+  // previous call's combine); the lengths, queries, cache and the prep kernel's plan are read
+  // only after it.
   pdl_wait_prerequisites();
+  int pre_tiles = 0;      // producer: tiles of the first segment already issued
+  bool pre_q = false;     // ... and its queries
+  if (p.self_plan) {
+    if (speculate) {
+      // The first segment's queries and tiles go out at once, on the speculative plan (bad-page
+      // bits into spec_flags until the plan is confirmed).
+      const int len = first_seg.w & 0x7fffffff;
+      pre_tiles = first_seg.z < NS ? first_seg.z : NS;
+      pre_q = true;
+      const int cache_seq = first_seg.x / p.q_per_seq;
+      if (lane == 0) issue_queries(first_seg.x);
+      for (int i = 0; i < pre_tiles; ++i) {
+        int rows[C::TB];
+        tile_rows(cache_seq, first_seg.y + i, len, spec_flags, rows);
+        if (lane == 0) issue_tile(i, rows);
+      }
+      __syncwarp();
+    }
+    if (warp == 0) {
+      // the lengths now final: keep the speculative plan if they did not change
+      int len_now[2];
+      uint32_t bits_now;
+      plan_read_lengths(p, lane, len_now, bits_now);
+      const bool same = __all_sync(kFull, len_now[0] == spec_len[0] && len_now[1] == spec_len[1]);
+      if (!same || p.force_replan) {
+        plan_bits = bits_now;
+        const int n = plan_segments(p, range, len_now, plan, plan_bits);
+        if (lane == 0) *plan_count = n;
+      }
+      if (lane == 0) *plan_stale = (!same || p.force_replan) ? 1 : 0;
+      plan_commit(p, range, group, plan_bits, flags);
+    }
+    __syncthreads();
+    if (*plan_stale) {
+      // The lengths changed under the speculative plan: let its loads land, reset the barriers
+      // and start over with the new plan.
+      if (speculate) {
+        if (pre_q) wait_warp(bar_q_full, 0, tmo, abort_flag, flags, false);
+        for (int i = 0; i < pre_tiles; ++i)
+          wait_warp(bar_stage_full + 8 * i, 0, tmo, abort_flag, flags, false);
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        for (int k = 0; k < C::NBAR; ++k) mbar_inval(bar0 + 8 * k);
+        init_barriers();
+        fence_barrier_init();
+      }
+      __syncthreads();
+      pre_tiles = 0;
+      pre_q = false;
+    } else if (speculate && lane == 0) {
+      atomicOr(flags, *spec_flags);
+    }
+    if (blockIdx.x == 0 && warp >= 1) plan_empty_outputs(p, plan);
+  }
   const int4* seg_list;
   int seg_count;
   if (p.self_plan) {
-    seg_count = plan_in_kernel(p, range, group, smem + C::OFF_PLAN, flags);
-    seg_list = reinterpret_cast<const int4*>(smem + C::OFF_PLAN);
+    seg_count = *plan_count;
+    seg_list = reinterpret_cast<const int4*>(plan);
   } else {
     const int2 r2 = __ldcg(reinterpret_cast<const int2*>(p.ranges + range));
     seg_list = reinterpret_cast<const int4*>(p.segs + r2.x);
@@ -372,47 +510,19 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     while (ok && walk.next(seg, L)) {
       if (nseg > 0) ok = wait_warp(bar_q_empty, (nseg - 1) & 1, tmo, abort_flag, flags);
       if (!ok) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(bar_q_full, C::QBYTES);
-#pragma unroll
-        for (int k = 0; k < C::NCB; ++k)
-          tma_load_3d(sQ + k * C::BOX, &tm_q, bar_q_full, col0 + 64 * k, h0, seg.seq);
-        tma_load_3d(sQ + C::NCB * C::BOX, &tm_qr, bar_q_full, 0, h0, seg.seq);
-      }
+      if (lane == 0 && !(nseg == 0 && pre_q)) issue_queries(seg.seq);
       __syncwarp();
       const int cache_seq = seg.seq / p.q_per_seq;  // whose cache rows (once per segment)
       for (int i = 0; i < seg.ntiles; ++i, ++it) {
-        // cache rows of the tile's 64-position sub-boxes (past the sequence end: zeros)
+        if (nseg == 0 && i < pre_tiles) continue;  // issued before the plan was confirmed
         int rows[C::TB];
-#pragma unroll
-        for (int l = 0; l < C::TB; ++l) {
-          const int t64 = (seg.tile0 + i) * C::TB + l;
-          rows[l] = (t64 * kTile < L)
-                        ? tile_row(p.page_table, p.max_pages, p.page_size, p.max_seq_len, p.n_pages,
-                                   p.oob_row, cache_seq, t64, lane == 0 ? flags : nullptr)
-                        : p.oob_row;
-        }
+        tile_rows(cache_seq, seg.tile0 + i, L, flags, rows);
         const int st = it % NS;
         if (it >= NS) {
           ok = wait_warp(bar_stage_empty + 8 * st, ((it / NS) - 1) & 1, tmo, abort_flag, flags);
           if (!ok) break;
         }
-        if (lane == 0) {
-          const uint32_t full = bar_stage_full + 8 * st;
-          const uint32_t dst = sStage + st * C::STAGE;
-          mbar_arrive_expect_tx(full, C::STAGE);
-          // the latent rows are read once per call (by this CTA alone): first out of L2, so the
-          // queries, RoPE rows (shared by the branch CTAs) and partial results stay
-          const uint64_t once = l2_policy_evict_first();
-#pragma unroll
-          for (int l = 0; l < C::TB; ++l) {
-#pragma unroll
-            for (int k = 0; k < C::NCB; ++k)
-              tma_load_2d_hint(dst + k * C::CBLK + l * C::BOX, &tm_c, full, col0 + 64 * k, rows[l],
-                               once);
-            tma_load_2d(dst + C::NCB * C::CBLK + l * C::BOX, &tm_kr, full, 0, rows[l]);
-          }
-        }
+        if (lane == 0) issue_tile(st, rows);
         __syncwarp();
       }
       ++nseg;
@@ -434,15 +544,14 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     while (ok && walk.next(seg, L)) {
       ok = wait_warp(bar_q_full, nseg & 1, tmo, abort_flag, flags);
       for (int i = 0; ok && i < seg.ntiles; ++i, ++it) {
+        // the landed tile implies the output product of tile it - NS completed, so its softmax
+        // has read score buffer it % NSB (NSB == NS)
         ok = wait_warp(bar_stage_full + 8 * (it % NS), (it / NS) & 1, tmo, abort_flag, flags);
-        if (ok && it >= NSB)  // score buffer free: the output product of tile it-NSB read its P
-          ok = wait_warp(bar_pv_done + 8 * ((it - NSB) % NPV), ((it - NSB) / NPV) & 1, tmo,
-                         abort_flag, flags);
         if (!ok) break;
         tc_fence_after();
         if (lane == 0) {
           const uint32_t stg = sStage + (it % NS) * C::STAGE;
-          const uint32_t d = tmem + C::O_COLS + (it % NSB) * T;
+          const uint32_t d = tmem + (it % NSB) * T;  // lane half 0
 #pragma unroll
           for (int kb = 0; kb < C::NCB; ++kb) {
 #pragma unroll
@@ -478,31 +587,35 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     int j = 0;
     bool ok = true;
     while (ok && walk.next(seg, L)) {
-      for (int i = 0; i < seg.ntiles; ++i, ++j) {
-        ok = wait_warp(bar_p_full + 8 * (j % NSB), (j / NSB) & 1, tmo, abort_flag, flags);
-        if (!ok) break;
-        tc_fence_after();
-        if (lane == 0) {
-          const bool first = (i == 0);  // the segment's first product overwrites O
-          const uint32_t stg = sStage + (j % NS) * C::STAGE;
-          const uint32_t pa = tmem + C::O_COLS + (j % NSB) * T;  // P: front of the score buffer
+      for (int i = 0; ok && i < seg.ntiles; ++i, ++j) {
+        const uint32_t stg = sStage + (j % NS) * C::STAGE;
+        const uint32_t pa = stg + C::NCB * C::CBLK;  // P over the tile's RoPE block
+#pragma unroll 1
+        for (int hb = 0; hb < C::TB; ++hb) {  // one 64-position half of P at a time
+          ok = wait_warp(bar_p_full + 8 * (hb * NSB + j % NSB), (j / NSB) & 1, tmo, abort_flag,
+                         flags);
+          if (!ok) break;
+          tc_fence_after();
+          if (lane == 0) {
+            const bool first = (i == 0 && hb == 0);  // the segment's first product overwrites O
 #pragma unroll
-          for (int ch = 0; ch < C::OCH; ++ch) {
-            // A from TMEM must sit in the accumulator's lanes: chunks in lane half 1 read the
-            // copy of P that the softmax writes there
-            const uint32_t d = tmem + ((uint32_t)(16 * (ch & 1)) << 16) + (ch >> 1) * C::OCW;
-            const uint32_t b0 = stg + ch * (C::OCW / 64) * C::CBLK;
+            for (int ch = 0; ch < C::OCH; ++ch) {
+              const uint32_t d = tmem + (16u << 16) + ch * C::OCW;  // lane half 1
+              const uint32_t b0 = stg + ch * (C::OCW / 64) * C::CBLK;
 #pragma unroll
-            for (int kk = 0; kk < T / 16; ++kk) {
-              const uint64_t bd = sw128_desc(b0 + kk * 2048, C::CBLK, 1024);
-              umma_bf16_ts(d, pa + ((uint32_t)(16 * (ch & 1)) << 16) + kk * 8, bd, kIdPV,
-                           (kk > 0 || !first) ? 1u : 0u);
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t ad = sw128_desc(pa + hb * C::BOX + kk * 32, 16, 1024);
+                const uint64_t bd = sw128_desc(b0 + (4 * hb + kk) * 2048, C::CBLK, 1024);
+                umma_bf16(d, ad, bd, kIdPV, (kk > 0 || !first) ? 1u : 0u);
+              }
+            }
+            if (hb == C::TB - 1) {
+              umma_commit(bar_stage_empty + 8 * (j % NS));
+              umma_commit(bar_pv_done + 8 * (j % NPV));
             }
           }
-          umma_commit(bar_stage_empty + 8 * (j % NS));
-          umma_commit(bar_pv_done + 8 * (j % NPV));
+          __syncwarp();
         }
-        __syncwarp();
       }
     }
     if (lane == 0) umma_commit(bar_final_pv);
@@ -528,25 +641,49 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         ok = wait_warp(bar_s_full + 8 * (it % NSB), (it / NSB) & 1, tmo, abort_flag, flags);
         if (!ok) break;
         tc_fence_after();
-        // this thread's scores: positions 64 l + 32 q + [0, 32) of the tile, l < T / 64
+        // this thread's scores: positions 64 l + 32 q + [0, 32) of the tile, l < T / 64 (both
+        // loads in flight, one wait)
         float v[C::TB][32];
 #pragma unroll
-        for (int l = 0; l < C::TB; ++l) {
-          uint32_t r[32];
-          tmem_ld16x2_32(tmem + lane_base + C::O_COLS + (it % NSB) * T + 64 * l, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) v[l][k] = __uint_as_float(r[k]);
-        }
+        for (int l = 0; l < C::TB; ++l)
+          tmem_ld16x2_32(tmem + lane_base + (it % NSB) * T + 64 * l,
+                         reinterpret_cast<uint32_t(&)[32]>(v[l]));
+        tmem_wait_ld();
         const int valid = min(T, L - T * t);
-        float mx = -CUDART_INF_F;
+        // Row maximum of the scaled scores (log2 units).  A whole tile holds only finite scores:
+        // the maximum of the raw dot products (the minimum for a negative scale) times the scale,
+        // and the scale is folded into each exponent below (one FFMA per score).  The ragged last
+        // tile scales first and masks the positions past the sequence end with -inf.
+        const bool whole_tile = valid == T;
+        const float sc = p.scale_log2;
+        float mx;
+        if (whole_tile) {
+          float a[4];
 #pragma unroll
-        for (int l = 0; l < C::TB; ++l) {
+          for (int u = 0; u < 4; ++u) a[u] = v[0][u];
+          if (sc >= 0.f) {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const float x = (64 * l + 32 * q + k < valid) ? v[l][k] * p.scale_log2 : -CUDART_INF_F;
-            v[l][k] = x;
-            mx = fmaxf(mx, x);
+            for (int l = 0; l < C::TB; ++l)
+#pragma unroll
+              for (int k = 0; k < 32; ++k) a[k & 3] = fmaxf(a[k & 3], v[l][k]);
+            mx = fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])) * sc;
+          } else {
+#pragma unroll
+            for (int l = 0; l < C::TB; ++l)
+#pragma unroll
+              for (int k = 0; k < 32; ++k) a[k & 3] = fminf(a[k & 3], v[l][k]);
+            mx = fminf(fminf(a[0], a[1]), fminf(a[2], a[3])) * sc;
+          }
+        } else {
+          mx = -CUDART_INF_F;
+#pragma unroll
+          for (int l = 0; l < C::TB; ++l) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              const float x = (64 * l + 32 * q + k < valid) ? v[l][k] * sc : -CUDART_INF_F;
+              v[l][k] = x;
+              mx = fmaxf(mx, x);
+            }
           }
         }
         mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
@@ -570,8 +707,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           for (int ch = 0; ch < C::OCH; ++ch) {
 #pragma unroll 1
             for (int c0 = 0; c0 < C::OCW; c0 += 64) {
-              const uint32_t a = tmem + ((uint32_t)(32 * warp + 16 * (ch & 1)) << 16) +
-                                 (ch >> 1) * C::OCW + c0;
+              const uint32_t a = tmem + ((uint32_t)(32 * warp + 16) << 16) + ch * C::OCW + c0;
               uint32_t r[32];
               tmem_ld16x2_32(a, r);
               tmem_wait_ld();
@@ -582,40 +718,49 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           }
           tmem_wait_st();
         }
-        // probabilities -> bf16 P over the front of this tile's score buffer: position
-        // 64 l + 32 q + k goes to column (64 l + 32 q + k) / 2, two positions per column
-        const uint32_t pcol = tmem + lane_base + C::O_COLS + (it % NSB) * T;
-        float sum = 0.f;
+        uint8_t* stage_ptr = smem + C::OFF_STAGE + (it % NS) * C::STAGE;
+        if (valid < T) {
+          // Ragged last tile: zero the latent rows past the sequence end so that the zero
+          // probabilities never multiply a non-finite value left in the cache (before the first
+          // half of P is released: the output product reads these rows)
+          for (int k = threadIdx.x; k < C::NCB * T * 8; k += 128) {
+            const int row = (k >> 3) % T;
+            if (row >= valid)
+              *reinterpret_cast<uint4*>(stage_ptr + (k / (T * 8)) * C::CBLK + row * 128 + (k & 7) * 16) =
+                  make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        // probabilities -> bf16 P over the tile's RoPE block, the K-major image of the output
+        // product's A operand: head row r, position 64 l + 32 q + k in 64-position block l, row r,
+        // 16-byte chunk (4 q + k / 8) ^ (r & 7) (128-byte swizzle).  Each block is released to the
+        // output product as soon as it is written.
+        // p = 2^(score - m): whole tiles hold the raw products (one FFMA applies the scale),
+        // the ragged tile the scaled and masked scores
+        const float mul = whole_tile ? sc : 1.f, neg_m = -m_used;
+        const int prow = 16 * warp + (lane & 15);
+        uint8_t* p_base = stage_ptr + C::NCB * C::CBLK + prow * 128;
+        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int l = 0; l < C::TB; ++l) {
           uint32_t pk[16];
 #pragma unroll
           for (int k = 0; k < 32; k += 2) {
-            const float p0 = ex2_approx(v[l][k] - m_used);
-            const float p1 = ex2_approx(v[l][k + 1] - m_used);
-            sum += p0 + p1;
+            const float p0 = ex2_approx(fmaf(v[l][k], mul, neg_m));
+            const float p1 = ex2_approx(fmaf(v[l][k + 1], mul, neg_m));
+            sum4[(k >> 1) & 3] += p0 + p1;
             pk[k / 2] = pack_bf16x2(p0, p1);
           }
-          tmem_st16x2_16(pcol + 32 * l, pk);
-          if (C::OCH > 1) tmem_st16x2_16(pcol + (16u << 16) + 32 * l, pk);  // copy in lane half 1
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(p_base + l * C::BOX + (((4 * q + c) ^ (prow & 7)) << 4)) =
+                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          fence_proxy_async_smem();  // P (and the zeroed rows) are read by the MMA (async proxy)
+          tc_fence_before();         // ... after this thread's TMEM loads (and O rescale)
+          mbar_arrive(bar_p_full + 8 * (l * NSB + it % NSB));
         }
-        tmem_wait_st();
+        float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
         sum += __shfl_xor_sync(kFull, sum, 16);
         l_sum += sum;
-        if (valid < T) {
-          uint8_t* stg = smem + C::OFF_STAGE + (it % NS) * C::STAGE;
-          // Ragged last tile: zero the latent rows past the sequence end so that the zero
-          // probabilities never multiply a non-finite value left in the cache.
-          for (int k = threadIdx.x; k < C::NCB * T * 8; k += 128) {
-            const int row = (k >> 3) % T;
-            if (row >= valid)
-              *reinterpret_cast<uint4*>(stg + (k / (T * 8)) * C::CBLK + row * 128 + (k & 7) * 16) =
-                  make_uint4(0u, 0u, 0u, 0u);
-          }
-          fence_proxy_async_smem();  // the zeros are read by the output MMA (async proxy)
-        }
-        tc_fence_before();
-        mbar_arrive(bar_p_full + 8 * (it % NSB));
       }
       if (!ok) break;
       // ------------------------------------------------ epilogue of the segment
@@ -657,7 +802,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll 1
             for (int c0 = 0; c0 < C::OCW; c0 += 64) {
               uint32_t r[32];
-              tmem_ld16x2_32(tmem + ((uint32_t)(32 * warp + 16 * (ch & 1)) << 16) + (ch >> 1) * C::OCW + c0, r);
+              tmem_ld16x2_32(tmem + ((uint32_t)(32 * warp + 16) << 16) + ch * C::OCW + c0, r);
               tmem_wait_ld();
               const int col = ch * C::OCW + c0 + 32 * q;
               if (col < ncols_out) {
@@ -683,7 +828,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll 1
             for (int c0 = 0; c0 < C::OCW; c0 += 64) {
               uint32_t r[32];
-              tmem_ld16x2_32(tmem + ((uint32_t)(32 * warp + 16 * (ch & 1)) << 16) + (ch >> 1) * C::OCW + c0, r);
+              tmem_ld16x2_32(tmem + ((uint32_t)(32 * warp + 16) << 16) + ch * C::OCW + c0, r);
               tmem_wait_ld();
 #pragma unroll
               for (int half = 0; half < 2; ++half) {
@@ -716,7 +861,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll 1
           for (int c0 = 0; c0 < C::OCW; c0 += 64) {
             uint32_t r[32];
-            tmem_ld16x2_32(tmem + ((uint32_t)(32 * warp + 16 * (ch & 1)) << 16) + (ch >> 1) * C::OCW + c0, r);
+            tmem_ld16x2_32(tmem + ((uint32_t)(32 * warp + 16) << 16) + ch * C::OCW + c0, r);
             tmem_wait_ld();
             if (live) {
               const int cbase = ch * C::OCW + c0 + 32 * q;

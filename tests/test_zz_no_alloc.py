@@ -38,6 +38,7 @@ def _close(a, b, what):
 
 def _lse_close(a, b, what):
     a = a.detach().cpu().double().numpy()
+    b = b.detach().cpu().double().numpy() if hasattr(b, "detach") else np.asarray(b)
     fin = np.isfinite(b)
     assert (np.isneginf(a) == np.isneginf(b)).all(), f"{what}: -inf pattern"
     assert (np.abs(a[fin] - b[fin]) <= 1e-3 + 1e-4 * np.abs(b[fin])).all(), what
