@@ -557,6 +557,103 @@ def run_ours(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- branch parallelism
+def branch_layout(num_branches: int, world: int, rank: int):
+    """(shard, shards, branches per device) of `rank` when the layer's B branches are spread over
+    `world` devices: device g keeps the g-th of `world` equal column blocks of the latent, i.e.
+    B / world adjacent branches ("Multi-Head Low-Rank Attention", section 3.2)."""
+    if world < 1 or world > num_branches or num_branches % world or not 0 <= rank < world:
+        raise ValueError(f"{num_branches} branches cannot be spread evenly over {world} devices")
+    return rank, world, num_branches // world
+
+
+def branch_step(w: workloads.Workload, inp: workloads.Inputs, dev, world: int, rank: int,
+                d_head: int = 128):
+    """This device's share of a branch-parallel layer step: steps 2 and 3 of its branches (CUDA)
+    and, with more than one device, the all-reduce of y over the devices.  The inputs and W^UV are
+    the same on every device (one layer, split by branches); each device cuts its blocks."""
+    from latent_kv_cache_mlra_b200 import tp
+    shard, shards, per_device = branch_layout(w.num_branches, world, rank)
+    g = torch.Generator().manual_seed(w.seed + 77)
+    w_uv = (torch.randn(w.heads, d_head, w.d_latent, generator=g) / w.d_latent ** 0.5).to(torch.bfloat16)
+    pt = None if inp.page_table is None else inp.page_table.to(dev)
+    step = tp.BranchShardStep(
+        tp.shard_queries(inp.q_lat, shard, shards).to(dev), inp.q_rope.to(dev),
+        tp.shard_latent(inp.c_kv, shard, shards).to(dev), inp.k_rope.to(dev), inp.seq_lens.to(dev),
+        pt, tp.shard_wuv(w_uv, shard, shards).to(dev), num_branches=w.num_branches,
+        branches_per_device=per_device, softmax_scale=w.sigma, max_seq_len=inp.max_seq_len,
+        page_size=w.page_size, reduce=world > 1)
+    return step, w_uv, per_device
+
+
+def run_branch(args):
+    """One attention layer's decode step with the branches spread over the devices (the pages'
+    tensor-parallel setting): each device runs steps 2 and 3 of its B / world branches on its
+    column block of the cache, then one NCCL all-reduce of y [N, H, d_head] sums the branches.
+    The same layer is split, so scaling is strong; the step time is the maximum over ranks."""
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = workloads.get(args.workload)
+    inp = workloads.make_inputs(w)
+    step, _, per_device = branch_step(w, inp, dev, world, rank)
+    stream = torch.cuda.current_stream(dev)
+    dc_dev = w.d_latent * per_device // w.num_branches
+    dev_bytes = int(inp.seq_lens.to(torch.int64).sum()) * (dc_dev + w.d_rope) * 2
+    flush = None if dev_bytes > L2_BYTES else torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            if flush is not None:
+                torch.sum(flush, dim=0, out=sink)
+            ev[i][0].record(stream)
+            y = step.local()
+            ev[i][1].record(stream)
+            if world > 1:
+                import torch.distributed as dist
+                dist.all_reduce(y, op=dist.ReduceOp.SUM, group=step.group)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    local_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b, _ in ev) / args.steps, world, dev)
+    ar_ms = max_over_ranks(sum(b.elapsed_time(c) for _, b, c in ev) / args.steps, world, dev)
+    ms = max_over_ranks(sum(a.elapsed_time(c) for a, _, c in ev) / args.steps, world, dev)
+    rc, flags = step.decoder.status()
+    if rc != 0:
+        raise RuntimeError(f"device status after timing: {rc} (flags {flags})")
+    peaks = measured_peaks()
+    line = {"metric": "attention layer decode (steps 2-3), branch-parallel", "value": w.batch / (ms * 1e-3),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {**workload_config(w, inp), "parallelism": f"branch{world}",
+                       "branches_per_device": per_device, "d_head": 128},
+            "branch_shard": {"local_us": local_ms * 1e3, "allreduce_us": ar_ms * 1e3,
+                             "allreduce_bytes": w.batch * w.heads * 128 * 4,
+                             "cache_bytes_per_device": dev_bytes,
+                             "cache_elements_per_token_per_device": dc_dev + w.d_rope,
+                             "local_gbs": dev_bytes / (local_ms * 1e-3) / 1e9,
+                             "local_frac": dev_bytes / (local_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                             "note": "local = decode + step 3 of this device's branches (events "
+                                     "around them, the L2 flush outside); the all-reduce is NCCL "
+                                     "over the devices (none on one device)"},
+            "gpu_launches": (step.decoder.plan.launches + 1) * args.steps,
+            "clocks": clk.summary()}
+    if rank == 0:
+        print(json.dumps(line))
+    del step
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 # ----------------------------------------------------------------------------- steps 1 and 3
 def graph_time(body, steps, pre=None):
     """Mean device time (ms) of body() over `steps` calls replayed from one CUDA graph (no host
@@ -724,6 +821,10 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--parallel", choices=["dp", "branch"], default="dp",
+                    help="dp: every device decodes its own batch (weak scaling, the default line); "
+                         "branch: one layer's branches spread over the devices, steps 2-3 and an "
+                         "all-reduce (strong scaling)")
     ap.add_argument("--no-side", action="store_true",
                     help="skip the sustained leg and the other workloads' sub-records")
     ap.add_argument("--q-len", type=int, default=2,
@@ -738,6 +839,8 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.parallel == "branch":
+        return run_branch(args)
     if args.stage != "decode":
         return run_stage(args)
     return run_ours(args)

@@ -1,4 +1,4 @@
-"""Branch-parallel MLRA decode: one branch per device.
+"""Branch-parallel MLRA decode: the branches spread over devices, one or more per device.
 
 "Multi-Head Low-Rank Attention" (yunpan.plus page), sections 3.2 and 4: MLRA-B splits the latent
 state into B blocks c_1 .. c_B whose attentions are independent (each branch has its own softmax)
@@ -13,6 +13,11 @@ attention output:
 Device b's arrays are the b-th column blocks of the full ones (cut once, at load), and its decode is
 the single-branch decode (num_branches = 1) with the full layer's softmax scale and branch scale
 gamma = 1 / B.  The all-reduce goes through torch.distributed (NCCL between GPUs).
+
+With fewer devices than branches (G devices, G dividing B), device g keeps the g-th of G equal
+column blocks, i.e. B / G adjacent branches, and runs the B / G-branch decode on it (still with
+gamma = 1 / B); the branches' softmaxes stay independent, so the sum over devices is unchanged.
+The helpers below cut G equal blocks whatever G is.
 """
 from __future__ import annotations
 
@@ -51,24 +56,28 @@ def shard_wuv(w_uv: torch.Tensor, branch: int, num_branches: int) -> torch.Tenso
 
 
 class BranchShardStep:
-    """Steps 2 and 3 of one branch on this device, then the sum over the branch devices.
+    """Steps 2 and 3 of this device's branches, then the sum over the branch devices.
 
-    q_lat_b [N, H, d_c / B] and c_b [rows, d_c / B] are this device's blocks (``shard_queries``,
-    ``shard_latent``); q_rope, k_rope, seq_lens and page_table are the full (replicated) arrays;
-    w_uv_b [H, d_head, d_c / B] bf16 is ``shard_wuv``'s block, packed here once.  ``group`` is the
-    process group of the B branch devices (None: the default group); with ``reduce=False`` the
-    call returns this device's share and leaves the sum to the caller.  The returned tensor is the
-    step's output buffer, overwritten by the next call.
+    q_lat_b [N, H, d_c / G] and c_b [rows, d_c / G] are this device's blocks (``shard_queries``,
+    ``shard_latent`` with G shards); q_rope, k_rope, seq_lens and page_table are the full
+    (replicated) arrays; w_uv_b [H, d_head, d_c / G] bf16 is ``shard_wuv``'s block, packed here
+    once.  ``num_branches`` is the layer's B and ``branches_per_device`` B / G (default 1: one
+    branch per device).  ``group`` is the process group of the G devices (None: the default
+    group); with ``reduce=False`` the call returns this device's share and leaves the sum to the
+    caller.  The returned tensor is the step's output buffer, overwritten by the next call.
     """
 
     def __init__(self, q_lat_b, q_rope, c_b, k_rope, seq_lens, page_table, w_uv_b, *,
                  num_branches: int, softmax_scale: float, max_seq_len=None, page_size=0,
-                 group: Optional[dist.ProcessGroup] = None, reduce: bool = True):
+                 group: Optional[dist.ProcessGroup] = None, reduce: bool = True,
+                 branches_per_device: int = 1):
+        if branches_per_device < 1 or num_branches % branches_per_device:
+            raise ValueError(f"{branches_per_device} branches per device of {num_branches}")
         self.num_branches = num_branches
         self.group = group
         self.reduce = reduce
         self.decoder = mlra.Decoder(q_lat_b, q_rope, c_b, k_rope, seq_lens, page_table,
-                                    num_branches=1, softmax_scale=softmax_scale,
+                                    num_branches=branches_per_device, softmax_scale=softmax_scale,
                                     branch_scale=1.0 / num_branches, max_seq_len=max_seq_len,
                                     page_size=page_size)
         self.w_packed = mlra.pack_wuv(w_uv_b)
@@ -76,7 +85,8 @@ class BranchShardStep:
         self.y = torch.empty(N, H, w_uv_b.shape[1], dtype=torch.float32, device=q_lat_b.device)
 
     def local(self) -> torch.Tensor:
-        """This branch's share W^UV_{h,b} (gamma o_b) [N, H, d_head] (fp32)."""
+        """This device's share sum over its branches b of W^UV_{h,b} (gamma o_b) [N, H, d_head]
+        (fp32)."""
         return mlra.project(self.decoder(), self.w_packed, self.y)
 
     def __call__(self) -> torch.Tensor:

@@ -31,3 +31,18 @@ def test_branch_shards_sum_to_the_full_step(B, page_size):
     o, _ = oracle.decode(inp.q_lat, inp.q_rope, inp.c_kv, inp.k_rope, inp.seq_lens, inp.page_table,
                          B, w.sigma, w.gamma, max_seq_len=inp.max_seq_len, page_size=page_size)
     assert_close(y, oracle.project(o, w_uv.float()), f"B={B} paged={page_size}")
+
+
+def test_branch_bench_step_on_one_device_matches_the_oracle():
+    """The step that ``bench.py --parallel branch`` times, on one device (all B branches there,
+    no all-reduce): steps 2 and 3 against the oracle's decode followed by step 3."""
+    import bench
+    inp = small_inputs(B=4, lens=[513, 1, 129, 700], heads=64, page_size=64, seed=43)
+    w = inp.workload
+    step, w_uv, per_device = bench.branch_step(w, inp, torch.device("cuda", 0), world=1, rank=0)
+    assert per_device == 4
+    y = step()
+    torch.cuda.synchronize()
+    o, _ = oracle.decode(inp.q_lat, inp.q_rope, inp.c_kv, inp.k_rope, inp.seq_lens, inp.page_table,
+                         4, w.sigma, w.gamma, max_seq_len=inp.max_seq_len, page_size=64)
+    assert_close(y, oracle.project(o, w_uv.float()), "branch step, one device")
