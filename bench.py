@@ -781,29 +781,47 @@ def run_stage(args):
                            softmax_scale=w.sigma, branch_scale=w.gamma,
                            max_seq_len=inp.max_seq_len, page_size=w.page_size)
         y = torch.empty(N, H, d_head, dtype=torch.float32, device=dev)
+        dims_l = mlra.dims_for(q_lat2, q_rope2, c, kr, lens, pt, w.num_branches,
+                               max_seq_len=inp.max_seq_len, page_size=w.page_size)
+        ws_l = torch.empty(mlra.workspace_size_project(dims_l), dtype=torch.uint8, device=dev)
 
-        def body():
+        def front():
             # RoPE/append first: the absorption's weight copies then start under its tail
             # (they precede the absorption kernel's dependency wait)
             mlra.rope_append(q_rope_in, k_new, c_new, lens_in, pt, c, kr,
                              max_seq_len=inp.max_seq_len if pt is None else None,
                              page_size=w.page_size, q_rope_out=q_rope2)
             mlra.absorb(q_nope, w_uk, q_lat2)
+
+        def body():  # steps 2 and 3 in one call: step 3 merges the split sequences itself
+            front()
+            mlra.decode_project(q_lat2, q_rope2, c, kr, lens, pt, w_uv, num_branches=w.num_branches,
+                                softmax_scale=w.sigma, branch_scale=w.gamma,
+                                max_seq_len=inp.max_seq_len, page_size=w.page_size, y=y,
+                                workspace=ws_l)
+
+        def body_unfused():  # the attention path's combine kernel, then step 3
+            front()
             mlra.project(dec(), w_uv, y)
 
         for _ in range(args.warmup):
             body()
+            body_unfused()
         with ClockSampler(0) as clk:
             # L2 evicted before every step, as after the model's other layers: this layer's
             # weights and queries come from HBM (the timed region is the step alone)
             ms = graph_time(body, args.steps, pre=evict)
+            ms_unfused = graph_time(body_unfused, args.steps, pre=evict)
             # back to back, the 16 MB of this layer's weights may stay in L2 (the cache stream is
             # evict-first): a single-layer best case, reported beside the value
             ms_kept = graph_time(body, args.steps)
         line = {"metric": "attention layer decode step (steps 1-3, RoPE and cache append)",
                 "value": N / (ms * 1e-3), "unit": "tokens/s", "higher_is_better": True,
                 "ms_per_step": ms, "ms_per_step_back_to_back": ms_kept,
-                "kernels_per_step": 5 + (0 if dec.plan.launches == 2 else 1),
+                "ms_per_step_unfused": ms_unfused,
+                "kernels_per_step": 4 + (0 if dec.plan.launches == 2 else 1),
+                "note": "steps 2-3 through mlra_decode_project (no combine kernel); "
+                        "ms_per_step_unfused: mlra_decode (with its combine) then mlra_project",
                 "l2": "L2 flushed (read of 2x L2) before each step, outside the timed region"}
     line.update({"steps": args.steps, "warmup": args.warmup, "dtype": "bf16", "data": "synthetic",
                  "config": {"workload": w.name, "batch": N, "heads": H, "d_latent": d_c,

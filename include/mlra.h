@@ -224,6 +224,28 @@ mlra_status mlra_decode_static_scratch(const void* q_lat, const void* q_rope, co
 mlra_status mlra_project(const float* o, const void* w_packed, float* y, int N, int H, int d_latent,
                          int d_head, uint32_t* status, mlra_stream_t stream);
 
+/* Steps 2 and 3 of one attention layer in one call ("Multi-Head Low-Rank Attention", yunpan.plus
+ * page, section 1.3 steps 2 and 3 with the branch sum of sections 3 and 3.3):
+ *     y[s, h, :] = W_h o[s, h, :],   o = mlra_decode's output in MLRA_OUT_BRANCHES mode
+ * The attention kernel runs as in mlra_decode; instead of the combine kernel and mlra_project, one
+ * step-3 kernel merges the partial softmax states of the sequences the attention kernel split
+ * while it stages o[s, h] for its product (one launch and the fp32 o round trip fewer).
+ *   q_lat ... scales   as mlra_decode (bf16 inputs read in place; dims->out_mode must be
+ *                      MLRA_OUT_BRANCHES)
+ *   w_packed, d_head   as mlra_project (H * d_head * d_latent bf16 from mlra_pack_wuv)
+ *   y                  [N, H, d_head] fp32 device (written)
+ *   workspace          >= mlra_workspace_size_project(dims) bytes, 256-byte aligned; its status word
+ *                      is read with mlra_read_status
+ * No LSE output.  Errors: as mlra_decode and mlra_project; MLRA_ERR_UNSUPPORTED for summed mode,
+ * fp32 inputs or padded branch widths (the repack path).  The pages give no kernel for this
+ * fusion. */
+mlra_status mlra_workspace_size_project(const mlra_dims* dims, size_t* bytes_host);
+mlra_status mlra_decode_project(const void* q_lat, const void* q_rope, const void* c_kv,
+                                const void* k_rope, const int32_t* seq_lens,
+                                const int32_t* page_table, int B, const mlra_scales* scales,
+                                const void* w_packed, int d_head, float* y, const mlra_dims* dims,
+                                void* workspace, size_t ws_bytes, mlra_stream_t stream);
+
 /* Packs the step-3 weights once for mlra_project (they are model weights: pack at load time).
  *   w_uv     [H, d_head, d_latent] bf16 device, row-major: W_h row k = w_uv[h, k, :]
  *   w_packed H * d_head * d_latent bf16 device (written; same size, caller-owned): per head and

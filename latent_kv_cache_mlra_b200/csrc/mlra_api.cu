@@ -37,6 +37,10 @@ struct Plan {
   int limit = 0;       // bound on seq_lens
   int seg_cost = 0;    // tiles a sequence start costs a CTA (plan balance)
   bool self_plan = false;  // the decode kernel plans its ranges (no prep kernel)
+  bool m128 = false;   // K1M: two query tokens x 64 heads per CTA (128 rows)
+  int unit_tokens = 1; // query tokens per unit (virtual sequence)
+  int64_t units = 0;   // virtual sequences of the plan
+  int rows = 0;        // query rows per unit (heads, or 2 x 64 for K1M)
   size_t off_scratch = 0, off_ranges = 0, off_segs = 0, off_seqs = 0, off_flags = 0;
   size_t off_ml = 0, off_o = 0;
   size_t off_rq = 0, off_rqr = 0, off_rc = 0, off_rkr = 0, total = 0;
@@ -98,7 +102,13 @@ mlra_status make_plan(const mlra_dims* d, bool paged, int sms, Plan* pl, int q_l
   pl->dblk_k = dk;
   pl->variant = dk == 64 ? kV64 : dk == 128 ? kV128 : dk == 256 ? kV256 : kV512;
   pl->tile = variant_tile(pl->variant);
-  pl->n_groups = B * ((d->heads + 63) / 64);  // CTAs per range: (64-head group, branch)
+  // An even number of query tokens of 64 heads with 128-wide branches read in place: two tokens
+  // per CTA (K1M), 128 query rows against each cache tile
+  pl->m128 = q_len >= 2 && q_len % 2 == 0 && d->heads == 64 && dk == 128 && !pl->repack;
+  pl->unit_tokens = pl->m128 ? 2 : 1;
+  pl->units = Nv / pl->unit_tokens;
+  pl->rows = pl->m128 ? 128 : d->heads;
+  pl->n_groups = pl->m128 ? B : B * ((d->heads + 63) / 64);  // CTAs per range
   if (pl->n_groups > 148) return MLRA_ERR_UNSUPPORTED;
   pl->dck = B * dk;
   if (d->num_ranges > 0) pl->R = d->num_ranges;
@@ -107,7 +117,7 @@ mlra_status make_plan(const mlra_dims* d, bool paged, int sms, Plan* pl, int q_l
     pl->R = sms / pl->n_groups > 0 ? sms / pl->n_groups : 1;
   }
   if ((int64_t)pl->R * pl->n_groups > INT_MAX / 2) return MLRA_ERR_INVALID_ARG;
-  pl->slots = (int64_t)pl->R + Nv - 1;
+  pl->slots = (int64_t)pl->R + pl->units - 1;
   pl->limit = paged ? d->max_pages_per_seq * d->page_size : d->max_seq_len;
   if (!paged) pl->limit = d->max_seq_len;
   else if (d->max_seq_len > 0 && d->max_seq_len < pl->limit) pl->limit = d->max_seq_len;
@@ -116,7 +126,7 @@ mlra_status make_plan(const mlra_dims* d, bool paged, int sms, Plan* pl, int q_l
   if (Nv * ((pl->limit + pl->tile - 1) / pl->tile + pl->seg_cost) > INT_MAX)
     return MLRA_ERR_INVALID_ARG;
 
-  const int64_t N = Nv, H = d->heads;
+  const int64_t N = pl->units, H = pl->rows;
   size_t off = kAlign;  // status word + padding
   pl->self_plan = N <= kSelfPlanMaxSeqs;
   pl->off_scratch = off; off = align_up(off + 4 * (5 * (size_t)N + 2));
@@ -155,13 +165,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 tensor map with 64 x 64 boxes and 128-byte swizzle.  dims/strides in elements.
+// bf16 tensor map with boxes of 64 columns x box_rows rows and 128-byte swizzle.  dims/strides in
+// elements.
 bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-              const uint64_t* strides_elems) {
+              const uint64_t* strides_elems, uint32_t box_rows = 64) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gdim[3], gstride[2];
-  cuuint32_t box[3] = {64, 64, 1}, estr[3] = {1, 1, 1};
+  cuuint32_t box[3] = {64, box_rows, 1}, estr[3] = {1, 1, 1};
   for (int i = 0; i < rank; ++i) gdim[i] = dims[i];
   for (int i = 0; i + 1 < rank; ++i) gstride[i] = strides_elems[i] * 2;
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gdim, gstride, box,
@@ -264,6 +275,8 @@ mlra_status mlra_decode(const void* q_lat, const void* q_rope, const void* c_kv,
 }
 
 namespace {
+mlra_status check_product(const void* a, const void* b, const void* c, int N, int H, int d_in,
+                          int d_out);
 // The decode call: q_len query tokens per caller sequence (1: single-token decode), run as
 // dims->batch * q_len virtual sequences (virtual_len).
 mlra_status decode_impl(const void* q_lat, const void* q_rope, const void* c_kv,
@@ -271,8 +284,12 @@ mlra_status decode_impl(const void* q_lat, const void* q_rope, const void* c_kv,
                         int B, const mlra_scales* scales, float* out, float* lse,
                         const mlra_dims* dims, void* workspace, size_t ws_bytes,
                         mlra_stream_t stream, mlra_event_t k1_begin, mlra_event_t k1_end,
-                        int q_len) {
-  if (!q_lat || !q_rope || !c_kv || !k_rope || !seq_lens || !scales || !out || !dims)
+                        int q_len, const void* w_packed = nullptr, int d_head = 0,
+                        float* y = nullptr) {
+  // y != nullptr: step 3 follows in the same call (mlra_decode_project); `out` is then unused
+  // and the attention kernel's final rows go to a region of the workspace
+  const bool fused = y != nullptr;
+  if (!q_lat || !q_rope || !c_kv || !k_rope || !seq_lens || !scales || !(out || fused) || !dims)
     return MLRA_ERR_INVALID_ARG;
   if (B != dims->num_branches) return MLRA_ERR_INVALID_ARG;
   if (!std::isfinite(scales->softmax_scale) || !std::isfinite(scales->branch_scale))
@@ -288,7 +305,18 @@ mlra_status decode_impl(const void* q_lat, const void* q_rope, const void* c_kv,
   Plan pl;
   st = make_plan(dims, paged, sms, &pl, q_len);
   if (st != MLRA_OK) return st;
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || ws_bytes < pl.total)
+  size_t need = pl.total;
+  if (fused) {
+    if (dims->out_mode != MLRA_OUT_BRANCHES || pl.repack || q_len != 1 || !w_packed)
+      return MLRA_ERR_UNSUPPORTED;
+    const mlra_status pst = check_product(w_packed, w_packed, y, dims->batch, dims->heads,
+                                          dims->d_latent, d_head);
+    if (pst != MLRA_OK) return pst;
+    need = pl.total + align_up((size_t)dims->batch * dims->heads * dims->d_latent * sizeof(float));
+    out = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + pl.total);
+    lse = nullptr;
+  }
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || ws_bytes < need)
     return MLRA_ERR_WORKSPACE;
   if (!pl.repack && !(aligned16(q_lat) && aligned16(q_rope) && aligned16(c_kv) && aligned16(k_rope)))
     return MLRA_ERR_UNSUPPORTED;
@@ -303,7 +331,8 @@ mlra_status decode_impl(const void* q_lat, const void* q_rope, const void* c_kv,
   RangeInfo* ranges = reinterpret_cast<RangeInfo*>(ws + pl.off_ranges);
   SegDesc* segs = reinterpret_cast<SegDesc*>(ws + pl.off_segs);
   SeqInfo* seqs = reinterpret_cast<SeqInfo*>(ws + pl.off_seqs);
-  const int N = dims->batch * q_len, H = dims->heads, dblk = dims->d_latent / B;  // virtual
+  // virtual sequences (units) and query rows per unit
+  const int N = static_cast<int>(pl.units), H = pl.rows, dblk = dims->d_latent / B;
   const int64_t rows = dims->cache_rows;
 
   const void* kq = q_lat; const void* kqr = q_rope; const void* kc = c_kv; const void* kkr = k_rope;
@@ -333,7 +362,8 @@ mlra_status decode_impl(const void* q_lat, const void* q_rope, const void* c_kv,
     const uint64_t scm[1] = {(uint64_t)c_pitch};
     const uint64_t dkr[2] = {64, (uint64_t)rows};
     const uint64_t skr[1] = {(uint64_t)kr_pitch};
-    if (!make_map(&tq, kq, 3, dq, sq) || !make_map(&tqr, kqr, 3, dqr, sqr) ||
+    const uint32_t qbox = pl.m128 ? 128 : 64;  // one unit's query rows per box
+    if (!make_map(&tq, kq, 3, dq, sq, qbox) || !make_map(&tqr, kqr, 3, dqr, sqr, qbox) ||
         !make_map(&tc, kc, 2, dcm, scm) || !make_map(&tkr, kkr, 2, dkr, skr))
       return MLRA_ERR_CUDA;
   }
@@ -361,7 +391,8 @@ mlra_status decode_impl(const void* q_lat, const void* q_rope, const void* c_kv,
   if (!pl.self_plan) {
     PrepParams pp;
     pp.seq_lens = seq_lens; pp.N = N; pp.limit = pl.limit; pp.tile = pl.tile; pp.num_ranges = pl.R;
-    pp.seg_cost = pl.seg_cost; pp.scratch = plan_scratch; pp.q_per_seq = q_len;
+    pp.seg_cost = pl.seg_cost; pp.scratch = plan_scratch;
+    pp.q_per_seq = q_len / pl.unit_tokens; pp.unit_tokens = pl.unit_tokens;
     pp.ranges = ranges; pp.segs = segs; pp.seqs = seqs;
     pp.flags = cta_flags + grid;
     pp.out = out; pp.lse = lse; pp.H = H; pp.B = B; pp.out_width = out_width;
@@ -382,7 +413,8 @@ mlra_status decode_impl(const void* q_lat, const void* q_rope, const void* c_kv,
   p.max_seq_len = dims->max_seq_len;
   p.n_pages = paged ? rows / dims->page_size : 0;
   p.oob_row = static_cast<int>(rows);
-  p.q_per_seq = q_len;
+  p.q_per_seq = q_len / pl.unit_tokens;
+  p.unit_tokens = pl.unit_tokens;
   p.scale_log2 = scales->softmax_scale * 1.4426950408889634f;
   p.gamma = scales->branch_scale;
   p.write_final = summed ? 0 : 1;
@@ -393,11 +425,27 @@ mlra_status decode_impl(const void* q_lat, const void* q_rope, const void* c_kv,
   p.force_replan = std::getenv("MLRA_TEST_FORCE_REPLAN") != nullptr ? 1 : 0;
   if (k1_begin && cudaEventRecord(reinterpret_cast<cudaEvent_t>(k1_begin), s) != cudaSuccess)
     return MLRA_ERR_CUDA;
-  if (launch_decode(pl.variant, tq, tqr, tc, tkr, tout, tpart, p, grid, s) != cudaSuccess)
-    return MLRA_ERR_CUDA;
+  const cudaError_t launched = pl.m128 ? launch_decode_m128(tq, tqr, tc, tkr, p, grid, s)
+                                       : launch_decode(pl.variant, tq, tqr, tc, tkr, tout, tpart, p, grid, s);
+  if (launched != cudaSuccess) return MLRA_ERR_CUDA;
   if (k1_end && cudaEventRecord(reinterpret_cast<cudaEvent_t>(k1_end), s) != cudaSuccess)
     return MLRA_ERR_CUDA;
 
+  if (fused) {
+    // step 3 merges the split sequences itself: no combine kernel
+    ProjectParams pp3;
+    pp3.w_packed = w_packed;
+    pp3.x = out; pp3.y = y; pp3.status = status;
+    pp3.N = N; pp3.H = H; pp3.d_in = dims->d_latent; pp3.d_out = d_head;
+    pp3.out_bf16 = 0;
+    pp3.timeout_ns = kTimeoutNs;
+    pp3.merge = 1;
+    pp3.seqs = seqs; pp3.part_ml = part_ml; pp3.part_o = part_o;
+    pp3.B = B; pp3.dblk = dblk; pp3.gamma = scales->branch_scale;
+    pp3.cta_flags = cta_flags; pp3.n_flag_slots = grid + (pl.self_plan ? 0 : 1);
+    if (launch_project(pp3, s) != cudaSuccess) return MLRA_ERR_CUDA;
+    return MLRA_OK;
+  }
   CombineParams cp;
   cp.cta_flags = cta_flags; cp.n_flag_slots = grid + (pl.self_plan ? 0 : 1); cp.status = status;
   cp.seqs = seqs; cp.part_o = part_o; cp.part_ml = part_ml; cp.out = out; cp.lse = lse;
@@ -457,6 +505,26 @@ mlra_status mlra_workspace_size_multi(const mlra_dims* dims, int q_len, size_t* 
   if (st != MLRA_OK) return st;
   *bytes_host = pl.total;
   return MLRA_OK;
+}
+
+mlra_status mlra_workspace_size_project(const mlra_dims* dims, size_t* bytes_host) {
+  if (!dims || !bytes_host) return MLRA_ERR_INVALID_ARG;
+  size_t base = 0;
+  const mlra_status st = mlra_workspace_size(dims, &base);
+  if (st != MLRA_OK) return st;
+  *bytes_host = base + align_up((size_t)dims->batch * dims->heads * dims->d_latent * sizeof(float));
+  return MLRA_OK;
+}
+
+mlra_status mlra_decode_project(const void* q_lat, const void* q_rope, const void* c_kv,
+                                const void* k_rope, const int32_t* seq_lens,
+                                const int32_t* page_table, int B, const mlra_scales* scales,
+                                const void* w_packed, int d_head, float* y, const mlra_dims* dims,
+                                void* workspace, size_t ws_bytes, mlra_stream_t stream) {
+  if (!y) return MLRA_ERR_INVALID_ARG;
+  return decode_impl(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table, B, scales, nullptr,
+                     nullptr, dims, workspace, ws_bytes, stream, nullptr, nullptr, 1, w_packed,
+                     d_head, y);
 }
 
 mlra_status mlra_decode_static_scratch(const void* q_lat, const void* q_rope, const void* c_kv,
@@ -528,6 +596,10 @@ mlra_status run_product(const float* x, const void* w_packed, void* y, int N, in
   p.N = N; p.H = H; p.d_in = d_in; p.d_out = d_out;
   p.out_bf16 = out_bf16 ? 1 : 0;
   p.timeout_ns = kTimeoutNs;
+  p.merge = 0;
+  p.seqs = nullptr; p.part_ml = nullptr; p.part_o = nullptr;
+  p.B = 1; p.dblk = d_in; p.gamma = 1.f;
+  p.cta_flags = nullptr; p.n_flag_slots = 0;
   if (launch_project(p, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MLRA_ERR_CUDA;
   return MLRA_OK;
 }

@@ -133,16 +133,17 @@ __device__ __forceinline__ int tile_row(const int32_t* page_table, int max_pages
 
 constexpr int kDecodeThreads = 224;
 
-// In-kernel plan for N <= kSelfPlanMaxSeqs = 64.  Warp 0 holds sequences lane and lane + 32.
+// In-kernel plan for N <= kSelfPlanMaxSeqs = 64.  Warp 0's lane l holds the adjacent sequences
+// 2 l and 2 l + 1, so one warp scan covers the batch.
 //
 // plan_read_lengths: the lengths (virtual lengths for several tokens per sequence), clamped to
 // [0, limit]; bit 6 of `bits` reports a length outside that range.
 //
 // plan_segments: scans the real and virtual tile prefixes (mlra_plan.cuh) across the warp, finds
 // the sequence holding each of the range's two virtual boundaries with one ballot, and lets every
-// sequence that overlaps the range write its own segment at its rank in the warp (shared memory
-// only).  Per lane it returns in `bits`: bit c (c = 0, 1) sequence 32 c + lane has its first tile
-// in this range, bit 2 + c its last tile, bit 4 + c it is empty.  Returns the segment count.
+// sequence that overlaps the range write its own segment at its rank (shared memory only).  Per
+// lane it adds to `bits`: bit c (c = 0, 1) sequence 2 lane + c has its first tile in this range,
+// bit 2 + c its last tile, bit 4 + c it is empty.  Returns the segment count.
 //
 // plan_commit: the plan's global records, written once the lengths are final: the CTAs of group 0
 // record for the combine kernel the ranges holding each sequence's first and last tile, CTA 0
@@ -150,98 +151,99 @@ constexpr int kDecodeThreads = 224;
 //
 // The decode kernel runs the first two before its dependency wait on the lengths as they are then
 // (a speculative plan), reads the lengths again after the wait and keeps the plan when they are
-// unchanged (plan_verify).
+// unchanged.
 __device__ __forceinline__ void plan_read_lengths(const DecodeParams& p, int lane, int (&L)[2],
                                                   uint32_t& bits) {
   bits = 0;
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
-    const int i = 32 * c + lane;
+    const int i = 2 * lane + c;
     int x = i < p.N ? (p.q_per_seq == 1 ? __ldcg(p.seq_lens + i)
                                         : __ldcg(p.seq_lens + i / p.q_per_seq) -
-                                              (p.q_per_seq - 1 - i % p.q_per_seq))
+                                              (p.q_per_seq - 1 - i % p.q_per_seq) * p.unit_tokens)
                     : 0;
-    if (i < p.N && (x < 0 || x > p.limit)) {
+    if (i < p.N && (x - (p.unit_tokens - 1) < 0 || x > p.limit)) {  // (or the unit's first token)
       bits |= 64u;
-      x = x < 0 ? 0 : p.limit;
+      x = x < 0 ? 0 : (x > p.limit ? p.limit : x);
     }
     L[c] = x;
   }
 }
 
-__device__ __noinline__ int plan_segments(const DecodeParams& p, int range, const int (&L)[2],
-                                          uint8_t* plan, uint32_t& bits) {
+// floor(a / b) for 0 <= a < 2^53, b >= 1.  Below 2^24 a single-precision quotient is within one
+// of the result and one correction step each way makes it exact (the common case: a few thousand
+// virtual tiles times the range index); above, a double division and the same correction.
+__device__ __forceinline__ int64_t floor_div_i64(int64_t a, int64_t b) {
+  int64_t q;
+  if (a < (int64_t{1} << 24))
+    q = static_cast<int64_t>(__fdiv_rz(static_cast<float>(a), static_cast<float>(b)));
+  else
+    q = static_cast<int64_t>(__ddiv_rz(static_cast<double>(a), static_cast<double>(b)));
+  if (q * b > a) --q;
+  if ((q + 1) * b <= a) ++q;
+  return q;
+}
+
+__device__ __forceinline__ int plan_segments(const DecodeParams& p, int range, int L0, int L1,
+                                             uint8_t* plan, uint32_t& bits) {
   int4* list = reinterpret_cast<int4*>(plan);                       // [kSelfPlanMaxSeqs]
   int32_t* lens = reinterpret_cast<int32_t*>(list + kSelfPlanMaxSeqs);
-  const int lane = threadIdx.x & 31, N = p.N;
-  int t[2], lo[2], hi[2], vlo[2], vhi[2];
-  int carry_t = 0, carry_v = 0;
+  const int lane = threadIdx.x & 31, N = p.N, cost = p.seg_cost;
+  const int i0 = 2 * lane, i1 = i0 + 1;
+  const int tile_shift = p.tile == 64 ? 6 : 7;  // tiles of 64 or 128 positions
+  const int t0 = i0 < N ? (L0 + p.tile - 1) >> tile_shift : 0;
+  const int t1 = i1 < N ? (L1 + p.tile - 1) >> tile_shift : 0;
+  const int v0 = t0 > 0 ? t0 + cost : 0, v1 = t1 > 0 ? t1 + cost : 0;
   bits &= 64u;
+  if (i0 < N && t0 == 0) bits |= 16u;
+  if (i1 < N && t1 == 0) bits |= 32u;
+  if (i0 < N) lens[i0] = L0;
+  if (i1 < N) lens[i1] = L1;
+  int x = t0 + t1, v = v0 + v1;
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    const int i = 32 * c + lane;
-    t[c] = i < N ? (L[c] + p.tile - 1) / p.tile : 0;
-    if (i < N && t[c] == 0) bits |= 16u << c;
-    int x = t[c], v = t[c] > 0 ? t[c] + p.seg_cost : 0;
-    const int vt = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {  // inclusive scans
-      const int yx = __shfl_up_sync(kFull, x, o), yv = __shfl_up_sync(kFull, v, o);
-      if (lane >= o) {
-        x += yx;
-        v += yv;
-      }
+  for (int o = 1; o < 32; o <<= 1) {  // inclusive scans of the pairs' tiles and virtual tiles
+    const int yx = __shfl_up_sync(kFull, x, o), yv = __shfl_up_sync(kFull, v, o);
+    if (lane >= o) {
+      x += yx;
+      v += yv;
     }
-    hi[c] = x + carry_t;
-    lo[c] = hi[c] - t[c];
-    vhi[c] = v + carry_v;
-    vlo[c] = vhi[c] - vt;
-    carry_t += __shfl_sync(kFull, x, 31);
-    carry_v += __shfl_sync(kFull, v, 31);
-    if (i < N) lens[i] = L[c];
   }
-  const int64_t total = carry_t, vtotal = carry_v;
+  const int total = __shfl_sync(kFull, x, 31), vtotal = __shfl_sync(kFull, v, 31);
+  const int lo0 = x - t0 - t1, hi0 = lo0 + t0, lo1 = hi0, hi1 = lo1 + t1;
+  const int vlo0 = v - v0 - v1, vhi0 = vlo0 + v0, vlo1 = vhi0, vhi1 = vlo1 + v1;
   const int64_t R = effective_ranges(p.num_ranges, total);
-  int n = 0;
-  if (range < R && total > 0) {
-    // real tile of a virtual position: the sequence whose virtual interval holds it
-    auto tile_of = [&](int64_t v) -> int64_t {
-      int64_t g = 0;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const bool own = t[c] > 0 && vlo[c] <= v && v < vhi[c];
-        const uint32_t m = __ballot_sync(kFull, own);
-        if (m) {
-          const int src = __ffs(m) - 1;
-          const int64_t o = v - vlo[c] - p.seg_cost;
-          const int64_t mine = lo[c] + (o > 0 ? o : 0);
-          g = __shfl_sync(kFull, mine, src);
-        }
-      }
-      return g;
-    };
-    const int64_t g0 = tile_of((range * vtotal) / R);
-    const int64_t g1 = range + 1 < R ? tile_of(((range + 1) * vtotal) / R) : total;
-    int base = 0;
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const int i = 32 * c + lane;
-      const bool ov = t[c] > 0 && lo[c] < g1 && hi[c] > g0;
-      const uint32_t m = __ballot_sync(kFull, ov);
-      if (ov) {
-        const int64_t a = g0 > lo[c] ? g0 : lo[c], e = g1 < hi[c] ? g1 : hi[c];
-        const bool whole = a == lo[c] && e == hi[c];
-        list[base + __popc(m & ((1u << lane) - 1u))] =
-            make_int4(i, static_cast<int>(a - lo[c]), static_cast<int>(e - a),
-                      L[c] | (whole ? (int32_t)0x80000000u : 0));
-        if (a == lo[c]) bits |= 1u << c;  // the sequence's first tile is in this range
-        if (e == hi[c]) bits |= 4u << c;  // ... its last tile
-      }
-      base += __popc(m);
-    }
-    n = base;
+  if (range >= R || total == 0) return 0;
+  // real tile of a virtual position: the sequence whose virtual interval holds it
+  auto tile_of = [&](int64_t vp) -> int {
+    const bool own0 = t0 > 0 && vlo0 <= vp && vp < vhi0;
+    const bool own1 = t1 > 0 && vlo1 <= vp && vp < vhi1;
+    const int64_t o = vp - (own0 ? vlo0 : vlo1) - cost;
+    const int mine = (own0 ? lo0 : lo1) + static_cast<int>(o > 0 ? o : 0);
+    const uint32_t m = __ballot_sync(kFull, own0 || own1);
+    return __shfl_sync(kFull, mine, m ? __ffs(m) - 1 : 0);
+  };
+  const int g0 = tile_of(floor_div_i64(range * (int64_t)vtotal, R));
+  const int g1 = range + 1 < R ? tile_of(floor_div_i64((range + 1) * (int64_t)vtotal, R)) : total;
+  const bool ov0 = t0 > 0 && lo0 < g1 && hi0 > g0;
+  const bool ov1 = t1 > 0 && lo1 < g1 && hi1 > g0;
+  const uint32_t m0 = __ballot_sync(kFull, ov0), m1 = __ballot_sync(kFull, ov1);
+  const uint32_t below = (1u << lane) - 1u;
+  const int rank0 = __popc(m0 & below) + __popc(m1 & below);
+  if (ov0) {
+    const int a = g0 > lo0 ? g0 : lo0, e = g1 < hi0 ? g1 : hi0;
+    list[rank0] = make_int4(i0, a - lo0, e - a,
+                            L0 | ((a == lo0 && e == hi0) ? (int32_t)0x80000000u : 0));
+    if (a == lo0) bits |= 1u;  // the sequence's first tile is in this range
+    if (e == hi0) bits |= 4u;  // ... its last tile
   }
-  return n;
+  if (ov1) {
+    const int a = g0 > lo1 ? g0 : lo1, e = g1 < hi1 ? g1 : hi1;
+    list[rank0 + (ov0 ? 1 : 0)] = make_int4(i1, a - lo1, e - a,
+                                            L1 | ((a == lo1 && e == hi1) ? (int32_t)0x80000000u : 0));
+    if (a == lo1) bits |= 2u;
+    if (e == hi1) bits |= 8u;
+  }
+  return __popc(m0) + __popc(m1);
 }
 
 __device__ __forceinline__ void plan_commit(const DecodeParams& p, int range, int group,
@@ -249,7 +251,7 @@ __device__ __forceinline__ void plan_commit(const DecodeParams& p, int range, in
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
-    const int i = 32 * c + lane;
+    const int i = 2 * lane + c;
     if (group == 0) {
       if (bits & (1u << c)) p.seqs[i].r0 = range;
       if (bits & (4u << c)) p.seqs[i].r1 = range;
@@ -381,7 +383,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   uint32_t plan_bits = 0;
   if (p.self_plan && warp == 0) {
     plan_read_lengths(p, lane, spec_len, plan_bits);
-    const int n = plan_segments(p, range, spec_len, plan, plan_bits);
+    const int n = plan_segments(p, range, spec_len[0], spec_len[1], plan, plan_bits);
     if (lane == 0) *plan_count = n;
   }
   tc_fence_before();
@@ -459,7 +461,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       const bool same = __all_sync(kFull, len_now[0] == spec_len[0] && len_now[1] == spec_len[1]);
       if (!same || p.force_replan) {
         plan_bits = bits_now;
-        const int n = plan_segments(p, range, len_now, plan, plan_bits);
+        const int n = plan_segments(p, range, len_now[0], len_now[1], plan, plan_bits);
         if (lane == 0) *plan_count = n;
       }
       if (lane == 0) *plan_stale = (!same || p.force_replan) ? 1 : 0;

@@ -26,19 +26,25 @@ struct alignas(16) SegDesc {
 };
 struct alignas(8) SeqInfo { int32_t r0, r1; };
 
-// Several query tokens per sequence (a speculative or chunked-prefill step): the decode runs
-// N = (caller sequences) x q_per_seq virtual sequences, v = s q_per_seq + t for token t of caller
-// sequence s, over s's cache rows; token t is at position seq_lens[s] - q_per_seq + t and sees the
-// positions up to its own (causal), so v's length is seq_lens[s] - (q_per_seq - 1 - t).
-__host__ __device__ inline int virtual_len(const int32_t* seq_lens, int v, int q_per_seq) {
-  if (q_per_seq == 1) return seq_lens[v];
-  return seq_lens[v / q_per_seq] - (q_per_seq - 1 - v % q_per_seq);
+// Several query tokens per sequence (a speculative or chunked-prefill step): the q tokens of
+// caller sequence s are grouped into units of `unit_tokens` (1, or 2 for the kernel with 128 query
+// rows) and the decode runs N = (caller sequences) x units_per_seq virtual sequences,
+// v = s units_per_seq + u for unit u, over s's cache rows.  Token t is at position
+// seq_lens[s] - q + t and sees the positions up to its own (causal), i.e. its length is
+// seq_lens[s] - (q - 1 - t); a unit's length is that of its last token,
+//   seq_lens[s] - (units_per_seq - 1 - u) unit_tokens,
+// and its first token's length is unit_tokens - 1 less.
+__host__ __device__ inline int virtual_len(const int32_t* seq_lens, int v, int units_per_seq,
+                                           int unit_tokens) {
+  if (units_per_seq == 1) return seq_lens[v];
+  return seq_lens[v / units_per_seq] - (units_per_seq - 1 - v % units_per_seq) * unit_tokens;
 }
 
 struct PrepParams {
   const int32_t* seq_lens;    // caller lengths [N / q_per_seq]
   int N, limit, tile, num_ranges;
-  int q_per_seq;              // query tokens per caller sequence (virtual_len)
+  int q_per_seq;              // units (virtual sequences) per caller sequence (virtual_len)
+  int unit_tokens;            // query tokens per unit (virtual_len)
   int seg_cost;               // tiles a sequence start costs a CTA (plan balance)
   int32_t* scratch;           // [5 N + 2] plan arrays when N is too large for shared memory
   RangeInfo* ranges;          // [num_ranges]
@@ -74,8 +80,9 @@ struct DecodeParams {
   int page_size, max_pages, max_seq_len;
   int64_t n_pages;            // pages in the pool (paged layout)
   int oob_row;                // tile row used for an invalid page id (reads zeros)
-  int q_per_seq;              // query tokens per caller sequence: virtual sequence v reads the
-                              // cache rows of caller sequence v / q_per_seq (virtual_len)
+  int q_per_seq;              // units per caller sequence: virtual sequence v reads the cache
+                              // rows of caller sequence v / q_per_seq (virtual_len)
+  int unit_tokens;            // query tokens per unit (virtual_len)
   float scale_log2;           // softmax_scale * log2(e)
   float gamma;                // branch_scale
   int write_final;            // whole-sequence segments write `out` directly
@@ -111,6 +118,17 @@ struct ProjectParams {
   int N, H, d_in, d_out;
   int out_bf16;
   uint64_t timeout_ns;
+  // Step 3 straight after the attention kernel (no combine kernel): x[s] is the attention
+  // kernel's final output for sequences held in one part (or empty), else the merge of the
+  // partial results of its parts, times gamma (mlra_merge.cuh).
+  int merge;
+  const SeqInfo* seqs;        // [N] parts r0 .. r1 of each sequence (slots r + s)
+  const float* part_ml;       // [slots, H, B, 2]
+  const float* part_o;        // [slots, H, d_in]
+  int B, dblk;                // branches, branch width (d_in = B dblk)
+  float gamma;
+  const uint32_t* cta_flags;  // the attention kernel's status slots, ORed into *status
+  int n_flag_slots;
 };
 
 // RoPE of the new token's query and key, and its append to the cache (K7).
@@ -151,6 +169,11 @@ cudaError_t launch_decode(Variant v, const CUtensorMap& tq, const CUtensorMap& t
                           const CUtensorMap& tc, const CUtensorMap& tkr, const CUtensorMap& tout,
                           const CUtensorMap& tpart, const DecodeParams& p, int grid,
                           cudaStream_t st);
+// K1M: 128 query rows per CTA (two tokens x 64 heads), branch width 128; tq / tqr with boxes of
+// 64 columns x 128 rows over [width, 128, units]
+cudaError_t launch_decode_m128(const CUtensorMap& tq, const CUtensorMap& tqr,
+                               const CUtensorMap& tc, const CUtensorMap& tkr,
+                               const DecodeParams& p, int grid, cudaStream_t st);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t st);
 cudaError_t launch_repack(const RepackParams& p, cudaStream_t st);
 cudaError_t launch_project(const ProjectParams& p, cudaStream_t st);

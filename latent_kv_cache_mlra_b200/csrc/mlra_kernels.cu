@@ -15,6 +15,7 @@
 #include <math_constants.h>
 
 #include "mlra_decode_kernel.cuh"
+#include "mlra_decode_m128_kernel.cuh"
 #include "mlra_merge.cuh"
 #include "mlra_project_kernel.cuh"
 #include "sm100_ptx.cuh"
@@ -62,10 +63,10 @@ __global__ void __launch_bounds__(1024) mlra_prep_kernel(const PrepParams p) {
     const int i = b0 + tid;
     int x[2] = {0, 0};  // tiles, virtual tiles
     if (i < N) {
-      int L = virtual_len(p.seq_lens, i, p.q_per_seq);
-      if (L < 0 || L > p.limit) {
+      int L = virtual_len(p.seq_lens, i, p.q_per_seq, p.unit_tokens);
+      if (L - (p.unit_tokens - 1) < 0 || L > p.limit) {  // (a unit's first token too short)
         atomicOr(&flags, kFlagBadLength);
-        L = L < 0 ? 0 : p.limit;
+        L = L < 0 ? 0 : (L > p.limit ? p.limit : L);
       }
       lens[i] = L;
       x[0] = (L + p.tile - 1) / p.tile;
@@ -226,6 +227,29 @@ cudaError_t launch_decode(Variant v, const CUtensorMap& tq, const CUtensorMap& t
 #undef X
     default: return cudaErrorInvalidValue;
   }
+}
+
+// ----------------------------------------------------------------------------- K1M
+constexpr int kM128Stages = 4;
+
+cudaError_t launch_decode_m128(const CUtensorMap& tq, const CUtensorMap& tqr,
+                               const CUtensorMap& tc, const CUtensorMap& tkr,
+                               const DecodeParams& p, int grid, cudaStream_t st) {
+  using C = DecodeM128Cfg<kM128Stages>;
+  auto kern = mlra_decode_m128_kernel<kM128Stages>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kDecodeM128Threads);
+  cfg.dynamicSmemBytes = C::SMEM_ALLOC;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tq, tqr, tc, tkr, p);
 }
 
 // ----------------------------------------------------------------------------- K2

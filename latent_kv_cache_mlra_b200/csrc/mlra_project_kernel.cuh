@@ -20,6 +20,10 @@
 //     time; the epilogue reads D with tcgen05.ld, transposes it through shared memory and writes
 //     x_out in fp32 or bf16 with 16-byte stores (64 consecutive rows of one sequence).
 // The work is bound by streaming A (H d_out d_in bf16) from HBM.
+//
+// Merge mode (step 3 fused behind the attention kernel, no combine kernel between them): the x
+// row of a sequence split over several work ranges is merged from its partial results while it is
+// staged (the combine's fold, mlra_merge.cuh), and block 0 writes the call's status word.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -27,11 +31,12 @@
 #include <cuda_bf16.h>
 
 #include "mlra_internal.h"
+#include "mlra_merge.cuh"
 #include "sm100_ptx.cuh"
 
 namespace mlra {
 
-constexpr int kProjThreads = 128;
+constexpr int kProjThreads = 256;  // warps 0-3 also read the accumulator
 constexpr int kProjM = 64;     // rows of A_h per CTA
 constexpr int kProjN = 64;     // sequences per CTA
 constexpr int kProjBox = 8192; // one [64 x 64] bf16 box
@@ -139,7 +144,94 @@ mlra_project_kernel(const __grid_constant__ ProjectParams p) {
   // (rows past the batch as zeros); the loads of 8 chunks are issued before any is converted.
   constexpr int kU = 8;
   const int chunks = npad * KB * 8;
-  for (int base = threadIdx.x; base < chunks; base += kProjThreads * kU) {
+  if (p.merge && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 32) {
+    // the call's status word: the bits every attention CTA (and the prep kernel) raised
+    uint32_t f = 0;
+    for (int i = threadIdx.x; i < p.n_flag_slots; i += 32) f |= __ldcg(p.cta_flags + i);
+    f = __reduce_or_sync(0xffffffffu, f);
+    if (threadIdx.x == 0) *p.status = f;  // (a time-out of this kernel is ORed in after it)
+  }
+  if (p.merge) {
+    // 8 columns (one branch) of row r per chunk: the attention kernel's final row, or the merge
+    // of the sequence's parts.  Each thread takes two chunks at a time and keeps the loads of
+    // both chunks' next kMergeBatch parts in flight (one memory round trip covers them).
+    constexpr int kMergeBatch = 4;
+    for (int base = threadIdx.x; base < chunks; base += 2 * kProjThreads) {
+      int np[2], r0[2], s_[2];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int idx = base + c * kProjThreads;
+        const int r = idx / (KB * 8);
+        np[c] = 0;
+        r0[c] = 0;
+        s_[c] = n0 + r;
+        if (idx < chunks && r < rows_n) {
+          const int2 si = __ldcg(reinterpret_cast<const int2*>(p.seqs + s_[c]));
+          np[c] = si.y - si.x + 1;
+          r0[c] = si.x;
+        } else {
+          np[c] = -1;  // a padding row or past the chunks: zeros
+        }
+      }
+      float4 a[2], b4[2];
+      MergeState lo[2] = {merge_empty(), merge_empty()}, hi[2] = {merge_empty(), merge_empty()};
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        a[c] = b4[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+        const int idx = base + c * kProjThreads;
+        const int cidx = idx % (KB * 8);
+        if (np[c] == 0 || np[c] == 1) {
+          const float4* src = reinterpret_cast<const float4*>(p.x + ((int64_t)s_[c] * p.H + h) * p.d_in + cidx * 8);
+          a[c] = __ldcg(src);
+          b4[c] = __ldcg(src + 1);
+        }
+      }
+      const int npmax = max(np[0], np[1]);
+      for (int q0 = 0; npmax > 1 && q0 < npmax; q0 += kMergeBatch) {
+        float2 ml[2][kMergeBatch];
+        float4 va[2][kMergeBatch], vb[2][kMergeBatch];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int col = ((base + c * kProjThreads) % (KB * 8)) * 8;
+          const int br = col / p.dblk;
+#pragma unroll
+          for (int u = 0; u < kMergeBatch; ++u) {
+            if (np[c] > 1 && q0 + u < np[c]) {
+              const int64_t row = ((int64_t)r0[c] + q0 + u + s_[c]) * p.H + h;
+              ml[c][u] = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (row * p.B + br) * 2));
+              const float4* o = reinterpret_cast<const float4*>(p.part_o + row * p.d_in + col);
+              va[c][u] = __ldcg(o);
+              vb[c][u] = __ldcg(o + 1);
+            }
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int u = 0; u < kMergeBatch; ++u)
+            if (np[c] > 1 && q0 + u < np[c]) {
+              merge_into(lo[c], ml[c][u].x, ml[c][u].y, va[c][u]);
+              merge_into(hi[c], ml[c][u].x, ml[c][u].y, vb[c][u]);
+            }
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int idx = base + c * kProjThreads;
+        if (idx >= chunks) continue;
+        const int r = idx / (KB * 8), cidx = idx - r * (KB * 8);
+        const int kb = cidx >> 3, j = cidx & 7;
+        if (np[c] > 1) {
+          const float sc = p.gamma / lo[c].l;
+          a[c] = make_float4(lo[c].acc.x * sc, lo[c].acc.y * sc, lo[c].acc.z * sc, lo[c].acc.w * sc);
+          b4[c] = make_float4(hi[c].acc.x * sc, hi[c].acc.y * sc, hi[c].acc.z * sc, hi[c].acc.w * sc);
+        }
+        *reinterpret_cast<uint4*>(sX + kb * kProjBox + r * 128 + ((j ^ (r & 7)) << 4)) =
+            make_uint4(pack_bf16x2(a[c].x, a[c].y), pack_bf16x2(a[c].z, a[c].w),
+                       pack_bf16x2(b4[c].x, b4[c].y), pack_bf16x2(b4[c].z, b4[c].w));
+      }
+    }
+  }
+  for (int base = p.merge ? chunks : threadIdx.x; base < chunks; base += kProjThreads * kU) {
     float4 va[kU], vb[kU];
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
@@ -198,13 +290,15 @@ mlra_project_kernel(const __grid_constant__ ProjectParams p) {
     // 32 q .. 32 q + 31 (the sequences n0 + column).  They go through shared memory (the A boxes
     // are free now) as sT[column][row], so that each output row segment of 64 values leaves as
     // 16-byte stores: one scattered 4-byte store per value costs several times more.
-    uint32_t r[32];
-    tmem_ld16x2_32(tmem + ((uint32_t)(32 * warp) << 16), r);
-    tmem_wait_ld();
     float* sT = reinterpret_cast<float*>(sW);  // [64][64] fp32 = 16 KB <= 2 * KB * 8 KB
-    const int q = lane >> 4, rr = 16 * warp + (lane & 15);
+    if (warp < 4) {  // the accumulator's sub-partitions
+      uint32_t r[32];
+      tmem_ld16x2_32(tmem + ((uint32_t)(32 * warp) << 16), r);
+      tmem_wait_ld();
+      const int q = lane >> 4, rr = 16 * warp + (lane & 15);
 #pragma unroll
-    for (int k = 0; k < 32; ++k) sT[(32 * q + k) * kProjM + rr] = __uint_as_float(r[k]);
+      for (int k = 0; k < 32; ++k) sT[(32 * q + k) * kProjM + rr] = __uint_as_float(r[k]);
+    }
     __syncthreads();
     if (p.out_bf16) {
       // 8 rows (16 bytes) per store

@@ -29,7 +29,8 @@ EXPORTS = ("mlra_workspace_size", "mlra_decode", "mlra_decode_profiled", "mlra_q
            "mlra_read_status", "mlra_debug_resolve_rows", "mlra_plan_host",
            "mlra_plan_segments_host", "mlra_project", "mlra_pack_wuv", "mlra_absorb",
            "mlra_pack_wuk", "mlra_rope_append", "mlra_decode_multi", "mlra_workspace_size_multi",
-           "mlra_status_string", "mlra_version")
+           "mlra_decode_project", "mlra_workspace_size_project", "mlra_status_string",
+           "mlra_version")
 
 
 class Dims(ctypes.Structure):
@@ -96,6 +97,10 @@ def lib() -> ctypes.CDLL:
                                         ctypes.c_size_t, vp]
         L.mlra_workspace_size_multi.argtypes = [ctypes.POINTER(Dims), ctypes.c_int,
                                                 ctypes.POINTER(ctypes.c_size_t)]
+        L.mlra_workspace_size_project.argtypes = [ctypes.POINTER(Dims), ctypes.POINTER(ctypes.c_size_t)]
+        L.mlra_decode_project.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.POINTER(Scales),
+                                          vp, ctypes.c_int, vp, ctypes.POINTER(Dims), vp,
+                                          ctypes.c_size_t, vp]
         L.mlra_status_string.argtypes = [ctypes.c_int]
         L.mlra_status_string.restype = ctypes.c_char_p
         L.mlra_version.argtypes = []
@@ -104,7 +109,7 @@ def lib() -> ctypes.CDLL:
                   "mlra_read_status", "mlra_debug_resolve_rows", "mlra_plan_host",
                   "mlra_plan_segments_host", "mlra_project", "mlra_pack_wuv", "mlra_absorb",
                   "mlra_pack_wuk", "mlra_rope_append", "mlra_decode_multi",
-                  "mlra_workspace_size_multi"):
+                  "mlra_workspace_size_multi", "mlra_decode_project", "mlra_workspace_size_project"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -323,6 +328,39 @@ def decode_multi(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table=None, *, num_
                                    _ptr(workspace), workspace.numel(), ctypes.c_void_p(st)),
            "mlra_decode_multi")
     return out, lse
+
+
+def workspace_size_project(dims: Dims) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().mlra_workspace_size_project(ctypes.byref(dims), ctypes.byref(n)),
+           "mlra_workspace_size_project")
+    return n.value
+
+
+def decode_project(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table, w_packed, *,
+                   num_branches: int, softmax_scale: float, d_head: int = 128,
+                   branch_scale: Optional[float] = None, max_seq_len=None, page_size=0, y=None,
+                   workspace=None, num_ranges=0, stream=None):
+    """``mlra_decode_project``: steps 2 and 3 of one layer in one call (the attention kernel, then
+    the step-3 product that merges split sequences itself).  ``w_packed`` from ``pack_wuv``.
+    Returns y [N, H, d_head] fp32."""
+    gamma = 1.0 / num_branches if branch_scale is None else branch_scale
+    dims = dims_for(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table, num_branches,
+                    max_seq_len=max_seq_len, page_size=page_size, num_ranges=num_ranges)
+    N, H, _ = q_lat.shape
+    dev = q_lat.device
+    if y is None:
+        y = torch.empty(N, H, d_head, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(workspace_size_project(dims), dtype=torch.uint8, device=dev)
+    st = stream if stream is not None else torch.cuda.current_stream(dev).cuda_stream
+    scales = Scales(softmax_scale, gamma)
+    _check(lib().mlra_decode_project(_ptr(q_lat), _ptr(q_rope), _ptr(c_kv), _ptr(k_rope),
+                                     _ptr(seq_lens), _ptr(page_table), num_branches,
+                                     ctypes.byref(scales), _ptr(w_packed), d_head, _ptr(y),
+                                     ctypes.byref(dims), _ptr(workspace), workspace.numel(),
+                                     ctypes.c_void_p(st)), "mlra_decode_project")
+    return y
 
 
 def decode_static_scratch(q_lat, q_rope, c_kv, k_rope, seq_lens, page_table=None, *,

@@ -98,3 +98,57 @@ def test_multi_token_full_size_sampled():
                                w.num_branches, w.sigma, w.gamma, max_seq_len=inp.max_seq_len,
                                seqs=seqs, heads=heads)
         assert_close(out[seqs][:, t][:, heads], ref, f"token {t}")
+
+
+# Two tokens of 64 heads per CTA (the 128-row attention kernel): an even number of tokens, 64
+# heads and 128-wide branches read in place.
+@pytest.mark.parametrize("q,lens,page_size", [
+    (4, [4, 5, 129, 1000, 3], 0),       # a sequence of 3: its first token has length 0
+    (2, [1, 2, 64, 65, 128, 129, 777], 64),
+    (6, [6, 300, 2049], 0),
+])
+def test_two_tokens_per_cta_match_oracle(q, lens, page_size):
+    w, inp, q_lat, q_rope = multi_inputs(q, lens, B=4, page_size=page_size, seed=71)
+    out, lse = run_multi(w, inp, q_lat, q_rope)
+    torch.cuda.synchronize()
+    ref, ref_lse = oracle.decode_multi(q_lat, q_rope, inp.c_kv, inp.k_rope, inp.seq_lens,
+                                       inp.page_table, w.num_branches, w.sigma, w.gamma,
+                                       page_size=page_size, max_seq_len=inp.max_seq_len)
+    assert_close(out, ref, f"q={q}")
+    assert_lse_close(lse, ref_lse, f"q={q} lse")
+
+
+def test_two_tokens_per_cta_summed_and_replanned(monkeypatch):
+    """Summed output mode (every result goes through the combine kernel) and the attention
+    kernel's re-plan path, on the 128-row kernel."""
+    q, lens = 2, [2, 300, 129, 1000]
+    w, inp, q_lat, q_rope = multi_inputs(q, lens, B=4, seed=73)
+    monkeypatch.setenv("MLRA_TEST_FORCE_REPLAN", "1")
+    out, lse = run_multi(w, inp, q_lat, q_rope, out_mode="summed")
+    torch.cuda.synchronize()
+    monkeypatch.delenv("MLRA_TEST_FORCE_REPLAN")
+    ref, ref_lse = oracle.decode_multi(q_lat, q_rope, inp.c_kv, inp.k_rope, inp.seq_lens, None,
+                                       w.num_branches, w.sigma, w.gamma,
+                                       max_seq_len=inp.max_seq_len, out_mode="summed")
+    assert_close(out, ref, "summed")
+    assert_lse_close(lse, ref_lse, "summed lse")
+
+
+def test_two_tokens_per_cta_through_the_prep_kernel():
+    """80 sequences x 2 tokens = 80 units of two tokens: the prep kernel plans them."""
+    g = torch.Generator().manual_seed(93)
+    lens = (torch.randint(1, 300, (80,), generator=g)).tolist()
+    lens[5] = 0                                   # first token -1 (flagged), second 0
+    w, inp, q_lat, q_rope = multi_inputs(2, lens, B=4, seed=94)
+    pt = None
+    dims = mlra.dims_for(q_lat[:, 0].cuda(), q_rope[:, 0].cuda(), inp.c_kv.cuda(), inp.k_rope.cuda(),
+                         inp.seq_lens.cuda(), pt, w.num_branches, max_seq_len=inp.max_seq_len)
+    ws = torch.zeros(mlra.workspace_size_multi(dims, 2), dtype=torch.uint8, device="cuda")
+    out, lse = run_multi(w, inp, q_lat, q_rope, workspace=ws)
+    rc, flags = mlra.read_status(ws)
+    assert flags & mlra.FLAG_BAD_LENGTH
+    ref, ref_lse = oracle.decode_multi(q_lat, q_rope, inp.c_kv, inp.k_rope, inp.seq_lens, None,
+                                       w.num_branches, w.sigma, w.gamma, max_seq_len=inp.max_seq_len)
+    assert torch.count_nonzero(out[5]) == 0
+    assert_close(out, ref, "80 units")
+    assert_lse_close(lse, ref_lse, "80 units lse")

@@ -315,3 +315,21 @@ def test_head_groups(B, heads, page_size):
 ])
 def test_full_size_sampled(name, seqs, heads):
     _sampled(name, seqs, heads)
+
+
+@pytest.mark.parametrize("B,paged", [(4, False), (2, True)])
+def test_replan_path(B, paged, monkeypatch):
+    """The attention kernel plans its work range before its dependency wait and keeps that plan
+    when the lengths read after the wait are unchanged; otherwise it lets the loads it issued on
+    the stale plan land, resets its barriers and re-plans.  The environment variable
+    MLRA_TEST_FORCE_REPLAN makes every call take that second path: the result must still match
+    the oracle, and equal bit for bit the result of the normal path."""
+    inp = small_inputs(B=B, lens=[300, 1, 65, 0, 1000, 63], page_size=64 if paged else 0, seed=19)
+    base, base_lse = run_gpu(inp)
+    monkeypatch.setenv("MLRA_TEST_FORCE_REPLAN", "1")
+    out, lse = run_gpu(inp)
+    monkeypatch.delenv("MLRA_TEST_FORCE_REPLAN")
+    ref, ref_lse = run_oracle(inp)
+    assert_close(out, ref, f"re-plan B={B} paged={paged}")
+    assert_lse_close(lse, ref_lse, "re-plan lse")
+    assert torch.equal(out, base) and torch.equal(lse, base_lse)

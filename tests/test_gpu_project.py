@@ -84,3 +84,32 @@ def test_pack_wuv_layout():
         got = packed[box * 4096 + r * 64 + pos * 8: box * 4096 + r * 64 + pos * 8 + 8]
         want = wc[h, m * 64 + r, kb * 64 + 8 * j: kb * 64 + 8 * j + 8]
         assert torch.equal(got, want), (h, m, kb, r, j)
+
+
+@pytest.mark.parametrize("B,d_latent,lens,page_size,num_ranges", [
+    (4, 512, [300, 1, 65, 0, 1000, 63, 2049], 0, 0),    # splits, an empty sequence
+    (1, 512, [129, 700, 5], 64, 0),                    # MLA, paged
+    (2, 512, [3000, 17], 0, 9),                        # forced ranges: many parts
+    (4, 256, [40] * 70, 64, 0),                        # more than 64 sequences: prep kernel
+])
+def test_decode_project_matches_oracle(B, d_latent, lens, page_size, num_ranges):
+    """mlra_decode_project: the attention kernel, then step 3 merging the split sequences itself
+    (no combine kernel), against the oracle's decode followed by its step 3."""
+    inp = small_inputs(B=B, d_latent=d_latent, lens=lens, page_size=page_size, seed=23)
+    w = inp.workload
+    q, qr, c, kr, sl, pt = to_dev(inp)
+    g = torch.Generator().manual_seed(24)
+    w_uv = (torch.randn(w.heads, 128, d_latent, generator=g) / d_latent ** 0.5).to(torch.bfloat16)
+    dims = mlra.dims_for(q, qr, c, kr, sl, pt, B, max_seq_len=inp.max_seq_len,
+                         page_size=page_size, num_ranges=num_ranges)
+    ws = torch.full((mlra.workspace_size_project(dims),), 0xFF, dtype=torch.uint8, device="cuda")
+    y = mlra.decode_project(q, qr, c, kr, sl, pt, mlra.pack_wuv(w_uv.cuda()), num_branches=B,
+                            softmax_scale=w.sigma, branch_scale=w.gamma,
+                            max_seq_len=inp.max_seq_len, page_size=page_size,
+                            num_ranges=num_ranges, workspace=ws)
+    torch.cuda.synchronize()
+    rc, flags = mlra.read_status(ws)
+    assert rc == mlra.MLRA_OK, flags
+    o, _ = oracle.decode(inp.q_lat, inp.q_rope, inp.c_kv, inp.k_rope, inp.seq_lens, inp.page_table,
+                         B, w.sigma, w.gamma, max_seq_len=inp.max_seq_len, page_size=page_size)
+    assert_close(y, oracle.project(o, w_uv.float()), f"B={B} lens={len(lens)}")

@@ -315,12 +315,24 @@ def test_head_groups_in_the_plan():
 
 
 def test_workspace_size_multi_covers_the_virtual_sequences():
-    """q query tokens per sequence plan N * q virtual sequences: the workspace equals that of a
-    single-token call with N * q sequences (paged, so the cache geometry is the same)."""
+    """q query tokens per sequence plan N * q virtual sequences of H rows (odd q, or shapes the
+    two-token kernel does not take): the workspace equals that of a single-token call with N * q
+    sequences.  An even q with 64 heads and 128-wide branches plans N * q / 2 units of two tokens
+    (128 rows each): the workspace holds their partial results, R + N q / 2 - 1 slots of
+    128 rows x d_c fp32 plus (m, l) per branch."""
     kw = dict(heads=64, num_branches=4, d_latent=512, d_rope=64, max_seq_len=4096,
               cache_rows=64 * 1024, page_size=64, max_pages_per_seq=64, num_ranges=37)
     d = mlra.make_dims(batch=8, **kw)
-    for q in (1, 2, 4):
+    for q in (1, 3):
         assert mlra.workspace_size_multi(d, q) == mlra.workspace_size(mlra.make_dims(batch=8 * q, **kw))
+    kw2 = {**kw, "num_branches": 2}   # 256-wide branches: one token per CTA for any q
+    d2 = mlra.make_dims(batch=8, **kw2)
+    assert mlra.workspace_size_multi(d2, 2) == mlra.workspace_size(mlra.make_dims(batch=16, **kw2))
+    for q in (2, 4):
+        units = 8 * q // 2
+        slots = 37 + units - 1
+        need = slots * 128 * 512 * 4 + slots * 128 * 4 * 2 * 4
+        got = mlra.workspace_size_multi(d, q)
+        assert need <= got <= need + 64 * 1024
     with pytest.raises(mlra.MlraError):
         mlra.workspace_size_multi(d, 0)
