@@ -749,11 +749,21 @@ def run_stage(args):
                                          softmax_scale=w.sigma, branch_scale=w.gamma,
                                          max_seq_len=inp.max_seq_len, page_size=w.page_size,
                                          out=outm, workspace=ws)
+        # the single-token call timed the same way (events around every call), for the ratio
+        q1, qr1 = qm[:, :1].contiguous(), qrm[:, :1].contiguous()
+        ws1 = torch.empty(mlra.workspace_size_multi(dims, 1), dtype=torch.uint8, device=dev)
+        out1 = torch.empty(N, 1, H, d_c, dtype=torch.float32, device=dev)
+        body1 = lambda: mlra.decode_multi(q1, qr1, c, kr, lens, pt, num_branches=w.num_branches,  # noqa: E731
+                                          softmax_scale=w.sigma, branch_scale=w.gamma,
+                                          max_seq_len=inp.max_seq_len, page_size=w.page_size,
+                                          out=out1, workspace=ws1)
         for _ in range(args.warmup):
             body()
+            body1()
         big = cache_bytes(inp) > L2_BYTES
         with ClockSampler(0) as clk:
             ms = graph_time(body, args.steps, pre=None if big else evict)
+            ms1 = graph_time(body1, args.steps, pre=None if big else evict)
         once = cache_bytes(inp)  # the cache read once: what a fused multi-token kernel needs
         token_bytes = once // max(1, int(inp.seq_lens.sum()))
         read = sum(max(0, int(L) - (q - 1 - t)) for L in inp.seq_lens.tolist()
@@ -762,6 +772,10 @@ def run_stage(args):
         line = {"metric": f"multi-token decode ({q} query tokens per sequence) query tokens/s",
                 "value": N * q / (ms * 1e-3), "unit": "tokens/s", "higher_is_better": True,
                 "ms_per_step": ms, "q_len": q,
+                "ms_per_step_one_token": ms1, "ratio_to_one_token": ms / ms1,
+                "path": "two tokens per CTA (128 query rows)" if (q % 2 == 0 and H == 64 and
+                                                                 w.d_latent // w.num_branches == 128)
+                        else "one token per CTA",
                 "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
                              "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
                              "kernel": "mlra_decode_kernel (whole call)",

@@ -17,10 +17,11 @@
 // NS = 4 stages; its RoPE block (16 KB, read by the score product only) in a ring of its own of
 // NR = 2 slots, so that the 48 KB of queries leave room for four latent stages.
 //
-// TMEM (512 columns, all 128 lanes): O in columns [0, 128); two score buffers of 128 columns; two
-// P slots of 64 columns (bf16 pairs).  The softmax writes a tile's P into the P slot of the tile's
-// parity (after the output product of two tiles earlier has read it), freeing its score buffer
-// for the score product of two tiles later; the output product reads P from TMEM (A operand).
+// TMEM (512 columns, all 128 lanes): O in columns [0, 128); one score buffer of 128 columns; four
+// P slots of 64 columns (bf16 pairs), one per latent stage.  The softmax warps release the score
+// buffer as soon as they have loaded it (the next tile's score product may start), and write a
+// tile's P into its stage's P slot: the landed tile implies the output product that last read
+// the slot (four tiles earlier) completed.  The output product reads P from TMEM (A operand).
 //
 // Warps (352 threads): 0-7 softmax, 8 TMA producer, 9 score-MMA issuer and TMEM owner, 10
 // output-MMA issuer.  Softmax warp w reads TMEM lanes 32 (w % 4) .. + 31 (one row per thread) and
@@ -31,9 +32,10 @@
 // Ordering facts the parity waits rely on (a barrier at most one phase past the phase awaited):
 //   * latent tile s loads after the output product of tile s - NS completed; RoPE block s loads
 //     after the score product of tile s - NR completed;
-//   * the score of tile s is issued after the softmax released P of tile s - NSB (it has read
-//     score buffer s % NSB), so neither issuer runs more than NSB tiles ahead of the softmax;
-//   * the softmax writes P of tile s after the output product of tile s - NP completed (P slot).
+//   * the score of tile s is issued after the softmax loaded the scores of tile s - 1 (one score
+//     buffer), so the score issuer runs at most one tile ahead of the softmax;
+//   * the softmax writes P of tile s into slot s % NS: tile s landed after the output product of
+//     tile s - NS, the slot's last reader, completed.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -58,8 +60,8 @@ struct DecodeM128Cfg {
   static constexpr int NR = 2;                      // RoPE slots
   static constexpr int QBYTES = (NCB + 1) * QBOX;   // query blocks + RoPE-query block
   static constexpr int O_COLS = DBLK;
-  static constexpr int NSB = 2;                     // score buffers
-  static constexpr int NP = 2;                      // P slots
+  static constexpr int NSB = 1;                     // score buffers
+  static constexpr int NP = NS;                     // P slots, one per latent stage
   static constexpr int S_COL = O_COLS;              // first score buffer
   static constexpr int P_COL = S_COL + NSB * T;     // first P slot (T / 2 columns each)
   static constexpr int NPV = NS;
@@ -68,7 +70,7 @@ struct DecodeM128Cfg {
   static constexpr int OFF_STAGE = QBYTES;
   static constexpr int OFF_ROPE = OFF_STAGE + NS * STAGE;
   static constexpr int OFF_BAR = OFF_ROPE + NR * CBLK;
-  static constexpr int NBAR = 2 * NS + 2 * NR + 2 + NSB + TB * NP + NPV + 2 + 4;
+  static constexpr int NBAR = 2 * NS + 2 * NR + 2 + 2 * NSB + TB * NP + NPV + 2 + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_PLAN = OFF_MISC + 16;
   static constexpr int PLAN_BYTES = 16 * kSelfPlanMaxSeqs + 4 * kSelfPlanMaxSeqs + 16;
@@ -78,7 +80,7 @@ struct DecodeM128Cfg {
   static constexpr int SMEM = OFF_XCH + 3 * 2 * QR * 4;
   static constexpr int SMEM_ALLOC = SMEM + 1024;
   static_assert(P_COL + NP * (T / 2) <= TMEM_COLS, "TMEM budget");
-  static_assert(NSB == NP, "the score issuer waits for P of the tile NSB earlier");
+  static_assert(NSB == 1 && NP == NS, "one score buffer; a P slot per latent stage");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
@@ -106,7 +108,8 @@ mlra_decode_m128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
   const uint32_t bar_q_full = bar_rope_empty + 8 * C::NR;    //       TMA -> MMA
   const uint32_t bar_q_empty = bar_q_full + 8;               //       MMA (last score) -> TMA
   const uint32_t bar_s_full = bar_q_full + 16;               // [NSB] MMA (score) -> softmax
-  const uint32_t bar_p_full = bar_s_full + 8 * NSB;          // [TB][NP] softmax (P half) -> MMA
+  const uint32_t bar_s_free = bar_s_full + 8 * NSB;          // [NSB] softmax (scores loaded) -> MMA
+  const uint32_t bar_p_full = bar_s_free + 8 * NSB;          // [TB][NP] softmax (P half) -> MMA
   const uint32_t bar_pv_done = bar_p_full + 8 * C::TB * C::NP;  // [NPV] MMA (PV done) -> softmax
   const uint32_t bar_final_s = bar_pv_done + 8 * NPV;
   const uint32_t bar_final_pv = bar_final_s + 8;
@@ -137,7 +140,10 @@ mlra_decode_m128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     }
     mbar_init(bar_q_full, 1);
     mbar_init(bar_q_empty, 1);
-    for (int k = 0; k < NSB; ++k) mbar_init(bar_s_full + 8 * k, 1);
+    for (int k = 0; k < NSB; ++k) {
+      mbar_init(bar_s_full + 8 * k, 1);
+      mbar_init(bar_s_free + 8 * k, 256);
+    }
     for (int k = 0; k < C::TB * C::NP; ++k) mbar_init(bar_p_full + 8 * k, 128);
     for (int k = 0; k < NPV; ++k) mbar_init(bar_pv_done + 8 * k, 1);
     mbar_init(bar_final_s, 1);
@@ -349,8 +355,8 @@ mlra_decode_m128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         ok = wait_warp(bar_stage_full + 8 * (it % NS), (it / NS) & 1, tmo, abort_flag, flags);
         if (ok)
           ok = wait_warp(bar_rope_full + 8 * (it % C::NR), (it / C::NR) & 1, tmo, abort_flag, flags);
-        if (ok && it >= NSB)  // score buffer free: the softmax released P of tile it - NSB
-          ok = wait_warp(bar_p_full + 8 * ((it - NSB) % C::NP), ((it - NSB) / C::NP) & 1, tmo,
+        if (ok && it >= NSB)  // score buffer free: the softmax loaded the scores of tile it - 1
+          ok = wait_warp(bar_s_free + 8 * ((it - NSB) % NSB), ((it - NSB) / NSB) & 1, tmo,
                          abort_flag, flags);
         if (!ok) break;
         tc_fence_after();
@@ -448,6 +454,8 @@ mlra_decode_m128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         tmem_ld32(sbuf, reinterpret_cast<uint32_t(&)[32]>(v[0]));
         tmem_ld32(sbuf + 32, reinterpret_cast<uint32_t(&)[32]>(v[32]));
         tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar_s_free + 8 * (it % NSB));  // the score buffer may take the next tile
         const int valid = min(T, row_len - T * t) - 64 * hc;  // of this thread's 64 positions
         const int tile_valid = min(T, L - T * t);             // of the unit's longest row
         const float sc = p.scale_log2;
@@ -527,8 +535,7 @@ mlra_decode_m128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           }
           fence_proxy_async_smem();
         }
-        // P: positions 64 hc + k -> bf16 pairs in columns 32 hc + k / 2 of the tile's P slot,
-        // once the output product of tile it - NP has read the slot
+        // P: positions 64 hc + k -> bf16 pairs in columns 32 hc + k / 2 of the tile's P slot
         const float mul = whole ? sc : 1.f;
         const float neg_m = m_used == -CUDART_INF_F ? 0.f : -m_used;
         float sum4[4] = {0.f, 0.f, 0.f, 0.f};
@@ -539,12 +546,6 @@ mlra_decode_m128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           const float p1 = ex2_approx(fmaf(v[k + 1], mul, neg_m));
           sum4[(k >> 1) & 3] += p0 + p1;
           pk[k / 2] = pack_bf16x2(p0, p1);
-        }
-        if (it >= C::NP) {
-          ok = wait_warp(bar_pv_done + 8 * ((it - C::NP) % NPV), ((it - C::NP) / NPV) & 1, tmo,
-                         abort_flag, flags);
-          if (!ok) break;
-          tc_fence_after();
         }
         tmem_st32(tmem + lane_base + C::P_COL + (it % C::NP) * (T / 2) + 32 * hc, pk);
         tmem_wait_st();
