@@ -88,6 +88,7 @@ struct DecodeCfg {
 };
 
 constexpr uint32_t kFull = 0xffffffffu;
+constexpr int kFirstTiles = 2;  // tiles issued at once when a CTA starts (the rest after tile 0)
 
 // Warp-collective bounded wait on an mbarrier phase.  Every lane polls; on time-out the
 // status word gets kFlagTimeout, the CTA abort flag is raised and all lanes return false.
@@ -222,8 +223,12 @@ __device__ __forceinline__ int plan_segments(const DecodeParams& p, int range, i
     const uint32_t m = __ballot_sync(kFull, own0 || own1);
     return __shfl_sync(kFull, mine, m ? __ffs(m) - 1 : 0);
   };
-  const int g0 = tile_of(floor_div_i64(range * (int64_t)vtotal, R));
-  const int g1 = range + 1 < R ? tile_of(floor_div_i64((range + 1) * (int64_t)vtotal, R)) : total;
+  // both boundaries' virtual positions first (independent divisions), then their tiles
+  const bool has_next = range + 1 < R;
+  const int64_t vp0 = floor_div_i64(range * (int64_t)vtotal, R);
+  const int64_t vp1 = has_next ? floor_div_i64((range + 1) * (int64_t)vtotal, R) : 0;
+  const int g0 = tile_of(vp0);
+  const int g1 = has_next ? tile_of(vp1) : total;
   const bool ov0 = t0 > 0 && lo0 < g1 && hi0 > g0;
   const bool ov1 = t1 > 0 && lo1 < g1 && hi1 > g0;
   const uint32_t m0 = __ballot_sync(kFull, ov0), m1 = __ballot_sync(kFull, ov1);
@@ -357,7 +362,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     mbar_init(bar_final_s, 1);
     mbar_init(bar_final_pv, 1);
   };
-  if (threadIdx.x == 0) {
+  if (warp == 6 && lane == 0) {  // (warp 0 starts the plan meanwhile)
     init_barriers();
     *abort_flag = 0;
     *spec_flags = 0;
@@ -442,7 +447,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       // The first segment's queries and tiles go out at once, on the speculative plan (bad-page
       // bits into spec_flags until the plan is confirmed).
       const int len = first_seg.w & 0x7fffffff;
-      pre_tiles = first_seg.z < NS ? first_seg.z : NS;
+      pre_tiles = first_seg.z < kFirstTiles ? first_seg.z : kFirstTiles;
       pre_q = true;
       const int cache_seq = first_seg.x / p.q_per_seq;
       if (lane == 0) issue_queries(first_seg.x);
@@ -517,6 +522,13 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       const int cache_seq = seg.seq / p.q_per_seq;  // whose cache rows (once per segment)
       for (int i = 0; i < seg.ntiles; ++i, ++it) {
         if (nseg == 0 && i < pre_tiles) continue;  // issued before the plan was confirmed
+        if (it == kFirstTiles && pre_tiles == kFirstTiles) {
+          // the remaining first stages once tile 0 has landed: every CTA's first tile arrives
+          // sooner (fewer bytes ahead of it in the memory queues), so the tensor core starts and
+          // frees stages while the first loads are still streaming
+          ok = wait_warp(bar_stage_full, 0, tmo, abort_flag, flags);
+          if (!ok) break;
+        }
         int rows[C::TB];
         tile_rows(cache_seq, seg.tile0 + i, L, flags, rows);
         const int st = it % NS;
@@ -894,7 +906,9 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
       }
     }
-    if (lane == 0) bulk_wait_all();  // every bulk store of this warp is performed before exit
+    // the staged boxes must stay in shared memory until the bulk stores have read them; their
+    // global writes complete with the grid, before a dependent kernel's wait returns
+    if (lane == 0) bulk_wait_read_all();
     __syncwarp();
   }
 
