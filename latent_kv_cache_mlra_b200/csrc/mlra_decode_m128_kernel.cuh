@@ -24,10 +24,11 @@
 // the slot (four tiles earlier) completed.  The output product reads P from TMEM (A operand).
 //
 // Warps (352 threads): 0-7 softmax, 8 TMA producer, 9 score-MMA issuer and TMEM owner, 10
-// output-MMA issuer.  Softmax warp w reads TMEM lanes 32 (w % 4) .. + 31 (one row per thread) and
-// positions 64 (w / 4) .. + 63 of every tile; the two warps of a row exchange their row maxima
-// through shared memory (an mbarrier of 64 arrivals per pair, waited on with a time limit) and
-// release P in two halves.
+// output-MMA issuer.  Softmax warp w reads the 16 TMEM lanes 32 (w % 4) + 16 (w / 4) .. + 15 (one
+// row each) in the 16-lane load shape: lanes l and l + 16 of the warp share row l % 16, lane l
+// taking the positions 64 k + 32 (l / 16) .. + 31 (k = 0, 1) of every tile, so a row's maximum and
+// sum need one shuffle.  P is released in two halves (positions 64 k ..), each once all 256
+// softmax threads wrote it.
 //
 // Ordering facts the parity waits rely on (a barrier at most one phase past the phase awaited):
 //   * latent tile s loads after the output product of tile s - NS completed; RoPE block s loads
@@ -70,14 +71,11 @@ struct DecodeM128Cfg {
   static constexpr int OFF_STAGE = QBYTES;
   static constexpr int OFF_ROPE = OFF_STAGE + NS * STAGE;
   static constexpr int OFF_BAR = OFF_ROPE + NR * CBLK;
-  static constexpr int NBAR = 2 * NS + 2 * NR + 2 + 2 * NSB + TB * NP + NPV + 2 + 4;
+  static constexpr int NBAR = 2 * NS + 2 * NR + 2 + 2 * NSB + TB * NP + NPV + 2;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_PLAN = OFF_MISC + 16;
   static constexpr int PLAN_BYTES = 16 * kSelfPlanMaxSeqs + 4 * kSelfPlanMaxSeqs + 16;
-  // row exchange between the two warps of a row: [3][2 halves][128 rows] floats (maxima of even
-  // and odd tiles, sums at the segment end)
-  static constexpr int OFF_XCH = (OFF_PLAN + PLAN_BYTES + 15) / 16 * 16;
-  static constexpr int SMEM = OFF_XCH + 3 * 2 * QR * 4;
+  static constexpr int SMEM = OFF_PLAN + PLAN_BYTES;
   static constexpr int SMEM_ALLOC = SMEM + 1024;
   static_assert(P_COL + NP * (T / 2) <= TMEM_COLS, "TMEM budget");
   static_assert(NSB == 1 && NP == NS, "one score buffer; a P slot per latent stage");
@@ -113,7 +111,6 @@ mlra_decode_m128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
   const uint32_t bar_pv_done = bar_p_full + 8 * C::TB * C::NP;  // [NPV] MMA (PV done) -> softmax
   const uint32_t bar_final_s = bar_pv_done + 8 * NPV;
   const uint32_t bar_final_pv = bar_final_s + 8;
-  const uint32_t bar_pair = bar_final_pv + 8;                 // [4] the two softmax warps of a row
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   uint32_t* spec_flags = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC + 8);
@@ -121,7 +118,6 @@ mlra_decode_m128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
   uint8_t* plan = smem + C::OFF_PLAN;
   volatile int32_t* plan_count = reinterpret_cast<volatile int32_t*>(plan + 20 * kSelfPlanMaxSeqs);
   volatile int32_t* plan_stale = plan_count + 1;
-  float* xch = reinterpret_cast<float*>(smem + C::OFF_XCH);  // [3][half][row]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int range = blockIdx.x / p.n_groups;
@@ -144,11 +140,10 @@ mlra_decode_m128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       mbar_init(bar_s_full + 8 * k, 1);
       mbar_init(bar_s_free + 8 * k, 256);
     }
-    for (int k = 0; k < C::TB * C::NP; ++k) mbar_init(bar_p_full + 8 * k, 128);
+    for (int k = 0; k < C::TB * C::NP; ++k) mbar_init(bar_p_full + 8 * k, 256);
     for (int k = 0; k < NPV; ++k) mbar_init(bar_pv_done + 8 * k, 1);
     mbar_init(bar_final_s, 1);
     mbar_init(bar_final_pv, 1);
-    for (int k = 0; k < 4; ++k) mbar_init(bar_pair + 8 * k, 64);
   };
   if (threadIdx.x == 0) {
     init_barriers();
@@ -430,11 +425,10 @@ mlra_decode_m128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     wait_warp(bar_final_pv, 0, tmo, abort_flag, flags, false);
   } else {
     // ------------------------------------------------------------------ softmax warps 0-7
-    const int sp = warp & 3, hc = warp >> 2;  // TMEM sub-partition (rows), half of the positions
-    const int row = 32 * sp + lane;           // query row: token row / 64 of the unit, head row % 64
-    const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
-    const uint32_t pair_bar = bar_pair + 8 * sp;  // the warps sp and sp + 4
-    int xphase = 0;                               // phases of pair_bar passed
+    const int q = lane >> 4;                               // which 32 of every 64 positions
+    const int row = 32 * (warp & 3) + 16 * (warp >> 2) + (lane & 15);  // query row (TMEM lane)
+    // token row / 64 of the unit, head row % 64
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3) + 16 * (warp >> 2)) << 16;
     SegCursor walk(seg_list, list_global, seg_count);
     Segment seg;
     int L = 0;
@@ -449,17 +443,18 @@ mlra_decode_m128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         ok = wait_warp(bar_s_full + 8 * (it % NSB), (it / NSB) & 1, tmo, abort_flag, flags);
         if (!ok) break;
         tc_fence_after();
+        // v[32 k + j] = score of position 64 k + 32 q + j
         float v[64];
-        const uint32_t sbuf = tmem + lane_base + C::S_COL + (it % NSB) * T + 64 * hc;
-        tmem_ld32(sbuf, reinterpret_cast<uint32_t(&)[32]>(v[0]));
-        tmem_ld32(sbuf + 32, reinterpret_cast<uint32_t(&)[32]>(v[32]));
+        const uint32_t sbuf = tmem + lane_base + C::S_COL + (it % NSB) * T;
+        tmem_ld16x2_32(sbuf, reinterpret_cast<uint32_t(&)[32]>(v[0]));
+        tmem_ld16x2_32(sbuf + 64, reinterpret_cast<uint32_t(&)[32]>(v[32]));
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(bar_s_free + 8 * (it % NSB));  // the score buffer may take the next tile
-        const int valid = min(T, row_len - T * t) - 64 * hc;  // of this thread's 64 positions
-        const int tile_valid = min(T, L - T * t);             // of the unit's longest row
+        const int rvalid = min(T, row_len - T * t);  // positions of this row in the tile
+        const int tile_valid = min(T, L - T * t);    // of the unit's longest row
         const float sc = p.scale_log2;
-        const bool whole = valid >= 64;
+        const bool whole = rvalid >= T;
         float mx;
         if (whole) {
           float a[4] = {v[0], v[1], v[2], v[3]};
@@ -476,20 +471,12 @@ mlra_decode_m128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           mx = -CUDART_INF_F;
 #pragma unroll
           for (int k = 0; k < 64; ++k) {
-            const float x = k < valid ? v[k] * sc : -CUDART_INF_F;
+            const float x = 64 * (k >> 5) + 32 * q + (k & 31) < rvalid ? v[k] * sc : -CUDART_INF_F;
             v[k] = x;
             mx = fmaxf(mx, x);
           }
         }
-        // the row's maximum over both halves of the tile
-        // (by tile parity: the partner reads tile it's value before it reaches tile it + 1's
-        // barrier, so tile it + 2 may write the slot again)
-        float* xm = xch + (it & 1) * 256;
-        xm[hc * 128 + row] = mx;
-        mbar_arrive(pair_bar);
-        ok = wait_warp(pair_bar, (xphase++) & 1, tmo, abort_flag, flags);
-        if (!ok) break;
-        mx = fmaxf(mx, xm[(1 - hc) * 128 + row]);
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));  // the row's maximum over the tile
         bool rescale = false;
         float alpha = 1.f;
         if (mx == -CUDART_INF_F) {
@@ -504,54 +491,59 @@ mlra_decode_m128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         }
         l_sum *= (i == 0 ? 1.f : alpha);
         if (__any_sync(kFull, rescale)) {
-          // O holds the output products up to tile it-1: wait for them, then scale this warp's
-          // half of O's columns
+          // O holds the output products up to tile it-1: wait for them, then scale this thread's
+          // 64 columns of its row
           ok = wait_warp(bar_pv_done + 8 * ((it - 1) % NPV), ((it - 1) / NPV) & 1, tmo, abort_flag,
                          flags);
           if (!ok) break;
           tc_fence_after();
           const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
-          for (int c0 = 64 * hc; c0 < 64 * hc + 64; c0 += 32) {
+          for (int c0 = 0; c0 < C::DBLK; c0 += 64) {
             uint32_t r[32];
-            tmem_ld32(tmem + lane_base + c0, r);
+            tmem_ld16x2_32(tmem + lane_base + c0, r);
             tmem_wait_ld();
 #pragma unroll
             for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * f);
-            tmem_st32(tmem + lane_base + c0, r);
+            tmem_st16x2_32(tmem + lane_base + c0, r);
           }
           tmem_wait_st();
         }
-        // Ragged last tile: this half zeroes its latent rows past the unit's end before its P is
-        // released (a zero probability must never meet a non-finite value left in the cache).
+        // Ragged last tile: the latent rows past the unit's end are zeroed before P is released
+        // (a zero probability must never meet a non-finite value left in the cache).
         uint8_t* stage_ptr = smem + C::OFF_STAGE + (it % NS) * C::STAGE;
         if (tile_valid < T) {
-          const int tid = threadIdx.x & 127;  // 128 threads of this half
-          for (int k = tid; k < C::NCB * 64 * 8; k += 128) {
-            const int r = 64 * hc + (k >> 3) % 64;
+          const int tid = threadIdx.x;  // the 256 softmax threads
+          for (int k = tid; k < C::NCB * T * 8; k += 256) {
+            const int r = (k >> 3) % T;
             if (r >= tile_valid)
-              *reinterpret_cast<uint4*>(stage_ptr + (k / (64 * 8)) * C::CBLK + r * 128 + (k & 7) * 16) =
+              *reinterpret_cast<uint4*>(stage_ptr + (k / (T * 8)) * C::CBLK + r * 128 + (k & 7) * 16) =
                   make_uint4(0u, 0u, 0u, 0u);
           }
           fence_proxy_async_smem();
         }
-        // P: positions 64 hc + k -> bf16 pairs in columns 32 hc + k / 2 of the tile's P slot
+        // P: positions 64 k + 32 q + j -> bf16 pairs in columns 32 k + 16 q + j / 2 of the tile's
+        // P slot, released half k by half k
         const float mul = whole ? sc : 1.f;
         const float neg_m = m_used == -CUDART_INF_F ? 0.f : -m_used;
         float sum4[4] = {0.f, 0.f, 0.f, 0.f};
-        uint32_t pk[32];
+        const uint32_t pslot = tmem + lane_base + C::P_COL + (it % C::NP) * (T / 2);
 #pragma unroll
-        for (int k = 0; k < 64; k += 2) {
-          const float p0 = ex2_approx(fmaf(v[k], mul, neg_m));
-          const float p1 = ex2_approx(fmaf(v[k + 1], mul, neg_m));
-          sum4[(k >> 1) & 3] += p0 + p1;
-          pk[k / 2] = pack_bf16x2(p0, p1);
+        for (int kb = 0; kb < 2; ++kb) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int k = 0; k < 32; k += 2) {
+            const float p0 = ex2_approx(fmaf(v[32 * kb + k], mul, neg_m));
+            const float p1 = ex2_approx(fmaf(v[32 * kb + k + 1], mul, neg_m));
+            sum4[(k >> 1) & 3] += p0 + p1;
+            pk[k / 2] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16x2_16(pslot + 32 * kb, pk);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar_p_full + 8 * (kb * C::NP + it % C::NP));
         }
-        tmem_st32(tmem + lane_base + C::P_COL + (it % C::NP) * (T / 2) + 32 * hc, pk);
-        tmem_wait_st();
         l_sum += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-        tc_fence_before();
-        mbar_arrive(bar_p_full + 8 * (hc * C::NP + it % C::NP));
       }
       if (!ok) break;
       // ------------------------------------------------ epilogue of the segment
@@ -559,12 +551,7 @@ mlra_decode_m128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
                      flags);
       if (!ok) break;
       tc_fence_after();
-      float* xl = xch + 2 * 256;  // rewritten only after the partner passed another barrier
-      xl[hc * 128 + row] = l_sum;
-      mbar_arrive(pair_bar);
-      ok = wait_warp(pair_bar, (xphase++) & 1, tmo, abort_flag, flags);
-      if (!ok) break;
-      const float l_row = l_sum + xl[(1 - hc) * 128 + row];
+      const float l_row = l_sum + __shfl_xor_sync(kFull, l_sum, 16);
       const bool to_final = seg.whole && p.write_final;
       const float scale = to_final ? (l_row > 0.f ? p.gamma / l_row : 0.f) : 1.f;
       float* dst;
@@ -573,19 +560,20 @@ mlra_decode_m128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       else
         dst = p.part_o + (((int64_t)range + seg.seq) * C::QR + row) * p.dck + (int64_t)branch * C::DBLK;
 #pragma unroll 1
-      for (int c0 = 64 * hc; c0 < 64 * hc + 64; c0 += 32) {
+      for (int c0 = 0; c0 < C::DBLK; c0 += 64) {
         uint32_t r[32];
-        tmem_ld32(tmem + lane_base + c0, r);
+        tmem_ld16x2_32(tmem + lane_base + c0, r);
         tmem_wait_ld();
-        if (!to_final || c0 + 32 <= p.d_blk_out) {
+        const int col = c0 + 32 * q;  // this thread's 32 columns
+        if (!to_final || col + 32 <= p.d_blk_out) {
 #pragma unroll
           for (int k = 0; k < 32; k += 4)
-            *reinterpret_cast<float4*>(dst + c0 + k) =
+            *reinterpret_cast<float4*>(dst + col + k) =
                 make_float4(__uint_as_float(r[k]) * scale, __uint_as_float(r[k + 1]) * scale,
                             __uint_as_float(r[k + 2]) * scale, __uint_as_float(r[k + 3]) * scale);
         }
       }
-      if (hc == 0) {
+      if (q == 0) {
         if (to_final) {
           if (p.lse)
             p.lse[((int64_t)seg.seq * C::QR + row) * p.B + branch] =
