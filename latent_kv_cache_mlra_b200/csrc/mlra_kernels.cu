@@ -400,11 +400,13 @@ cudaError_t launch_pack(const void* w, void* packed, int H, int d_in, int d_out,
 
 cudaError_t launch_project(const ProjectParams& p, cudaStream_t st) {
   const int smem = project_smem_bytes(p.d_in / 64);
-  cudaError_t e = cudaFuncSetAttribute(mlra_project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  auto kern = p.merge ? mlra_project_kernel<kProjMergeThreads, true>
+                      : mlra_project_kernel<kProjThreads, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.H * (p.d_out / kProjM), (p.N + kProjN - 1) / kProjN);
-  cfg.blockDim = dim3(kProjThreads);
+  cfg.blockDim = dim3(p.merge ? kProjMergeThreads : kProjThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -412,7 +414,7 @@ cudaError_t launch_project(const ProjectParams& p, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, mlra_project_kernel, p);
+  return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 // ----------------------------------------------------------------------------- K7

@@ -36,7 +36,9 @@
 
 namespace mlra {
 
-constexpr int kProjThreads = 256;  // warps 0-3 also read the accumulator
+// Threads per CTA: 128 for the plain products (warps 0-3 read the accumulator), 256 when the
+// staging also merges split sequences (more loads in flight; warps 0-3 still read the accumulator).
+constexpr int kProjThreads = 128, kProjMergeThreads = 256;
 constexpr int kProjM = 64;     // rows of A_h per CTA
 constexpr int kProjN = 64;     // sequences per CTA
 constexpr int kProjBox = 8192; // one [64 x 64] bf16 box
@@ -91,7 +93,8 @@ __device__ __forceinline__ bool project_wait(uint32_t bar, uint32_t parity, uint
   return true;
 }
 
-__global__ void __launch_bounds__(kProjThreads, 1)
+template <int kThreads, bool kMerge>
+__global__ void __launch_bounds__(kThreads, 1)
 mlra_project_kernel(const __grid_constant__ ProjectParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -144,23 +147,23 @@ mlra_project_kernel(const __grid_constant__ ProjectParams p) {
   // (rows past the batch as zeros); the loads of 8 chunks are issued before any is converted.
   constexpr int kU = 8;
   const int chunks = npad * KB * 8;
-  if (p.merge && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 32) {
+  if (kMerge && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 32) {
     // the call's status word: the bits every attention CTA (and the prep kernel) raised
     uint32_t f = 0;
     for (int i = threadIdx.x; i < p.n_flag_slots; i += 32) f |= __ldcg(p.cta_flags + i);
     f = __reduce_or_sync(0xffffffffu, f);
     if (threadIdx.x == 0) *p.status = f;  // (a time-out of this kernel is ORed in after it)
   }
-  if (p.merge) {
+  if constexpr (kMerge) {
     // 8 columns (one branch) of row r per chunk: the attention kernel's final row, or the merge
     // of the sequence's parts.  Each thread takes two chunks at a time and keeps the loads of
     // both chunks' next kMergeBatch parts in flight (one memory round trip covers them).
     constexpr int kMergeBatch = 4;
-    for (int base = threadIdx.x; base < chunks; base += 2 * kProjThreads) {
+    for (int base = threadIdx.x; base < chunks; base += 2 * kThreads) {
       int np[2], r0[2], s_[2];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        const int idx = base + c * kProjThreads;
+        const int idx = base + c * kThreads;
         const int r = idx / (KB * 8);
         np[c] = 0;
         r0[c] = 0;
@@ -178,7 +181,7 @@ mlra_project_kernel(const __grid_constant__ ProjectParams p) {
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         a[c] = b4[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-        const int idx = base + c * kProjThreads;
+        const int idx = base + c * kThreads;
         const int cidx = idx % (KB * 8);
         if (np[c] == 0 || np[c] == 1) {
           const float4* src = reinterpret_cast<const float4*>(p.x + ((int64_t)s_[c] * p.H + h) * p.d_in + cidx * 8);
@@ -192,7 +195,7 @@ mlra_project_kernel(const __grid_constant__ ProjectParams p) {
         float4 va[2][kMergeBatch], vb[2][kMergeBatch];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          const int col = ((base + c * kProjThreads) % (KB * 8)) * 8;
+          const int col = ((base + c * kThreads) % (KB * 8)) * 8;
           const int br = col / p.dblk;
 #pragma unroll
           for (int u = 0; u < kMergeBatch; ++u) {
@@ -216,7 +219,7 @@ mlra_project_kernel(const __grid_constant__ ProjectParams p) {
       }
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        const int idx = base + c * kProjThreads;
+        const int idx = base + c * kThreads;
         if (idx >= chunks) continue;
         const int r = idx / (KB * 8), cidx = idx - r * (KB * 8);
         const int kb = cidx >> 3, j = cidx & 7;
@@ -231,11 +234,11 @@ mlra_project_kernel(const __grid_constant__ ProjectParams p) {
       }
     }
   }
-  for (int base = p.merge ? chunks : threadIdx.x; base < chunks; base += kProjThreads * kU) {
+  for (int base = kMerge ? chunks : threadIdx.x; base < chunks; base += kThreads * kU) {
     float4 va[kU], vb[kU];
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
-      const int idx = base + u * kProjThreads;
+      const int idx = base + u * kThreads;
       const int r = idx / (KB * 8), cidx = idx - r * (KB * 8);
       va[u] = vb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (idx < chunks && r < rows_n) {
@@ -247,7 +250,7 @@ mlra_project_kernel(const __grid_constant__ ProjectParams p) {
     }
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
-      const int idx = base + u * kProjThreads;
+      const int idx = base + u * kThreads;
       if (idx >= chunks) break;
       const int r = idx / (KB * 8), cidx = idx - r * (KB * 8);
       const int kb = cidx >> 3, j = cidx & 7;
@@ -302,7 +305,7 @@ mlra_project_kernel(const __grid_constant__ ProjectParams p) {
     __syncthreads();
     if (p.out_bf16) {
       // 8 rows (16 bytes) per store
-      for (int it = threadIdx.x; it < rows_n * (kProjM / 8); it += kProjThreads) {
+      for (int it = threadIdx.x; it < rows_n * (kProjM / 8); it += kThreads) {
         const int col = it / (kProjM / 8), c8 = it % (kProjM / 8);
         const float4 a = *reinterpret_cast<const float4*>(sT + col * kProjM + 8 * c8);
         const float4 b = *reinterpret_cast<const float4*>(sT + col * kProjM + 8 * c8 + 4);
@@ -313,7 +316,7 @@ mlra_project_kernel(const __grid_constant__ ProjectParams p) {
       }
     } else {
       // 4 rows (16 bytes) per store
-      for (int it = threadIdx.x; it < rows_n * (kProjM / 4); it += kProjThreads) {
+      for (int it = threadIdx.x; it < rows_n * (kProjM / 4); it += kThreads) {
         const int col = it / (kProjM / 4), c4 = it % (kProjM / 4);
         const int64_t at = ((int64_t)(n0 + col) * p.H + h) * p.d_out + m0 + 4 * c4;
         *reinterpret_cast<float4*>(static_cast<float*>(p.y) + at) =
