@@ -16,14 +16,19 @@
 //
 // TMEM.  An M = 64 accumulator occupies 16 of the 32 lanes of each sub-partition (rows 16k..16k+15
 // in lanes 32k + [0,16) + 16h for lane half h).  The score buffers (one per stage, T columns
-// each) fill lane half 0; O, cut into chunks of up to 128 columns, sits in lane half 1.
+// each) fill lane half 0; O, cut into chunks of up to 128 columns, sits in lane half 1, followed
+// there by one P slot per stage (T / 2 columns of bf16 pairs): the output product reads P from
+// TMEM as its A operand (which must share the accumulator's lanes).  The landed tile implies the
+// output product of the tile NS earlier, the slot's last reader, completed.  P is released in
+// 64-position halves: the output product of the first half starts while the softmax still
+// computes the second.  Keeping P out of shared memory leaves the tensor core's operand reads
+// and the TMA writes the shared-memory bandwidth (both products were slowed by it).  Where O
+// leaves no room (512-wide branches), P goes into shared memory over the tile's RoPE block,
+// which only the score product reads ([64 heads x T positions], K-major, the 128-byte swizzled
+// image of an MMA operand).
 //
 // Shared memory: the branch's queries (per segment), an NS-deep ring of cache tiles
-// [latent blocks | RoPE block].  The RoPE block is read only by the score product, so the bf16
-// probabilities P of the tile overwrite it ([64 heads x T positions], K-major, the 128-byte
-// swizzled image of an MMA operand) and the output product reads them from there as its A
-// operand.  P is released in 64-position halves: the output product of the first half starts
-// while the softmax still computes the second.
+// [latent blocks | RoPE block].
 //
 // Warp roles (224 threads): warps 0-3 softmax / rescale / epilogue, warp 4 TMA producer,
 // warp 5 score-MMA issuer and TMEM owner, warp 6 output-MMA issuer.  The two issuers feed the
@@ -56,14 +61,18 @@ struct DecodeCfg {
   static constexpr int TB = T / 64;                 // 64-row sub-boxes per tile
   static constexpr int BOX = 64 * 64 * 2;           // one [64 x 64] bf16 box, 8 KB
   static constexpr int CBLK = T * 128;              // one 64-column block of a tile (T rows)
-  static constexpr int STAGE = (NCB + 1) * CBLK;    // latent blocks + RoPE block (later P)
+  static constexpr int STAGE = (NCB + 1) * CBLK;    // latent blocks + RoPE block
   static constexpr int QBYTES = (NCB + 1) * BOX;    // query blocks + RoPE-query block
   static constexpr int OCW = DBLK < 128 ? DBLK : 128;   // O chunk width (columns)
   static constexpr int OCH = DBLK / OCW;                // O chunks
   static constexpr int O_COLS = OCH * OCW;              // TMEM columns of O (lane half 1)
   static constexpr int NSB = NS;                        // score buffers (lane half 0)
   static constexpr int NPV = NS;                    // ring of output-MMA completion barriers
-  static constexpr int TMEM_USED = O_COLS > NSB * T ? O_COLS : NSB * T;
+  // P slots in lane half 1 after O (one per stage), when they fit
+  static constexpr bool P_TMEM = O_COLS + NS * (T / 2) <= 512;
+  static constexpr int P_COL = O_COLS;
+  static constexpr int HALF1 = O_COLS + (P_TMEM ? NS * (T / 2) : 0);
+  static constexpr int TMEM_USED = HALF1 > NSB * T ? HALF1 : NSB * T;
   static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 :
                                    TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
   static constexpr int OFF_Q = 0;
@@ -603,7 +612,8 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     while (ok && walk.next(seg, L)) {
       for (int i = 0; ok && i < seg.ntiles; ++i, ++j) {
         const uint32_t stg = sStage + (j % NS) * C::STAGE;
-        const uint32_t pa = stg + C::NCB * C::CBLK;  // P over the tile's RoPE block
+        const uint32_t pa = stg + C::NCB * C::CBLK;  // P over the tile's RoPE block (!P_TMEM)
+        const uint32_t pt = tmem + (16u << 16) + C::P_COL + (j % NS) * (T / 2);  // P slot (P_TMEM)
 #pragma unroll 1
         for (int hb = 0; hb < C::TB; ++hb) {  // one 64-position half of P at a time
           ok = wait_warp(bar_p_full + 8 * (hb * NSB + j % NSB), (j / NSB) & 1, tmo, abort_flag,
@@ -618,9 +628,13 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
               const uint32_t b0 = stg + ch * (C::OCW / 64) * C::CBLK;
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t ad = sw128_desc(pa + hb * C::BOX + kk * 32, 16, 1024);
                 const uint64_t bd = sw128_desc(b0 + (4 * hb + kk) * 2048, C::CBLK, 1024);
-                umma_bf16(d, ad, bd, kIdPV, (kk > 0 || !first) ? 1u : 0u);
+                if constexpr (C::P_TMEM) {  // 16 positions: 8 TMEM columns of P
+                  umma_bf16_ts(d, pt + 8 * (4 * hb + kk), bd, kIdPV, (kk > 0 || !first) ? 1u : 0u);
+                } else {
+                  const uint64_t ad = sw128_desc(pa + hb * C::BOX + kk * 32, 16, 1024);
+                  umma_bf16(d, ad, bd, kIdPV, (kk > 0 || !first) ? 1u : 0u);
+                }
               }
             }
             if (hb == C::TB - 1) {
@@ -744,15 +758,18 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                   make_uint4(0u, 0u, 0u, 0u);
           }
         }
-        // probabilities -> bf16 P over the tile's RoPE block, the K-major image of the output
-        // product's A operand: head row r, position 64 l + 32 q + k in 64-position block l, row r,
-        // 16-byte chunk (4 q + k / 8) ^ (r & 7) (128-byte swizzle).  Each block is released to the
-        // output product as soon as it is written.
+        // probabilities -> bf16 P, each 64-position block l released to the output product as
+        // soon as it is written: into the tile's P slot in TMEM (position 64 l + 32 q + k in
+        // column 32 l + 16 q + k / 2 of the head row's lane), or over the tile's RoPE block, the
+        // K-major image of the output product's A operand (head row r, position 64 l + 32 q + k in
+        // 64-position block l, row r, 16-byte chunk (4 q + k / 8) ^ (r & 7), 128-byte swizzle).
         // p = 2^(score - m): whole tiles hold the raw products (one FFMA applies the scale),
         // the ragged tile the scaled and masked scores
         const float mul = whole_tile ? sc : 1.f, neg_m = -m_used;
         const int prow = 16 * warp + (lane & 15);
         uint8_t* p_base = stage_ptr + C::NCB * C::CBLK + prow * 128;
+        const uint32_t p_slot =
+            tmem + ((uint32_t)(32 * warp + 16) << 16) + C::P_COL + (it % NS) * (T / 2);
         float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int l = 0; l < C::TB; ++l) {
@@ -764,12 +781,17 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             sum4[(k >> 1) & 3] += p0 + p1;
             pk[k / 2] = pack_bf16x2(p0, p1);
           }
+          if constexpr (C::P_TMEM) {
+            tmem_st16x2_16(p_slot + 32 * l, pk);
+            tmem_wait_st();
+          } else {
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint4*>(p_base + l * C::BOX + (((4 * q + c) ^ (prow & 7)) << 4)) =
-                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            for (int c = 0; c < 4; ++c)
+              *reinterpret_cast<uint4*>(p_base + l * C::BOX + (((4 * q + c) ^ (prow & 7)) << 4)) =
+                  make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          }
           fence_proxy_async_smem();  // P (and the zeroed rows) are read by the MMA (async proxy)
-          tc_fence_before();         // ... after this thread's TMEM loads (and O rescale)
+          tc_fence_before();         // ... after this thread's TMEM accesses (and O rescale)
           mbar_arrive(bar_p_full + 8 * (l * NSB + it % NSB));
         }
         float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
