@@ -102,10 +102,13 @@ mlra_status make_plan(const mlra_dims* d, bool paged, int sms, Plan* pl, int q_l
   pl->dblk_k = dk;
   pl->variant = dk == 64 ? kV64 : dk == 128 ? kV128 : dk == 256 ? kV256 : kV512;
   pl->tile = variant_tile(pl->variant);
-  // An even number of query tokens of 64 heads with 128-wide branches read in place: two tokens
-  // per CTA (K1M), 128 query rows against each cache tile
-  pl->m128 = q_len >= 2 && q_len % 2 == 0 && d->heads == 64 && dk == 128 && !pl->repack;
-  pl->unit_tokens = pl->m128 ? 2 : 1;
+  // 128 query rows against each cache tile (K1M), for 128-wide branches read in place: an even
+  // number of query tokens of 64 heads (two tokens per CTA), or one token of 128 heads (both head
+  // groups in one CTA instead of two CTAs reading the same tiles)
+  const bool m128_tokens = q_len >= 2 && q_len % 2 == 0 && d->heads == 64 && dk == 128 && !pl->repack;
+  const bool m128_heads = q_len == 1 && d->heads == 128 && dk == 128 && !pl->repack;
+  pl->m128 = m128_tokens || m128_heads;
+  pl->unit_tokens = m128_tokens ? 2 : 1;
   pl->units = Nv / pl->unit_tokens;
   pl->rows = pl->m128 ? 128 : d->heads;
   pl->n_groups = pl->m128 ? B : B * ((d->heads + 63) / 64);  // CTAs per range

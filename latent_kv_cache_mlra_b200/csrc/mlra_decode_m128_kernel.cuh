@@ -3,13 +3,13 @@
 // The same computation as K1 (mlra_decode_kernel.cuh: step 2 of the absorbed decode, section 1.3
 // of the "Multi-Head Low-Rank Attention" page, in the branch form of section 3.1), for calls that
 // carry 128 query rows against the same cache rows: two consecutive query tokens of one sequence
-// with 64 heads each (several new tokens per sequence, causal among them).  Every tcgen05 product
-// then has M = 128 rows, the tensor core's full rate, and each cache tile is read once for both
-// tokens:
+// with 64 heads each (several new tokens per sequence, causal among them), or one token of 128
+// heads (rows = heads, unit_tokens = 1).  Every tcgen05 product then has M = 128 rows, the tensor
+// core's full rate, and each cache tile is read once for all 128 rows:
 //   score:  S[128 x 128]  = Q[128 x d] . C_b^T  +  Q^R[128 x 64] . K^R^T     (TMEM, fp32)
 //   output: O[128 x d]   += P[128 x 128] . C_b[128 x d]                     (TMEM, fp32)
-// Rows 0..63 are the unit's first token (heads 0..63), rows 64..127 its second; the first token
-// sits one position earlier, so its row attends one position fewer.
+// For two tokens, rows 0..63 are the unit's first token (heads 0..63), rows 64..127 its second;
+// the first token sits one position earlier, so its row attends one position fewer.
 //
 // One persistent CTA per (work range, branch); a work range covers units (pairs of tokens of a
 // sequence) exactly as K1's ranges cover sequences (mlra_plan.cuh).  Branch width 128, tiles of

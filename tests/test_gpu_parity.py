@@ -295,7 +295,8 @@ def _sampled(name, seqs, heads, R=0):
     return out
 
 
-@pytest.mark.parametrize("B,heads,page_size", [(1, 128, 0), (4, 128, 0), (2, 96, 64), (1, 72, 0)])
+@pytest.mark.parametrize("B,heads,page_size", [(1, 128, 0), (4, 128, 0), (4, 128, 64), (2, 96, 64),
+                                               (1, 72, 0)])
 def test_head_groups(B, heads, page_size):
     """More than 64 heads: one CTA per (range, branch, 64-head group); a partial last group."""
     inp = small_inputs(B=B, heads=heads, lens=[300, 1, 129, 700], page_size=page_size, seed=71)
@@ -305,8 +306,27 @@ def test_head_groups(B, heads, page_size):
     assert_lse_close(lse, ref_lse, f"B={B} H={heads}")
 
 
+def test_128_heads_in_one_cta():
+    """128 heads with 128-wide branches read in place: one CTA per (range, branch) carries both
+    head groups as 128-row products (the plan counts B CTAs per range, not 2 B); against the
+    oracle with ragged lengths, forced ranges, summed output and a replanned call."""
+    inp = small_inputs(B=4, heads=128, lens=[1, 700, 129, 2049, 64], seed=73)
+    w = inp.workload
+    q, qr, c, kr, lens, pt = to_dev(inp)
+    dims = mlra.dims_for(q, qr, c, kr, lens, pt, 4, max_seq_len=inp.max_seq_len, num_ranges=9)
+    assert mlra.query_plan(dims).ctas == 9 * 4
+    out, lse = run_gpu(inp, num_ranges=9)
+    ref, ref_lse = run_oracle(inp)
+    assert_close(out, ref, "128 heads, 9 ranges")
+    assert_lse_close(lse, ref_lse, "128 heads lse")
+    outs, _ = run_gpu(inp, out_mode="summed")
+    refs, _ = run_oracle(inp, out_mode="summed")
+    assert_close(outs, refs, "128 heads, summed")
+
+
 @pytest.mark.parametrize("name,seqs,heads", [
     ("mla_h128_n8_l32k", [0, 7], [0, 63, 64, 127]),
+    ("mlra4_h128_n8_l32k", [0, 5], [0, 63, 64, 127]),
     ("mlra4_n8_l32k", [0, 5, 7], [0, 17, 33, 63]),
     ("mla_n8_l32k", [1, 6], [2, 40, 63]),
     ("long_mlra4_l128k", [0], [0, 9, 31, 62]),

@@ -106,6 +106,10 @@ WORKLOADS = {
     "mla_h128_n8_l32k": Workload(
         name="mla_h128_n8_l32k", batch=8, heads=128, num_branches=1, d_latent=512, d_rope=64,
         seq_len=32768, seed=1007),
+    # MLRA-4 with 128 heads (both head groups as one 128-row product per cache tile)
+    "mlra4_h128_n8_l32k": Workload(
+        name="mlra4_h128_n8_l32k", batch=8, heads=128, num_branches=4, d_latent=512, d_rope=64,
+        seq_len=32768, seed=1008),
     "serving_mlra4_n64_paged": Workload(
         name="serving_mlra4_n64_paged", batch=64, heads=64, num_branches=4, d_latent=512,
         d_rope=64, seq_len=65536, min_seq_len=1024, ragged=True, page_size=64, seed=1005),
