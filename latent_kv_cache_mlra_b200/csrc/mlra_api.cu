@@ -426,6 +426,10 @@ mlra_status decode_impl(const void* q_lat, const void* q_rope, const void* c_kv,
   // Test hook: with MLRA_TEST_FORCE_REPLAN set in the environment, the attention kernel treats
   // its speculative plan as stale and takes the re-plan path (results are unchanged).
   p.force_replan = std::getenv("MLRA_TEST_FORCE_REPLAN") != nullptr ? 1 : 0;
+  // Test hook: with MLRA_TEST_FORCE_TIMEOUT set, the producer of every CTA that has a copy left
+  // to issue after its speculative ones waits (1 ms) on a barrier nothing arrives at; the call
+  // then reports MLRA_ERR_TIMEOUT and its outputs are undefined.
+  p.force_timeout = std::getenv("MLRA_TEST_FORCE_TIMEOUT") != nullptr ? 1 : 0;
   if (k1_begin && cudaEventRecord(reinterpret_cast<cudaEvent_t>(k1_begin), s) != cudaSuccess)
     return MLRA_ERR_CUDA;
   const cudaError_t launched = pl.m128 ? launch_decode_m128(tq, tqr, tc, tkr, p, grid, s)

@@ -82,7 +82,8 @@ struct DecodeCfg {
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // TMEM address, abort flag, status bits
   static constexpr int OFF_PLAN = OFF_MISC + 16;       // in-kernel plan (self_plan)
   static constexpr int PLAN_BYTES = 16 * kSelfPlanMaxSeqs +     // segment list
-                                    4 * kSelfPlanMaxSeqs + 16;    // lengths, count
+                                    4 * kSelfPlanMaxSeqs + 16;    // lengths, count, stale, hook
+  static constexpr int OFF_HOOK_BAR = OFF_PLAN + 20 * kSelfPlanMaxSeqs + 8;  // force_timeout
   // epilogue staging: one [16 rows x 32 fp32] box per softmax warp, 128-byte swizzled
   static constexpr int OFF_STG = (OFF_PLAN + PLAN_BYTES + 1023) / 1024 * 1024;
   static constexpr int STG_BYTES = 16 * 128;
@@ -93,6 +94,7 @@ struct DecodeCfg {
   static_assert(NSB >= 2 && NSB == NS, "score buffers: one per stage, at least 2");
   static_assert(TB * BOX == CBLK, "P of a tile fills the RoPE block of its stage");
   static_assert(TMEM_USED <= 512, "TMEM budget");
+  static_assert(OFF_HOOK_BAR % 8 == 0 && OFF_HOOK_BAR + 8 <= OFF_PLAN + PLAN_BYTES, "hook barrier");
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
@@ -123,6 +125,23 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, uint64_
     }
   }
   return __all_sync(kFull, ok);
+}
+
+// Test hook (force_timeout): the producer waits, with a short limit, on an mbarrier that nothing
+// arrives at, so that the time-out path runs for real: the status flag, the CTA abort seen by the
+// other warps, the drain of the copies already issued and the release of TMEM.  Returns false.
+__device__ __forceinline__ bool forced_timeout_wait(uint32_t bar, uint64_t timeout_ns,
+                                                    volatile int* abort_flag, uint32_t* status,
+                                                    int lane) {
+  if (lane == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  const bool ok = wait_warp(bar, 0, timeout_ns, abort_flag, status);
+  if (lane == 0) mbar_inval(bar);
+  __syncwarp();
+  return ok;
 }
 
 // First cache row of the 64-position block t (positions [64t, 64t+64)) of sequence s.  Shared by
@@ -522,15 +541,24 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     Segment seg;
     int L = 0;
     int it = 0, nseg = 0;
+    int q_loads = pre_q ? 1 : 0;  // query loads issued so far (for a drain)
     bool ok = true;
     while (ok && walk.next(seg, L)) {
       if (nseg > 0) ok = wait_warp(bar_q_empty, (nseg - 1) & 1, tmo, abort_flag, flags);
       if (!ok) break;
-      if (lane == 0 && !(nseg == 0 && pre_q)) issue_queries(seg.seq);
+      if (!(nseg == 0 && pre_q)) {
+        if (lane == 0) issue_queries(seg.seq);
+        ++q_loads;
+      }
       __syncwarp();
       const int cache_seq = seg.seq / p.q_per_seq;  // whose cache rows (once per segment)
       for (int i = 0; i < seg.ntiles; ++i, ++it) {
         if (nseg == 0 && i < pre_tiles) continue;  // issued before the plan was confirmed
+        if (p.force_timeout) {
+          ok = forced_timeout_wait(smem_u32(smem + C::OFF_HOOK_BAR), tmo >> 10, abort_flag, flags,
+                                   lane);
+          if (!ok) break;
+        }
         if (it == kFirstTiles && pre_tiles == kFirstTiles) {
           // the remaining first stages once tile 0 has landed: every CTA's first tile arrives
           // sooner (fewer bytes ahead of it in the memory queues), so the tensor core starts and
@@ -552,7 +580,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     if (!ok) {
       // Aborting: let the copies already issued land before the CTA can exit.
-      if (nseg > 0) wait_warp(bar_q_full, (nseg - 1) & 1, tmo / 8, abort_flag, flags, false);
+      if (q_loads > 0) wait_warp(bar_q_full, (q_loads - 1) & 1, tmo / 8, abort_flag, flags, false);
       for (int k = (it > NS ? it - NS : 0); k < it; ++k)
         wait_warp(bar_stage_full + 8 * (k % NS), (k / NS) & 1, tmo / 8, abort_flag, flags, false);
     }

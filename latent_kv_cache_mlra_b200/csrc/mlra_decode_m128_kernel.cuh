@@ -75,6 +75,8 @@ struct DecodeM128Cfg {
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_PLAN = OFF_MISC + 16;
   static constexpr int PLAN_BYTES = 16 * kSelfPlanMaxSeqs + 4 * kSelfPlanMaxSeqs + 16;
+  static constexpr int OFF_HOOK_BAR = OFF_PLAN + 20 * kSelfPlanMaxSeqs + 8;  // force_timeout
+  static_assert(OFF_HOOK_BAR % 8 == 0 && OFF_HOOK_BAR + 8 <= OFF_PLAN + PLAN_BYTES, "hook barrier");
   static constexpr int SMEM = OFF_PLAN + PLAN_BYTES;
   static constexpr int SMEM_ALLOC = SMEM + 1024;
   static_assert(P_COL + NP * (T / 2) <= TMEM_COLS, "TMEM budget");
@@ -293,17 +295,26 @@ mlra_decode_m128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     int L = 0;
     int it = 0, nseg = 0;
     int lat_issued = pre_tiles, rope_issued = pre_rope;  // copies issued so far (for a drain)
+    int q_loads = pre_q ? 1 : 0;
     bool ok = true;
     while (ok && walk.next(seg, L)) {
       if (nseg > 0) ok = wait_warp(bar_q_empty, (nseg - 1) & 1, tmo, abort_flag, flags);
       if (!ok) break;
-      if (lane == 0 && !(nseg == 0 && pre_q)) issue_queries(seg.seq);
+      if (!(nseg == 0 && pre_q)) {
+        if (lane == 0) issue_queries(seg.seq);
+        ++q_loads;
+      }
       __syncwarp();
       const int cache_seq = seg.seq / p.q_per_seq;
       for (int i = 0; i < seg.ntiles; ++i, ++it) {
         const bool latent_done = nseg == 0 && i < pre_tiles;  // issued before the plan was
         const bool rope_done = nseg == 0 && i < pre_rope;     // confirmed
         if (latent_done && rope_done) continue;
+        if (p.force_timeout) {
+          ok = forced_timeout_wait(smem_u32(smem + C::OFF_HOOK_BAR), tmo >> 10, abort_flag, flags,
+                                   lane);
+          if (!ok) break;
+        }
         int rows[C::TB];
         tile_rows(cache_seq, seg.tile0 + i, L, flags, rows);
         if (!latent_done) {
@@ -330,7 +341,7 @@ mlra_decode_m128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     }
     if (!ok) {
       // let the copies already issued land before the CTA can exit
-      if (nseg > 0) wait_warp(bar_q_full, (nseg - 1) & 1, tmo / 8, abort_flag, flags, false);
+      if (q_loads > 0) wait_warp(bar_q_full, (q_loads - 1) & 1, tmo / 8, abort_flag, flags, false);
       for (int k = (lat_issued > NS ? lat_issued - NS : 0); k < lat_issued; ++k)
         wait_warp(bar_stage_full + 8 * (k % NS), (k / NS) & 1, tmo / 8, abort_flag, flags, false);
       for (int k = (rope_issued > C::NR ? rope_issued - C::NR : 0); k < rope_issued; ++k)

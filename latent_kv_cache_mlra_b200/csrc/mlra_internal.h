@@ -88,6 +88,7 @@ struct DecodeParams {
   int write_final;            // whole-sequence segments write `out` directly
   int tma_out;                // ... through the out tensor map (d_blk_out % 32 == 0)
   int force_replan;           // test hook: treat the speculative in-kernel plan as stale
+  int force_timeout;          // test hook: the TMA producer's first wait runs out (short limit)
   uint64_t timeout_ns;        // bound on every wait inside the kernel
 };
 
