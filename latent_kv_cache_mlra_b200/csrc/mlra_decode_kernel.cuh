@@ -99,6 +99,18 @@ struct DecodeCfg {
 };
 
 constexpr uint32_t kFull = 0xffffffffu;
+
+// Three-input maximum / minimum (one instruction; a NaN input is ignored, as by fmaxf / fminf).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 constexpr int kFirstTiles = 2;  // tiles issued at once when a CTA starts (the rest after tile 0)
 
 // Warp-collective bounded wait on an mbarrier phase.  Every lane polls; on time-out the
@@ -721,13 +733,13 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
             for (int l = 0; l < C::TB; ++l)
 #pragma unroll
-              for (int k = 0; k < 32; ++k) a[k & 3] = fmaxf(a[k & 3], v[l][k]);
+              for (int k = 0; k < 32; k += 2) a[(k >> 1) & 3] = max3f(a[(k >> 1) & 3], v[l][k], v[l][k + 1]);
             mx = fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])) * sc;
           } else {
 #pragma unroll
             for (int l = 0; l < C::TB; ++l)
 #pragma unroll
-              for (int k = 0; k < 32; ++k) a[k & 3] = fminf(a[k & 3], v[l][k]);
+              for (int k = 0; k < 32; k += 2) a[(k >> 1) & 3] = min3f(a[(k >> 1) & 3], v[l][k], v[l][k + 1]);
             mx = fminf(fminf(a[0], a[1]), fminf(a[2], a[3])) * sc;
           }
         } else {
@@ -798,15 +810,17 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         uint8_t* p_base = stage_ptr + C::NCB * C::CBLK + prow * 128;
         const uint32_t p_slot =
             tmem + ((uint32_t)(32 * warp + 16) << 16) + C::P_COL + (it % NS) * (T / 2);
-        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+        // (pairs of positions through the packed two-lane FMA and add)
+        const float2 mul2 = make_float2(mul, mul), negm2 = make_float2(neg_m, neg_m);
+        float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int l = 0; l < C::TB; ++l) {
           uint32_t pk[16];
 #pragma unroll
           for (int k = 0; k < 32; k += 2) {
-            const float p0 = ex2_approx(fmaf(v[l][k], mul, neg_m));
-            const float p1 = ex2_approx(fmaf(v[l][k + 1], mul, neg_m));
-            sum4[(k >> 1) & 3] += p0 + p1;
+            const float2 x = __ffma2_rn(make_float2(v[l][k], v[l][k + 1]), mul2, negm2);
+            const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+            sum2[(k >> 1) & 1] = __fadd2_rn(sum2[(k >> 1) & 1], make_float2(p0, p1));
             pk[k / 2] = pack_bf16x2(p0, p1);
           }
           if constexpr (C::P_TMEM) {
@@ -822,7 +836,7 @@ mlra_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           tc_fence_before();         // ... after this thread's TMEM accesses (and O rescale)
           mbar_arrive(bar_p_full + 8 * (l * NSB + it % NSB));
         }
-        float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+        float sum = (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
         sum += __shfl_xor_sync(kFull, sum, 16);
         l_sum += sum;
       }

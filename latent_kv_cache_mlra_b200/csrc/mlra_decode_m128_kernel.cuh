@@ -471,11 +471,11 @@ mlra_decode_m128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           float a[4] = {v[0], v[1], v[2], v[3]};
           if (sc >= 0.f) {
 #pragma unroll
-            for (int k = 4; k < 64; ++k) a[k & 3] = fmaxf(a[k & 3], v[k]);
+            for (int k = 4; k < 64; k += 2) a[(k >> 1) & 3] = max3f(a[(k >> 1) & 3], v[k], v[k + 1]);
             mx = fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])) * sc;
           } else {
 #pragma unroll
-            for (int k = 4; k < 64; ++k) a[k & 3] = fminf(a[k & 3], v[k]);
+            for (int k = 4; k < 64; k += 2) a[(k >> 1) & 3] = min3f(a[(k >> 1) & 3], v[k], v[k + 1]);
             mx = fminf(fminf(a[0], a[1]), fminf(a[2], a[3])) * sc;
           }
         } else {
@@ -537,16 +537,17 @@ mlra_decode_m128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         // P slot, released half k by half k
         const float mul = whole ? sc : 1.f;
         const float neg_m = m_used == -CUDART_INF_F ? 0.f : -m_used;
-        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+        const float2 mul2 = make_float2(mul, mul), negm2 = make_float2(neg_m, neg_m);
+        float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         const uint32_t pslot = tmem + lane_base + C::P_COL + (it % C::NP) * (T / 2);
 #pragma unroll
         for (int kb = 0; kb < 2; ++kb) {
           uint32_t pk[16];
 #pragma unroll
-          for (int k = 0; k < 32; k += 2) {
-            const float p0 = ex2_approx(fmaf(v[32 * kb + k], mul, neg_m));
-            const float p1 = ex2_approx(fmaf(v[32 * kb + k + 1], mul, neg_m));
-            sum4[(k >> 1) & 3] += p0 + p1;
+          for (int k = 0; k < 32; k += 2) {  // pairs through the packed two-lane FMA and add
+            const float2 x = __ffma2_rn(make_float2(v[32 * kb + k], v[32 * kb + k + 1]), mul2, negm2);
+            const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+            sum2[(k >> 1) & 1] = __fadd2_rn(sum2[(k >> 1) & 1], make_float2(p0, p1));
             pk[k / 2] = pack_bf16x2(p0, p1);
           }
           tmem_st16x2_16(pslot + 32 * kb, pk);
@@ -554,7 +555,7 @@ mlra_decode_m128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           tc_fence_before();
           mbar_arrive(bar_p_full + 8 * (kb * C::NP + it % C::NP));
         }
-        l_sum += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+        l_sum += (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
       }
       if (!ok) break;
       // ------------------------------------------------ epilogue of the segment
