@@ -103,3 +103,23 @@ def test_m128_timeout_path(q_len, heads, lens, monkeypatch):
                                num_ranges=RANGES)
 
     forced_then_normal(call, ws, monkeypatch)
+
+
+def test_decode_project_timeout_path(monkeypatch):
+    """Steps 2 and 3 in one call: the step-3 product folds the attention CTAs' status bits into the
+    call's status word, so a time-out inside the attention kernel reaches the caller there too."""
+    inp = inputs([2000, 700, 1300], seed=75)
+    w = inp.workload
+    q, qr, c, kr, sl, pt = to_dev(inp)
+    g = torch.Generator().manual_seed(76)
+    w_uv = (torch.randn(w.heads, 128, 512, generator=g) / 512 ** 0.5).to(torch.bfloat16).cuda()
+    wp = mlra.pack_wuv(w_uv)
+    dims = mlra.dims_for(q, qr, c, kr, sl, pt, 4, max_seq_len=inp.max_seq_len, num_ranges=RANGES)
+    ws = torch.zeros(mlra.workspace_size_project(dims), dtype=torch.uint8, device="cuda")
+
+    def call():
+        return (mlra.decode_project(q, qr, c, kr, sl, pt, wp, num_branches=4, softmax_scale=w.sigma,
+                                    branch_scale=w.gamma, max_seq_len=inp.max_seq_len,
+                                    num_ranges=RANGES, workspace=ws),)
+
+    forced_then_normal(call, ws, monkeypatch)
