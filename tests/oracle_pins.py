@@ -200,6 +200,24 @@ def pin_closed_forms(orc, seed=5):
     assert np.allclose(ls - lb, 800.0, rtol=0, atol=1e-9), "lse shifts by sigma * 1000"
 
 
+def pin_scale_sign(orc, seed=13, H=4, B=4, d_c=16, d_R=4, L=21):
+    """The softmax scale's sign: a negative scale equals the positive one applied to the negated
+    query (both parts), output and log-sum-exp; a zero scale gives uniform weights (the mean of
+    each branch block, lse = log L) whatever the query."""
+    rng = np.random.default_rng(seed)
+    q_lat, q_rope = _rand(rng, H, d_c), _rand(rng, H, d_R)
+    c, kr = _rand(rng, L, d_c), _rand(rng, L, d_R)
+    neg, lneg = _one_seq(orc, q_lat, q_rope, c, kr, B, -0.7, 0.5)
+    flip, lflip = _one_seq(orc, -q_lat, -q_rope, c, kr, B, 0.7, 0.5)
+    assert np.allclose(neg, flip, rtol=0, atol=1e-14), "negative scale = negated query"
+    assert np.allclose(lneg, lflip, rtol=0, atol=1e-13), "negative scale lse"
+    pos, _ = _one_seq(orc, q_lat, q_rope, c, kr, B, 0.7, 0.5)
+    assert not np.allclose(neg, pos, rtol=0, atol=1e-6), "the sign matters"
+    zero, lz = _one_seq(orc, q_lat, q_rope, c, kr, B, 0.0, 0.5)
+    assert np.allclose(zero, 0.5 * c.mean(0)[None], rtol=0, atol=1e-14), "zero scale: mean"
+    assert np.allclose(lz, math.log(L), rtol=0, atol=1e-13), "zero scale: lse = log L"
+
+
 def pin_branch_independence(orc, seed=6, H=5, B=4, d_c=32, d_R=8, L=31):
     """Changing block b' of the latent leaves every other branch's output bit-identical."""
     rng = np.random.default_rng(seed)
@@ -470,6 +488,7 @@ ALL_PINS = [
     pin_brute_force,
     pin_probabilities,
     pin_closed_forms,
+    pin_scale_sign,
     pin_branch_independence,
     pin_position_permutation,
     pin_batch_rows_and_paging,
