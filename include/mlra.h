@@ -69,7 +69,15 @@ typedef enum {
 typedef enum { MLRA_BF16 = 0, MLRA_F32 = 1 } mlra_dtype;
 typedef enum { MLRA_OUT_BRANCHES = 0, MLRA_OUT_SUMMED = 1 } mlra_out_mode;
 
-/* Device status bits (mlra_read_status). */
+/* Device status bits (mlra_read_status).
+ *
+ * Test hooks, read from the environment at every decode call (unset in normal use):
+ *   MLRA_TEST_FORCE_REPLAN   the attention kernel treats its speculative work plan as stale and
+ *                            re-plans after its dependency wait; results are unchanged.
+ *   MLRA_TEST_FORCE_TIMEOUT  each attention CTA with a copy left to issue after its speculative
+ *                            ones waits 1 ms on a barrier nothing completes, so the call reports
+ *                            MLRA_ERR_TIMEOUT / MLRA_FLAG_TIMEOUT; its outputs are undefined and
+ *                            the next call on the same workspace is unaffected. */
 #define MLRA_FLAG_TIMEOUT 0x1u
 #define MLRA_FLAG_BAD_PAGE 0x2u
 #define MLRA_FLAG_BAD_LENGTH 0x4u
