@@ -353,3 +353,19 @@ def test_replan_path(B, paged, monkeypatch):
     assert_close(out, ref, f"re-plan B={B} paged={paged}")
     assert_lse_close(lse, ref_lse, "re-plan lse")
     assert torch.equal(out, base) and torch.equal(lse, base_lse)
+
+
+@pytest.mark.parametrize("page_size", [0, 64])
+def test_large_batch(page_size):
+    """700 short ragged sequences (some empty): the prep kernel's plan over many sequences, and
+    work ranges that each run through about twenty segments (a query load and an epilogue each)."""
+    g = torch.Generator().manual_seed(41)
+    lens = torch.randint(0, 160, (700,), generator=g)
+    lens[::97] = 0
+    inp = small_inputs(B=4, lens=lens.tolist(), page_size=page_size, seed=42)
+    out, lse = run_gpu(inp)
+    ref, ref_lse = run_oracle(inp)
+    empty = (lens == 0).nonzero().flatten()
+    assert (out[empty] == 0).all() and torch.isneginf(lse[empty]).all()
+    assert_close(out, ref, f"N=700 paged={page_size}")
+    assert_lse_close(lse, ref_lse, f"N=700 paged={page_size} lse")
