@@ -152,3 +152,18 @@ def test_two_tokens_per_cta_through_the_prep_kernel():
     assert torch.count_nonzero(out[5]) == 0
     assert_close(out, ref, "80 units")
     assert_lse_close(lse, ref_lse, "80 units lse")
+
+
+def test_two_token_units_through_the_prep_kernel():
+    """100 sequences x 2 tokens with 64 heads and 128-wide branches: 100 two-token units, more than
+    the attention kernel plans itself, so the 128-row kernel reads the prep kernel's plan."""
+    g = torch.Generator().manual_seed(93)
+    lens = torch.randint(2, 300, (100,), generator=g).tolist()
+    w, inp, q_lat, q_rope = multi_inputs(2, lens, B=4, heads=64, d_latent=512, page_size=64, seed=94)
+    out, lse = run_multi(w, inp, q_lat, q_rope)
+    torch.cuda.synchronize()
+    ref, ref_lse = oracle.decode_multi(q_lat, q_rope, inp.c_kv, inp.k_rope, inp.seq_lens,
+                                       inp.page_table, w.num_branches, w.sigma, w.gamma,
+                                       page_size=64, max_seq_len=inp.max_seq_len)
+    assert_close(out, ref, "100 two-token units")
+    assert_lse_close(lse, ref_lse, "100 two-token units lse")

@@ -369,3 +369,15 @@ def test_large_batch(page_size):
     assert (out[empty] == 0).all() and torch.isneginf(lse[empty]).all()
     assert_close(out, ref, f"N=700 paged={page_size}")
     assert_lse_close(lse, ref_lse, f"N=700 paged={page_size} lse")
+
+
+def test_128_heads_through_the_prep_kernel():
+    """80 sequences with 128 heads: the 128-row kernel (all heads of a branch in one CTA) reading the
+    prep kernel's plan."""
+    g = torch.Generator().manual_seed(43)
+    lens = torch.randint(0, 400, (80,), generator=g).tolist()
+    inp = small_inputs(B=4, heads=128, lens=lens, page_size=64, seed=44)
+    out, lse = run_gpu(inp)
+    ref, ref_lse = run_oracle(inp)
+    assert_close(out, ref, "H=128, N=80")
+    assert_lse_close(lse, ref_lse, "H=128, N=80 lse")
