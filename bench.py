@@ -24,7 +24,6 @@ import statistics
 import sys
 import threading
 import time
-import time
 
 ROOT = pathlib.Path(__file__).resolve().parent
 sys.path.insert(0, str(ROOT))
