@@ -1,5 +1,5 @@
-// mlra_merge.cuh -- merging the partial softmax states of a split sequence, shared by the decode
-// kernel (in-kernel merge) and the combine kernel.
+// mlra_merge.cuh -- merging the partial softmax states of a split sequence, shared by the combine
+// kernel and the step-3 product kernel that merges while it stages its input.
 //
 // A part p of (sequence, head, branch) holds m_p (running maximum of the scaled scores, log2
 // units), l_p = sum_j 2^(s_j - m_p) and the unnormalised output o_p = sum_j 2^(s_j - m_p) c_j.
