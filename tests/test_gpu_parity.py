@@ -381,3 +381,16 @@ def test_128_heads_through_the_prep_kernel():
     ref, ref_lse = run_oracle(inp)
     assert_close(out, ref, "H=128, N=80")
     assert_lse_close(lse, ref_lse, "H=128, N=80 lse")
+
+
+def test_plan_in_workspace_scratch():
+    """2600 sequences: past the 2400 whose plan the prep kernel keeps in shared memory, so its
+    prefixes and part ranges live in the workspace instead."""
+    g = torch.Generator().manual_seed(45)
+    lens = torch.randint(0, 40, (2600,), generator=g)
+    lens[::50] = 0
+    inp = small_inputs(B=4, heads=8, lens=lens.tolist(), seed=46)
+    out, lse = run_gpu(inp)
+    ref, ref_lse = run_oracle(inp)
+    assert_close(out, ref, "N=2600")
+    assert_lse_close(lse, ref_lse, "N=2600 lse")
